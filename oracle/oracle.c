@@ -1,0 +1,260 @@
+/*
+ * CPU oracle for the MoE layer's plan -> dispatch -> grouped SwiGLU FFN -> combine.
+ *
+ * TEST INFRASTRUCTURE ONLY. The tests, the package's smoke check and the CPU
+ * baseline leg of the benchmark call this file; the product path never does,
+ * and it shares no code, header, table or helper with the CUDA library.
+ *
+ * It is plain and slow on purpose: integer work is written as its definition,
+ * floating point is computed in double from the bf16 / fp32 inputs with no
+ * intermediate rounding, and nothing is blocked, fused or reordered beyond what
+ * each definition states (sums run over their index in ascending order).
+ *
+ * Source of each definition: the StreamEP README ("How it works"):
+ *   - "Pool-layout dispatch": routed (token, k) pairs land in an expert-major,
+ *     tile-padded pool, so dispatch's output is the grouped GEMM input.
+ *     -> oracle_plan, oracle_pool
+ *   - "CuTeDSL compute kernels": forward grouped GEMMs A (up/gate) and Y (down)
+ *     over the pool; the expert function is the SwiGLU FFN
+ *     W2 (silu(x W1_gate) * (x W1_up)).
+ *     -> oracle_expert_ffn, oracle_moe_forward
+ *   - "Per-tile streaming" / combine: each token's output is the routing-weighted
+ *     sum of its k expert outputs. -> oracle_combine, oracle_moe_forward
+ * Readings where the README is silent (each one also listed in the design notes):
+ *   - order inside an expert's pool segment: flat pair id f = t*k + j ascending;
+ *   - W1[e] is [H, 2I]: columns [0, I) gate, [I, 2I) up (concatenated);
+ *   - padding rows of the pool are all-zero;
+ *   - topk_idx == -1 marks a dropped pair (no pool row, no contribution);
+ *     any other index outside [0, E) is an error;
+ *   - silu(v) = v / (1 + exp(-v)).
+ *
+ * Pins (tests/test_oracle_pins.py): a hand-worked example, a stable-sort brute
+ * force of the plan, invariants, a dense all-experts brute force of the layer,
+ * the E=1/k=1 textbook SwiGLU FFN against torch float64 matmuls, closed forms
+ * (identity-like W1/W2, identity experts), linearity and permutation
+ * equivariance, plus planted-mistake variants of this file that must fail them.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG (-1)
+#define ORACLE_ERR_MISSING_EXPERT (-2)
+#define ORACLE_ERR_BAD_INDEX (-10)
+
+/* bf16 bit pattern -> double. Exact: bf16 is the top half of an fp32. */
+static double bf16_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+/* Dropless bound on the pool rows: every real pair, plus at most tile-1 padding
+ * rows for each expert that receives at least one pair. */
+int64_t oracle_pool_rows_max(int64_t T, int32_t k, int32_t E, int32_t tile) {
+  int64_t pairs = T * (int64_t)k;
+  int64_t nonempty = pairs < (int64_t)E ? pairs : (int64_t)E;
+  return round_up(pairs + nonempty * (int64_t)(tile - 1), tile);
+}
+
+/*
+ * Routing plan (StreamEP README, How it works, "Pool-layout dispatch").
+ *   counts[e]      = #{ f : topk_idx[f] == e }
+ *   offsets[0] = 0, offsets[e+1] = offsets[e] + ceil(counts[e]/tile)*tile
+ *   P              = offsets[E]
+ *   pool_row[f]    = offsets[e] + (number of f' < f with topk_idx[f'] == e),
+ *                    or -1 for a dropped pair (topk_idx[f] == -1)
+ *   row_src[p]     = the f with pool_row[f] == p, or -1 for a padding row
+ *                    (rows [P, row_src_len) are -1 as well)
+ *   tile_expert[i] = e for the pool tile i = p / tile of rows p in
+ *                    [offsets[e], offsets[e+1]); -1 for tiles at or past P/tile
+ * Returns ORACLE_ERR_BAD_INDEX if any index is outside [-1, E).
+ */
+int oracle_plan(int64_t T, int32_t k, int32_t E, int32_t tile, const int32_t *topk_idx,
+                int32_t *counts, int32_t *offsets, int32_t *pool_row, int32_t *row_src,
+                int64_t row_src_len, int32_t *tile_expert, int64_t tile_expert_len,
+                int64_t *P_out) {
+  if (T < 0 || k <= 0 || E <= 0 || tile <= 0) return ORACLE_ERR_ARG;
+  int64_t pairs = T * (int64_t)k;
+  for (int64_t f = 0; f < pairs; ++f) {
+    int32_t e = topk_idx[f];
+    if (e < -1 || e >= E) return ORACLE_ERR_BAD_INDEX;
+  }
+  for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t f = 0; f < pairs; ++f)
+    if (topk_idx[f] >= 0) counts[topk_idx[f]] += 1;
+  offsets[0] = 0;
+  for (int32_t e = 0; e < E; ++e)
+    offsets[e + 1] = offsets[e] + (int32_t)round_up(counts[e], tile);
+  int64_t P = offsets[E];
+  if (P > row_src_len || P / tile > tile_expert_len) return ORACLE_ERR_ARG;
+
+  for (int64_t p = 0; p < row_src_len; ++p) row_src[p] = -1;
+  int32_t *seen = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+  if (!seen) return ORACLE_ERR_ARG;
+  for (int64_t f = 0; f < pairs; ++f) {
+    int32_t e = topk_idx[f];
+    if (e < 0) {
+      pool_row[f] = -1;
+      continue;
+    }
+    int32_t p = offsets[e] + seen[e];
+    seen[e] += 1;
+    pool_row[f] = p;
+    row_src[p] = (int32_t)f;
+  }
+  free(seen);
+  for (int64_t i = 0; i < tile_expert_len; ++i) tile_expert[i] = -1;
+  for (int32_t e = 0; e < E; ++e)
+    for (int64_t p = offsets[e]; p < offsets[e + 1]; p += tile) tile_expert[p / tile] = e;
+  *P_out = P;
+  return ORACLE_OK;
+}
+
+/*
+ * Dispatched pool (StreamEP README, How it works, "Pool-layout dispatch"):
+ * row p holds x[row_src[p] / k] for a real row and zeros for a padding row.
+ * Bit copy of the bf16 patterns.
+ */
+void oracle_pool(int64_t P, int32_t H, int32_t k, const int32_t *row_src, const uint16_t *x,
+                 uint16_t *pool) {
+  for (int64_t p = 0; p < P; ++p) {
+    int32_t f = row_src[p];
+    for (int32_t h = 0; h < H; ++h)
+      pool[p * H + h] = (f >= 0) ? x[(int64_t)(f / k) * H + h] : (uint16_t)0;
+  }
+}
+
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+/*
+ * One expert applied to one token row (StreamEP README, How it works,
+ * "CuTeDSL compute kernels": GEMM A then GEMM Y), in double:
+ *   g[n] = sum_h x[h] * W1e[h][n]          n in [0, I)   (gate)
+ *   u[n] = sum_h x[h] * W1e[h][I + n]                     (up)
+ *   a[n] = silu(g[n]) * u[n]
+ *   z[m] = sum_n a[n] * W2e[n][m]          m in [0, H)
+ * W1e is [H, 2I] row-major, W2e is [I, H] row-major. Scratch: g, u, a of I doubles.
+ */
+void oracle_expert_ffn(int32_t H, int32_t I, const uint16_t *x_row, const uint16_t *W1e,
+                       const uint16_t *W2e, double *g, double *u, double *a, double *z) {
+  const int64_t two_i = 2 * (int64_t)I;
+  for (int32_t n = 0; n < I; ++n) {
+    g[n] = 0.0;
+    u[n] = 0.0;
+  }
+  /* h outer so that W1e streams row by row; each g[n], u[n] still sums h ascending. */
+  for (int32_t h = 0; h < H; ++h) {
+    double xh = bf16_to_double(x_row[h]);
+    const uint16_t *w = W1e + (int64_t)h * two_i;
+    for (int32_t n = 0; n < I; ++n) {
+      g[n] += xh * bf16_to_double(w[n]);
+      u[n] += xh * bf16_to_double(w[I + n]);
+    }
+  }
+  for (int32_t n = 0; n < I; ++n) a[n] = silu(g[n]) * u[n];
+  for (int32_t m = 0; m < H; ++m) z[m] = 0.0;
+  /* n outer: each z[m] sums n ascending. */
+  for (int32_t n = 0; n < I; ++n) {
+    const uint16_t *w = W2e + (int64_t)n * H;
+    for (int32_t m = 0; m < H; ++m) z[m] += a[n] * bf16_to_double(w[m]);
+  }
+}
+
+/*
+ * The layer for a list of tokens, straight from x (never through a pool):
+ *   y[t][m] = sum_{j < k, e = topk_idx[t][j] >= 0} w[t][j] * z_{t,j}[m]
+ * with z_{t,j} = oracle_expert_ffn(x[t], W1[e], W2[e]); j ascending.
+ * x_rows [n, H] bf16, idx_rows / w_rows [n, k], W1 / W2: E pointers to one
+ * expert's matrix each (NULL allowed for experts no listed token uses).
+ * y [n, H] double. Tokens are independent and run on up to n_threads threads.
+ */
+int oracle_moe_forward(int64_t n, int32_t H, int32_t I, int32_t E, int32_t k,
+                       const uint16_t *x_rows, const int32_t *idx_rows, const float *w_rows,
+                       const uint16_t *const *W1, const uint16_t *const *W2, double *y,
+                       int n_threads) {
+  if (n < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return ORACLE_ERR_ARG;
+  for (int64_t f = 0; f < n * k; ++f) {
+    int32_t e = idx_rows[f];
+    if (e < -1 || e >= E) return ORACLE_ERR_BAD_INDEX;
+    if (e >= 0 && (!W1[e] || !W2[e])) return ORACLE_ERR_MISSING_EXPERT;
+  }
+  int err = 0;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+  {
+    double *g = (double *)malloc(sizeof(double) * (size_t)I);
+    double *u = (double *)malloc(sizeof(double) * (size_t)I);
+    double *a = (double *)malloc(sizeof(double) * (size_t)I);
+    double *z = (double *)malloc(sizeof(double) * (size_t)H);
+    if (!g || !u || !a || !z) {
+#pragma omp atomic write
+      err = 1;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < n; ++t) {
+      if (!g || !u || !a || !z) continue;
+      double *yt = y + t * H;
+      for (int32_t m = 0; m < H; ++m) yt[m] = 0.0;
+      for (int32_t j = 0; j < k; ++j) {
+        int32_t e = idx_rows[t * k + j];
+        if (e < 0) continue;
+        double w = (double)w_rows[t * k + j];
+        oracle_expert_ffn(H, I, x_rows + t * H, W1[e], W2[e], g, u, a, z);
+        for (int32_t m = 0; m < H; ++m) yt[m] += w * z[m];
+      }
+    }
+    free(g);
+    free(u);
+    free(a);
+    free(z);
+  }
+  return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/*
+ * The layer with identity experts (the expert returns its input row):
+ *   y[t][m] = sum_{j < k, topk_idx[t][j] >= 0} w[t][j] * x[t][m]
+ */
+int oracle_moe_forward_identity(int64_t T, int32_t H, int32_t k, const uint16_t *x,
+                                const int32_t *topk_idx, const float *topk_w, double *y) {
+  if (T < 0 || H <= 0 || k <= 0) return ORACLE_ERR_ARG;
+  for (int64_t t = 0; t < T; ++t) {
+    for (int32_t m = 0; m < H; ++m) {
+      double acc = 0.0;
+      for (int32_t j = 0; j < k; ++j)
+        if (topk_idx[t * k + j] >= 0)
+          acc += (double)topk_w[t * k + j] * bf16_to_double(x[t * H + m]);
+      y[t * H + m] = acc;
+    }
+  }
+  return ORACLE_OK;
+}
+
+/*
+ * Combine over a given expert-output pool (StreamEP README, How it works,
+ * "Per-tile streaming": combine sends each token once its compute is done):
+ *   y[t][m] = sum_{j < k, pool_row[t*k+j] >= 0} w[t][j] * ypool[pool_row[t*k+j]][m]
+ * ypool [*, H] bf16; y [T, H] double.
+ */
+int oracle_combine(int64_t T, int32_t H, int32_t k, const int32_t *pool_row,
+                   const float *topk_w, const uint16_t *ypool, double *y) {
+  if (T < 0 || H <= 0 || k <= 0) return ORACLE_ERR_ARG;
+  for (int64_t t = 0; t < T; ++t) {
+    for (int32_t m = 0; m < H; ++m) {
+      double acc = 0.0;
+      for (int32_t j = 0; j < k; ++j) {
+        int32_t p = pool_row[t * k + j];
+        if (p < 0) continue;
+        acc += (double)topk_w[t * k + j] * bf16_to_double(ypool[(int64_t)p * H + m]);
+      }
+      y[t * H + m] = acc;
+    }
+  }
+  return ORACLE_OK;
+}
