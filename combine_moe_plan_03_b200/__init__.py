@@ -1,0 +1,205 @@
+"""B200 (sm_100a) MoE layer hot path: plan -> dispatch -> grouped SwiGLU FFN -> combine.
+
+Thin ctypes binding of ``libmoe.so`` (declared in ``include/moe.h``). Every
+function here only marshals arguments; all of the layer's work runs in the CUDA
+kernels of ``csrc/``. Tensor arguments are device pointers (ints, e.g.
+``tensor.data_ptr()``) and streams/events are raw handles (``stream.cuda_stream``).
+Importing fails loudly when the library has not been built: there is no
+fallback path.
+
+Method: StreamEP README, "How it works" (pool-layout dispatch into an
+expert-major tile-padded pool, per-tile streaming flags, caller-owned compute and
+communicate streams, grouped GEMMs A / Y).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED_SHAPE = -2
+MOE_ERR_MISALIGNED = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_NO_DEVICE = -5
+MOE_ERR_BAD_INDEX = -10
+MOE_ERR_FLAG_TIMEOUT = -11
+MOE_ERR_POOL_OVERFLOW = -12
+MOE_ERR_PIPE_TIMEOUT = -13
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("tile", ctypes.c_int32)]
+
+
+class moe_plan_buffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "counts", "offsets", "pool_row", "row_src", "tile_expert", "mblk", "meta",
+        "tile_flags", "workspace", "status")]
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("streaming", ctypes.c_int32), ("ffn_ctas", ctypes.c_int32),
+                ("wait_timeout_us", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {moe_strerror(code)} ({code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libmoe.so is not built ({LIB_PATH}); run combine_moe_plan_03_b200/build.py "
+            "or __graft_entry__.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    sig = {
+        "moe_pool_rows_max": [P(moe_shape), P(ctypes.c_int64)],
+        "moe_plan_arena_bytes": [P(moe_shape), P(ctypes.c_size_t)],
+        "moe_plan_bind": [P(moe_shape), vp, P(moe_plan_buffers)],
+        "moe_plan": [P(moe_shape), vp, P(moe_plan_buffers), vp, vp],
+        "moe_dispatch": [P(moe_shape), vp, P(moe_plan_buffers), vp, i32, vp],
+        "moe_grouped_ffn": [P(moe_shape), vp, vp, vp, P(moe_plan_buffers), vp, vp,
+                            P(moe_config), vp],
+        "moe_combine": [P(moe_shape), vp, vp, P(moe_plan_buffers), vp, vp],
+        "moe_forward": [P(moe_shape), vp, vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp,
+                        P(moe_config), vp, vp, vp, vp],
+        "moe_events_create": [P(vp), i32],
+        "moe_events_destroy": [P(vp), i32],
+        "moe_get_status": [P(moe_plan_buffers), P(i32), P(i32)],
+        "moe_clear_status": [P(moe_plan_buffers), vp],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.moe_strerror.argtypes = [ctypes.c_int]
+    L.moe_strerror.restype = ctypes.c_char_p
+    L.moe_version.argtypes = []
+    L.moe_version.restype = ctypes.c_char_p
+    return L
+
+
+_lib = _load()
+
+# Names exported by include/moe.h, in declaration order.
+EXPORTS = ["moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
+           "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_events_create",
+           "moe_events_destroy", "moe_get_status", "moe_clear_status", "moe_strerror",
+           "moe_version"]
+
+
+def lib():
+    return _lib
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoEError(fn, rc)
+
+
+def _shape(s) -> moe_shape:
+    if isinstance(s, moe_shape):
+        return s
+    return moe_shape(int(s.T), int(s.H), int(s.I), int(s.E), int(s.k), int(s.tile))
+
+
+def moe_strerror(code: int) -> str:
+    return _lib.moe_strerror(int(code)).decode()
+
+
+def moe_version() -> str:
+    return _lib.moe_version().decode()
+
+
+def moe_pool_rows_max(shape) -> int:
+    out = ctypes.c_int64(0)
+    _check("moe_pool_rows_max", _lib.moe_pool_rows_max(ctypes.byref(_shape(shape)),
+                                                       ctypes.byref(out)))
+    return int(out.value)
+
+
+def moe_plan_arena_bytes(shape) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moe_plan_arena_bytes", _lib.moe_plan_arena_bytes(ctypes.byref(_shape(shape)),
+                                                             ctypes.byref(out)))
+    return int(out.value)
+
+
+def moe_plan_bind(shape, arena_ptr: int) -> moe_plan_buffers:
+    p = moe_plan_buffers()
+    _check("moe_plan_bind", _lib.moe_plan_bind(ctypes.byref(_shape(shape)), arena_ptr,
+                                               ctypes.byref(p)))
+    return p
+
+
+def moe_plan(shape, topk_idx_ptr: int, plan: moe_plan_buffers, host_P_ptr: int = 0,
+             stream: int = 0) -> None:
+    _check("moe_plan", _lib.moe_plan(ctypes.byref(_shape(shape)), topk_idx_ptr,
+                                     ctypes.byref(plan), host_P_ptr or None, stream or None))
+
+
+def moe_dispatch(shape, x_ptr: int, plan: moe_plan_buffers, pool_ptr: int,
+                 signal_flags: bool = False, stream: int = 0) -> None:
+    _check("moe_dispatch", _lib.moe_dispatch(ctypes.byref(_shape(shape)), x_ptr,
+                                             ctypes.byref(plan), pool_ptr, int(signal_flags),
+                                             stream or None))
+
+
+def moe_grouped_ffn(shape, pool_ptr: int, w1_ptr: int, w2_ptr: int, plan: moe_plan_buffers,
+                    act_ptr: int, ypool_ptr: int, cfg: moe_config | None = None,
+                    stream: int = 0) -> None:
+    cfg = cfg or moe_config()
+    _check("moe_grouped_ffn", _lib.moe_grouped_ffn(ctypes.byref(_shape(shape)), pool_ptr, w1_ptr,
+                                                   w2_ptr, ctypes.byref(plan), act_ptr, ypool_ptr,
+                                                   ctypes.byref(cfg), stream or None))
+
+
+def moe_combine(shape, ypool_ptr: int, topk_w_ptr: int, plan: moe_plan_buffers, out_ptr: int,
+                stream: int = 0) -> None:
+    _check("moe_combine", _lib.moe_combine(ctypes.byref(_shape(shape)), ypool_ptr, topk_w_ptr,
+                                           ctypes.byref(plan), out_ptr, stream or None))
+
+
+def moe_forward(shape, x_ptr: int, topk_idx_ptr: int, topk_w_ptr: int, w1_ptr: int, w2_ptr: int,
+                plan: moe_plan_buffers, pool_ptr: int, act_ptr: int, ypool_ptr: int, out_ptr: int,
+                cfg: moe_config | None, comm_stream: int, compute_stream: int, ev_plan: int,
+                ev_dispatch: int) -> None:
+    cfg = cfg or moe_config()
+    _check("moe_forward", _lib.moe_forward(
+        ctypes.byref(_shape(shape)), x_ptr, topk_idx_ptr, topk_w_ptr, w1_ptr or None,
+        w2_ptr or None, ctypes.byref(plan), pool_ptr, act_ptr or None, ypool_ptr or None, out_ptr,
+        ctypes.byref(cfg), comm_stream or None, compute_stream or None, ev_plan, ev_dispatch))
+
+
+def moe_events_create(n: int) -> list[int]:
+    arr = (ctypes.c_void_p * n)()
+    _check("moe_events_create", _lib.moe_events_create(arr, n))
+    return [int(a) for a in arr]
+
+
+def moe_events_destroy(events: list[int]) -> None:
+    arr = (ctypes.c_void_p * len(events))(*events)
+    _check("moe_events_destroy", _lib.moe_events_destroy(arr, len(events)))
+
+
+def moe_get_status(plan: moe_plan_buffers) -> tuple[int, int]:
+    code, aux = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("moe_get_status", _lib.moe_get_status(ctypes.byref(plan), ctypes.byref(code),
+                                                 ctypes.byref(aux)))
+    return int(code.value), int(aux.value)
+
+
+def moe_clear_status(plan: moe_plan_buffers, stream: int = 0) -> None:
+    _check("moe_clear_status", _lib.moe_clear_status(ctypes.byref(plan), stream or None))
+
+
+from .layer import MoELayerBuffers  # noqa: E402  (torch-allocated buffers for one shape)

@@ -1,0 +1,274 @@
+// C ABI of libmoe.so (declared in include/moe.h): argument checks, plan arena
+// layout, and the ordering of the layer's kernels on the caller's communicate
+// and compute streams (StreamEP README, How it works, "Caller-owned streams").
+#include <string.h>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+using namespace moe;
+
+namespace {
+
+int sm_count_cached(int *out) {
+  static int counts[64] = {0};
+  static int ok[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (!ok[dev]) {
+    int major = 0, n = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (major != 10) return MOE_ERR_NO_DEVICE;
+    counts[dev] = n;
+    ok[dev] = 1;
+  }
+  *out = counts[dev];
+  return MOE_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(const moe_shape *s, bool need_ffn) {
+  if (s == nullptr) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->H <= 0 || s->E <= 0 || s->k <= 0) return MOE_ERR_INVALID_ARG;
+  if (s->k > kMaxTopK || s->E > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (s->tile != 64 && s->tile != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->H % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (need_ffn && (s->I <= 0 || s->I % 64 != 0)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const PlanGeom g = plan_geom(*s);
+  if (g.pairs > INT32_MAX || g.pmax > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)s->E * s->H > INT32_MAX || (int64_t)s->E * (s->I > 0 ? s->I : 0) > INT32_MAX)
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int check_plan(const moe_plan_buffers *p) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!p->counts || !p->offsets || !p->pool_row || !p->row_src || !p->tile_expert || !p->mblk ||
+      !p->meta || !p->tile_flags || !p->workspace || !p->status)
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// Sizes (in 4-byte words) of the plan buffers, in moe_plan_buffers field order.
+void plan_sizes(const moe_shape &s, size_t words[10]) {
+  const PlanGeom g = plan_geom(s);
+  words[0] = (size_t)s.E;
+  words[1] = (size_t)s.E + 1;
+  words[2] = (size_t)g.pairs;
+  words[3] = (size_t)g.pmax;
+  words[4] = (size_t)g.n_tiles;
+  words[5] = 3 * (size_t)g.n_tiles;
+  words[6] = 4;
+  words[7] = (size_t)g.n_tiles;
+  words[8] = plan_workspace_ints(s);
+  words[9] = 4;
+}
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+int moe_pool_rows_max(const moe_shape *s, int64_t *rows_out) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if (rows_out == nullptr) return MOE_ERR_INVALID_ARG;
+  *rows_out = plan_geom(*s).pmax;
+  return MOE_OK;
+}
+
+int moe_plan_arena_bytes(const moe_shape *s, size_t *bytes_out) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if (bytes_out == nullptr) return MOE_ERR_INVALID_ARG;
+  size_t w[10];
+  plan_sizes(*s, w);
+  size_t total = 0;
+  for (int i = 0; i < 10; ++i) total += round256(w[i] * 4);
+  *bytes_out = total;
+  return MOE_OK;
+}
+
+int moe_plan_bind(const moe_shape *s, void *arena, moe_plan_buffers *out) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if (arena == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(arena) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  size_t w[10];
+  plan_sizes(*s, w);
+  char *base = static_cast<char *>(arena);
+  void *ptrs[10];
+  for (int i = 0; i < 10; ++i) {
+    ptrs[i] = base;
+    base += round256(w[i] * 4);
+  }
+  out->counts = static_cast<int32_t *>(ptrs[0]);
+  out->offsets = static_cast<int32_t *>(ptrs[1]);
+  out->pool_row = static_cast<int32_t *>(ptrs[2]);
+  out->row_src = static_cast<int32_t *>(ptrs[3]);
+  out->tile_expert = static_cast<int32_t *>(ptrs[4]);
+  out->mblk = static_cast<int32_t *>(ptrs[5]);
+  out->meta = static_cast<int32_t *>(ptrs[6]);
+  out->tile_flags = static_cast<uint32_t *>(ptrs[7]);
+  out->workspace = static_cast<int32_t *>(ptrs[8]);
+  out->status = static_cast<int32_t *>(ptrs[9]);
+  return MOE_OK;
+}
+
+int moe_plan(const moe_shape *s, const int32_t *topk_idx, const moe_plan_buffers *p,
+             int32_t *host_P, void *stream) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (topk_idx == nullptr && s->T > 0) return MOE_ERR_INVALID_ARG;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (launch_plan(*s, topk_idx, *p, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (host_P != nullptr) {
+    if (cudaMemcpyAsync(host_P, p->meta + 1, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, void *pool,
+                 int32_t signal_flags, void *stream) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if ((x == nullptr && s->T > 0) || pool == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(pool)) return MOE_ERR_MISALIGNED;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  if (launch_dispatch(*s, x, *p, pool, signal_flags != 0, nsm, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_grouped_ffn(const moe_shape *s, const void *pool, const void *W1, const void *W2,
+                    const moe_plan_buffers *p, void *act, void *ypool, const moe_config *cfg,
+                    void *stream) {
+  int rc = check_shape(s, true);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (!pool || !W1 || !W2 || !act || !ypool) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned16(W1) || !aligned16(W2) || !aligned16(act) ||
+      !aligned16(ypool))
+    return MOE_ERR_MISALIGNED;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  moe_config c{};
+  if (cfg != nullptr) c = *cfg;
+  return launch_ffn(*s, pool, W1, W2, *p, act, ypool, c, nsm, static_cast<cudaStream_t>(stream));
+}
+
+int moe_combine(const moe_shape *s, const void *ypool, const float *topk_w,
+                const moe_plan_buffers *p, void *out, void *stream) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (s->T > 0 && (!ypool || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ypool) || !aligned16(out)) return MOE_ERR_MISALIGNED;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  if (launch_combine(*s, ypool, topk_w, *p, out, nsm, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, const float *topk_w,
+                const void *W1, const void *W2, const moe_plan_buffers *p, void *pool, void *act,
+                void *ypool, void *out, const moe_config *cfg, void *comm_stream,
+                void *compute_stream, void *ev_plan, void *ev_dispatch) {
+  const bool identity = (W1 == nullptr && W2 == nullptr);
+  int rc = check_shape(s, !identity);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (ev_plan == nullptr || ev_dispatch == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((W1 == nullptr) != (W2 == nullptr)) return MOE_ERR_INVALID_ARG;
+  moe_config c{};
+  if (cfg != nullptr) c = *cfg;
+  cudaStream_t comm = static_cast<cudaStream_t>(comm_stream);
+  cudaStream_t comp = static_cast<cudaStream_t>(compute_stream);
+  cudaEvent_t evp = static_cast<cudaEvent_t>(ev_plan);
+  cudaEvent_t evd = static_cast<cudaEvent_t>(ev_dispatch);
+  // The plan buffers and the pool are reused: wait for the previous call's compute work.
+  if (comm != comp) {
+    if (cudaEventRecord(evd, comp) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamWaitEvent(comm, evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if ((rc = moe_plan(s, topk_idx, p, nullptr, comm)) != MOE_OK) return rc;
+  if (cudaEventRecord(evp, comm) != cudaSuccess) return MOE_ERR_CUDA;
+  const int signal = (!identity && c.streaming) ? 1 : 0;
+  if ((rc = moe_dispatch(s, x, p, pool, signal, comm)) != MOE_OK) return rc;
+  if (cudaEventRecord(evd, comm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!identity) {
+    if (cudaStreamWaitEvent(comp, c.streaming ? evp : evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((rc = moe_grouped_ffn(s, pool, W1, W2, p, act, ypool, &c, comp)) != MOE_OK) return rc;
+  }
+  if (cudaStreamWaitEvent(comp, evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
+  return moe_combine(s, identity ? pool : ypool, topk_w, p, out, comp);
+}
+
+int moe_events_create(void **events, int32_t n) {
+  if (events == nullptr || n < 0) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+    events[i] = e;
+  }
+  return MOE_OK;
+}
+
+int moe_events_destroy(void **events, int32_t n) {
+  if (events == nullptr || n < 0) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (events[i] != nullptr) cudaEventDestroy(static_cast<cudaEvent_t>(events[i]));
+  return MOE_OK;
+}
+
+int moe_get_status(const moe_plan_buffers *p, int32_t *code, int32_t *aux) {
+  if (p == nullptr || p->status == nullptr || code == nullptr) return MOE_ERR_INVALID_ARG;
+  int32_t h[2] = {0, 0};
+  if (cudaMemcpy(h, p->status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *code = h[0];
+  if (aux != nullptr) *aux = h[1];
+  return MOE_OK;
+}
+
+int moe_clear_status(const moe_plan_buffers *p, void *stream) {
+  if (p == nullptr || p->status == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(p->status, 0, 4 * sizeof(int32_t), static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+const char *moe_strerror(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (H, I multiples of 64; tile 64 or 128)";
+    case MOE_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_NO_DEVICE: return "current device is not sm_100";
+    case MOE_ERR_BAD_INDEX: return "topk_idx value outside [-1, E)";
+    case MOE_ERR_FLAG_TIMEOUT: return "streaming FFN timed out waiting for a pool tile";
+    case MOE_ERR_POOL_OVERFLOW: return "pool rows exceeded the dropless bound";
+    case MOE_ERR_PIPE_TIMEOUT: return "FFN pipeline wait timed out";
+    default: return "unknown error";
+  }
+}
+
+const char *moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,40 @@
+// Launchers shared between the kernel files and the C ABI (moe_api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Pairs per plan chunk (one warp counts and ranks one chunk) and warps per block.
+constexpr int kPlanChunk = 256;
+constexpr int kPlanWarps = 8;
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kGemmBlockM = 128;
+
+struct PlanGeom {
+  int64_t pairs;     // T * k
+  int64_t pmax;      // dropless pool bound
+  int64_t n_tiles;   // pmax / tile
+  int32_t n_chunks;  // ceil(pairs / kPlanChunk)
+};
+
+PlanGeom plan_geom(const moe_shape &s);
+size_t plan_workspace_ints(const moe_shape &s);
+
+cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_plan_buffers &p,
+                        cudaStream_t st);
+cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_buffers &p,
+                            void *pool, int signal, int num_sms, cudaStream_t st);
+cudaError_t launch_combine(const moe_shape &s, const void *ypool, const float *topk_w,
+                           const moe_plan_buffers &p, void *out, int num_sms, cudaStream_t st);
+// Returns MOE_OK or a MOE_ERR_* code.
+int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void *W2,
+               const moe_plan_buffers &p, void *act, void *ypool, const moe_config &cfg,
+               int num_sms, cudaStream_t st);
+
+}  // namespace moe

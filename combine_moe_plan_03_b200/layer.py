@@ -1,0 +1,86 @@
+"""Device buffers for one MoE layer shape, allocated with torch, used through the C ABI.
+
+PyTorch only provides device memory, streams and events here; every step of the
+layer runs in libmoe's kernels. ``forward`` is the StreamEP ``stream_moe_func``
+call shape (x, topk_idx, topk_weights, w1, w2, streams) on one GPU.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (moe_config, moe_events_create, moe_events_destroy, moe_forward, moe_plan_arena_bytes,
+               moe_plan_bind, moe_pool_rows_max, moe_shape)
+
+_PLAN_FIELDS = ("counts", "offsets", "pool_row", "row_src", "tile_expert", "mblk", "meta",
+                "tile_flags", "workspace", "status")
+
+
+class MoELayerBuffers:
+    """Plan arena, pool, act, ypool and out for shape (T, H, I, E, k, tile), plus the
+    caller-owned communicate / compute streams and the two ordering events."""
+
+    def __init__(self, T: int, H: int, I: int, E: int, k: int, tile: int,
+                 device: str | torch.device = "cuda", identity: bool = False,
+                 streams: tuple[torch.cuda.Stream, torch.cuda.Stream] | None = None):
+        self.shape = moe_shape(T, H, I, E, k, tile)
+        self.device = torch.device(device)
+        self.identity = identity
+        self.P_max = moe_pool_rows_max(self.shape)
+        nbytes = moe_plan_arena_bytes(self.shape)
+        self.arena = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        self.plan = moe_plan_bind(self.shape, self.arena.data_ptr())
+        bf = torch.bfloat16
+        self.pool = torch.empty((max(self.P_max, 1), H), dtype=bf, device=self.device)
+        if identity:
+            self.act = None
+            self.ypool = None
+        else:
+            self.act = torch.empty((max(self.P_max, 1), I), dtype=bf, device=self.device)
+            self.ypool = torch.empty((max(self.P_max, 1), H), dtype=bf, device=self.device)
+        self.out = torch.empty((max(T, 1), H), dtype=bf, device=self.device)
+        if streams is None:
+            streams = (torch.cuda.Stream(self.device), torch.cuda.Stream(self.device))
+        self.comm, self.compute = streams
+        self.events = moe_events_create(2)
+
+    def close(self):
+        if self.events:
+            moe_events_destroy(self.events)
+            self.events = []
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def plan_view(self, name: str) -> torch.Tensor:
+        """int32 view of one plan buffer inside the arena (for inspection and tests)."""
+        ptr = getattr(self.plan, name)
+        off = ptr - self.arena.data_ptr()
+        i = _PLAN_FIELDS.index(name)
+        end = (getattr(self.plan, _PLAN_FIELDS[i + 1]) - self.arena.data_ptr()
+               if i + 1 < len(_PLAN_FIELDS) else self.arena.numel())
+        return self.arena[off:end].view(torch.int32)
+
+    def forward(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
+                W1: torch.Tensor | None, W2: torch.Tensor | None,
+                cfg: moe_config | None = None) -> torch.Tensor:
+        """Enqueue the layer (plan + dispatch on comm, FFN + combine on compute).
+        Returns ``out`` [T, H]; it is ready once the compute stream reaches this point."""
+        s = self.shape
+        assert x.dtype == torch.bfloat16 and tuple(x.shape) == (s.T, s.H) and x.is_contiguous()
+        assert topk_idx.dtype == torch.int32 and tuple(topk_idx.shape) == (s.T, s.k)
+        assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (s.T, s.k)
+        w1 = w2 = act = ypool = 0
+        if not self.identity:
+            assert W1 is not None and W2 is not None
+            assert tuple(W1.shape) == (s.E, s.H, 2 * s.I) and W1.dtype == torch.bfloat16
+            assert tuple(W2.shape) == (s.E, s.I, s.H) and W2.dtype == torch.bfloat16
+            w1, w2 = W1.data_ptr(), W2.data_ptr()
+            act, ypool = self.act.data_ptr(), self.ypool.data_ptr()
+        moe_forward(s, x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), w1, w2, self.plan,
+                    self.pool.data_ptr(), act, ypool, self.out.data_ptr(), cfg,
+                    self.comm.cuda_stream, self.compute.cuda_stream, self.events[0],
+                    self.events[1])
+        return self.out[: s.T]

@@ -1,0 +1,194 @@
+/*
+ * moe.h - C ABI of libmoe.so: the Mixture-of-Experts layer's plan, dispatch,
+ * grouped SwiGLU FFN and combine on one NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the StreamEP README, section "How it works":
+ *   - "Pool-layout dispatch": routed (token, k) pairs land directly in an
+ *     expert-major, tile-padded pool, so dispatch's output is the grouped GEMM's
+ *     input with no separate permute            -> moe_plan, moe_dispatch
+ *   - "Per-tile streaming": dispatch signals each pool tile as it fills and the
+ *     compute kernels claim ready tiles while later tokens are still arriving;
+ *     combine handles a token once its compute is done
+ *                                                -> tile flags, moe_grouped_ffn
+ *                                                   (streaming), moe_combine
+ *   - "Caller-owned streams": the layer runs on a compute stream and a
+ *     communicate stream that the caller supplies; the only host sync is one
+ *     poll that sizes the dropless pool          -> every call takes the stream;
+ *                                                   moe_plan's optional host_P
+ *   - "CuTeDSL compute kernels": the forward grouped GEMMs A (gate/up) and
+ *     Y (down)                                   -> moe_grouped_ffn
+ * and the StreamEP call stream_moe_func(buffer, x, topk_idx, topk_weights, ...,
+ * w1_local, w2_local, streams=...) shown there            -> moe_forward.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument named as a tensor is a DEVICE pointer owned by the
+ *     caller (for example a torch tensor's data_ptr()); the library never
+ *     allocates, frees or keeps device memory, and never synchronises the device
+ *     except in moe_get_status.
+ *   - Streams and events are passed as void* holding a cudaStream_t /
+ *     cudaEvent_t (0 = the legacy default stream). Work is enqueued on the
+ *     given stream; calls return once it is enqueued.
+ *   - Layouts are row-major and dense:
+ *       x       [T, H]      bf16     token activations
+ *       topk_idx[T, k]      int32    expert of pair f = t*k + j; -1 = dropped pair
+ *       topk_w  [T, k]      fp32     routing weight of pair f
+ *       W1      [E, H, 2I]  bf16     per expert: columns [0, I) gate, [I, 2I) up
+ *       W2      [E, I, H]   bf16     per expert down projection
+ *       pool    [P_max, H]  bf16     expert-major, tile-padded dispatched rows
+ *       act     [P_max, I]  bf16     silu(pool W1_gate) * (pool W1_up), per row
+ *       ypool   [P_max, H]  bf16     act W2, per row
+ *       out     [T, H]      bf16     out[t] = sum_j topk_w[t,j] * ypool[pool_row[t,j]]
+ *     with P_max = moe_pool_rows_max(shape). bf16 buffers must be 16-byte
+ *     aligned; H and I must be multiples of 64 (I a multiple of 128 is fastest).
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code, checked on the
+ *     host before anything is launched. Errors found on the device (an expert
+ *     index out of range, a wait that ran out of time) never trap: the first
+ *     one is written to the plan's status word and read with moe_get_status.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes ------------------------------------------------------------------- */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)       /* null pointer, negative size, k > 32, E > 1024 ... */
+#define MOE_ERR_UNSUPPORTED_SHAPE (-2) /* H or I not a multiple of 64, tile not 64 or 128 */
+#define MOE_ERR_MISALIGNED (-3)        /* a tensor pointer not 16-byte aligned */
+#define MOE_ERR_CUDA (-4)              /* a CUDA runtime / driver call failed */
+#define MOE_ERR_NO_DEVICE (-5)         /* current device is not sm_100 */
+/* device-side errors, reported through the status word (moe_get_status) */
+#define MOE_ERR_BAD_INDEX (-10)     /* topk_idx value outside [-1, E); aux = pair id */
+#define MOE_ERR_FLAG_TIMEOUT (-11)  /* streaming FFN gave up waiting on a tile flag; aux = tile */
+#define MOE_ERR_POOL_OVERFLOW (-12) /* plan produced more rows than P_max (cannot happen for valid input) */
+#define MOE_ERR_PIPE_TIMEOUT (-13)  /* an FFN pipeline barrier wait ran out of time; aux = unit */
+
+/* Layer shape. T tokens, hidden H, expert intermediate I, E experts, top-k,
+ * pool tile rows (64 or 128). */
+typedef struct moe_shape {
+  int32_t T, H, I, E, k, tile;
+} moe_shape;
+
+/* Routing plan buffers (device). Carve them from one caller-allocated arena with
+ * moe_plan_bind, or point each field at a buffer of the size moe_plan_bind uses. */
+typedef struct moe_plan_buffers {
+  int32_t *counts;      /* [E]          pairs routed to each expert */
+  int32_t *offsets;     /* [E + 1]      start row of each expert's pool segment; offsets[E] = P */
+  int32_t *pool_row;    /* [T * k]      pool row of pair f, -1 for a dropped pair */
+  int32_t *row_src;     /* [P_max]      pair id of pool row p, -1 for padding */
+  int32_t *tile_expert; /* [P_max/tile] expert of pool tile i, -1 past P/tile */
+  int32_t *mblk;        /* [3 * P_max/tile] GEMM row blocks: {row_start, expert, rows} */
+  int32_t *meta;        /* [4]          num_tiles, P, num_mblk, 0 */
+  uint32_t *tile_flags; /* [P_max/tile] rows landed per tile (streaming) */
+  int32_t *workspace;   /* plan scratch: per-(expert, 256-pair chunk) counts + 1 counter */
+  int32_t *status;      /* [4]          code, aux, 0, 0 (first device error wins) */
+} moe_plan_buffers;
+
+/* FFN launch options (all fields 0 = defaults). */
+typedef struct moe_config {
+  int32_t streaming;       /* 1: the FFN claims pool tiles as their flags fill (dispatch may
+                              still be running on the communicate stream); 0: the caller
+                              orders the FFN after dispatch. */
+  int32_t ffn_ctas;        /* persistent FFN CTAs; 0 = number of SMs (streaming: SMs - 16) */
+  int32_t wait_timeout_us; /* bound on every device-side wait; 0 = 2,000,000 us */
+  int32_t reserved;
+} moe_config;
+
+/* Dropless pool bound: T*k + min(E, T*k)*(tile-1), rounded up to a multiple of tile. */
+int moe_pool_rows_max(const moe_shape *s, int64_t *rows_out);
+
+/* Bytes of the plan arena for this shape (one device allocation, 256-byte aligned). */
+int moe_plan_arena_bytes(const moe_shape *s, size_t *bytes_out);
+
+/* Point the fields of *out into a caller-owned device arena of moe_plan_arena_bytes
+ * bytes. Host-only, no device work. The arena's status word must be zeroed once
+ * by the caller (or with moe_clear_status) before first use. */
+int moe_plan_bind(const moe_shape *s, void *arena, moe_plan_buffers *out);
+
+/*
+ * Routing plan (StreamEP README, How it works, "Pool-layout dispatch").
+ * From topk_idx [T, k] (device int32) computes, on `stream`:
+ *   counts[e], offsets (exclusive prefix of counts padded up to the tile), P,
+ *   pool_row[f] = offsets[e] + rank of f among the pairs of expert e (flat pair id
+ *   ascending: a stable map), row_src (inverse map, -1 for padding), tile_expert,
+ *   the GEMM row-block table mblk, meta, and resets tile_flags to 0.
+ * If host_P is not NULL (pinned host memory), P is copied there asynchronously:
+ * the one poll that sizes the dropless pool. Values outside [-1, E) in topk_idx
+ * give MOE_ERR_BAD_INDEX in the status word and those pairs are dropped.
+ */
+int moe_plan(const moe_shape *s, const int32_t *topk_idx, const moe_plan_buffers *p,
+             int32_t *host_P, void *stream);
+
+/*
+ * Dispatch (StreamEP README, How it works, "Pool-layout dispatch" and "Per-tile
+ * streaming"): pool[pool_row[t*k+j]] = x[t] for every live pair, padding rows of
+ * each expert's segment set to zero, and (signal_flags != 0) tile_flags[p / tile]
+ * incremented with release order once row p has landed. Reads x [T, H], writes
+ * pool [P_max, H] (rows >= P are not touched). Runs after moe_plan on `stream`.
+ */
+int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, void *pool,
+                 int32_t signal_flags, void *stream);
+
+/*
+ * Grouped SwiGLU FFN over the pool (StreamEP README, How it works, "CuTeDSL
+ * compute kernels": grouped GEMM A then grouped GEMM Y), tcgen05 tensor cores:
+ *   act[p]   = bf16( silu(pool[p] W1[e]_gate) * (pool[p] W1[e]_up) )   (fp32 accumulate)
+ *   ypool[p] = bf16( act[p] W2[e] )                                     (fp32 accumulate)
+ * for every row p < P, e = the expert of p's tile. Padding rows give zeros.
+ * With cfg->streaming the first GEMM waits (bounded) until tile_flags[tile] == tile
+ * for each tile it reads, so it may be launched while moe_dispatch is still running
+ * on another stream; otherwise it must be ordered after moe_dispatch.
+ */
+int moe_grouped_ffn(const moe_shape *s, const void *pool, const void *W1, const void *W2,
+                    const moe_plan_buffers *p, void *act, void *ypool, const moe_config *cfg,
+                    void *stream);
+
+/*
+ * Combine (StreamEP README, How it works, "Per-tile streaming": combine of a token
+ * once its compute is done): out[t] = bf16( sum_j topk_w[t,j] * ypool[pool_row[t,j]] ),
+ * an fp32 fused multiply-add chain over j ascending; dropped pairs add nothing.
+ * Pass the pool itself as ypool for identity experts.
+ */
+int moe_combine(const moe_shape *s, const void *ypool, const float *topk_w,
+                const moe_plan_buffers *p, void *out, void *stream);
+
+/*
+ * The whole layer (the StreamEP stream_moe_func call): plan and dispatch on
+ * comm_stream, grouped FFN and combine on compute_stream, ordered with the two
+ * caller-owned events (ev_plan, ev_dispatch; create them with moe_events_create).
+ * W1 == NULL and W2 == NULL selects identity experts (combine reads the pool;
+ * act and ypool are not used). compute_stream waits for the previous work on
+ * comm_stream, and comm_stream for the previous work on compute_stream, so calls
+ * may be issued back to back with the same buffers.
+ */
+int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, const float *topk_w,
+                const void *W1, const void *W2, const moe_plan_buffers *p, void *pool, void *act,
+                void *ypool, void *out, const moe_config *cfg, void *comm_stream,
+                void *compute_stream, void *ev_plan, void *ev_dispatch);
+
+/* Create / destroy n cudaEvent_t (timing disabled) for moe_forward. */
+int moe_events_create(void **events, int32_t n);
+int moe_events_destroy(void **events, int32_t n);
+
+/* Read the status word (synchronous: waits for work already queued that writes it). */
+int moe_get_status(const moe_plan_buffers *p, int32_t *code, int32_t *aux);
+
+/* Zero the status word on `stream`. */
+int moe_clear_status(const moe_plan_buffers *p, void *stream);
+
+/* Text for an error code. */
+const char *moe_strerror(int code);
+
+/* Library version string. */
+const char *moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

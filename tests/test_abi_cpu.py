@@ -1,0 +1,67 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol, and rejects
+bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"^(?:int|const char \*)\s*(moe_\w+)\(", src, re.M)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    import combine_moe_plan_03_b200 as moe
+    L = ctypes.CDLL(moe.LIB_PATH)
+    syms = declared_symbols()
+    assert len(syms) >= 14
+    for s in syms:
+        assert hasattr(L, s), f"{s} declared in include/moe.h but not exported"
+    assert sorted(moe.EXPORTS) == syms
+
+
+def test_sizes_and_bind_are_host_only():
+    import combine_moe_plan_03_b200 as moe
+    s = moe.moe_shape(8192, 7168, 2048, 256, 8, 128)
+    assert moe.moe_pool_rows_max(s) == 65536 + 256 * 127
+    nbytes = moe.moe_plan_arena_bytes(s)
+    assert nbytes > 0 and nbytes % 256 == 0
+    p = moe.moe_plan_bind(s, 1 << 20)
+    ptrs = [getattr(p, f) for f, _ in moe.moe_plan_buffers._fields_]
+    assert ptrs == sorted(ptrs) and all(q % 256 == 0 for q in ptrs)
+    assert ptrs[-1] < (1 << 20) + nbytes
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((16, 100, 128, 8, 2, 64), -2),     # H not a multiple of 64
+    ((16, 128, 128, 8, 2, 32), -2),     # tile not 64/128
+    ((16, 128, 128, 8, 33, 64), -1),    # k > 32
+    ((16, 128, 128, 2000, 2, 64), -1),  # E > 1024
+    ((-1, 128, 128, 8, 2, 64), -1),
+])
+def test_bad_shapes_rejected(shape, code):
+    import combine_moe_plan_03_b200 as moe
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_pool_rows_max(moe.moe_shape(*shape))
+    assert ei.value.code == code
+
+
+def test_misaligned_and_null_rejected_without_device():
+    import combine_moe_plan_03_b200 as moe
+    s = moe.moe_shape(16, 128, 128, 8, 2, 64)
+    p = moe.moe_plan_bind(s, 1 << 20)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_dispatch(s, (1 << 20) + 8, p, 1 << 24)
+    assert ei.value.code == moe.MOE_ERR_MISALIGNED
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_grouped_ffn(s, 1 << 20, 1 << 21, 0, p, 1 << 22, 1 << 23)
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    bad = moe.moe_plan_buffers()
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_combine(s, 1 << 20, 1 << 21, bad, 1 << 22)
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_strerror(-11).startswith("streaming FFN")

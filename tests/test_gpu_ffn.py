@@ -1,0 +1,108 @@
+"""The grouped SwiGLU FFN (tcgen05) and the whole layer vs the oracle, on small shapes that
+still span several tiles, both N-block widths and a ragged tail."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+
+def run_layer(cfg, streaming=0, mb=0, W=None):
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import bf16_dev, f32_dev, i32_dev, weights_dev
+    x = si.make_x(cfg, mb)
+    idx, w = si.make_routing(cfg, mb)
+    W1, W2 = W if W is not None else weights_dev(cfg)
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    for t in (buf.pool, buf.act, buf.ypool, buf.out):
+        t.view(torch.int16).fill_(0x7FC0)                     # poisoned storage
+    out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2,
+                      moe.moe_config(streaming, 0, 0, 0))
+    torch.cuda.synchronize()
+    return buf, x, idx, w, W1, W2, out
+
+
+def oracle_rows(cfg, x, idx, w, tokens):
+    W1 = [si.make_w1_expert(cfg, e) for e in range(cfg.E)]
+    W2 = [si.make_w2_expert(cfg, e) for e in range(cfg.E)]
+    return oracle.get().moe_forward(x[tokens], idx[tokens], w[tokens], W1, W2)
+
+
+SHAPES = [
+    # name, T, H, I, E, k, tile
+    ("tiny-like", 256, 256, 512, 8, 2, 64),
+    ("tile128", 300, 256, 256, 4, 2, 128),
+    ("I64-H192", 200, 192, 64, 3, 2, 64),       # GEMM A half width 64, GEMM Y N=64
+    ("H128-I192", 150, 128, 192, 5, 3, 128),    # GEMM Y N=128, GEMM A half width 64
+    ("one-expert", 130, 320, 384, 1, 1, 128),
+    ("deep-K", 64, 1024, 256, 2, 2, 64),
+]
+
+
+@pytest.mark.parametrize("streaming", [0, 1])
+@pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
+def test_layer_small_shapes(shape, streaming):
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import assert_layer_close, to_f64, check_plan_exact
+    name, T, H, I, E, k, tile = shape
+    cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=1234 + T)
+    buf, x, idx, w, W1, W2, out = run_layer(cfg, streaming)
+    code, aux = moe.moe_get_status(buf.plan)
+    assert code == 0, (moe.moe_strerror(code), aux)
+    check_plan_exact(buf, oracle.get().plan(idx, E, tile), T, k)
+    ref = oracle_rows(cfg, x, idx, w, np.arange(T))
+    assert_layer_close(to_f64(out), ref, name)
+    buf.close()
+
+
+def test_tiny_config_all_tokens_and_act():
+    """The tiny config end to end, plus GEMM A's act rows against the oracle's a = silu(g)*u."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import assert_layer_close, to_f64
+    cfg = si.CONFIGS["tiny"]
+    buf, x, idx, w, W1, W2, out = run_layer(cfg)
+    assert moe.moe_get_status(buf.plan)[0] == 0
+    ref = oracle_rows(cfg, x, idx, w, np.arange(cfg.T))
+    assert_layer_close(to_f64(out), ref, "tiny")
+    plan = oracle.get().plan(idx, cfg.E, cfg.tile)
+    act = to_f64(buf.act[: plan["P"]])
+    for f in (0, 1, 77, 300, cfg.T * cfg.k - 1):
+        t, j = divmod(f, cfg.k)
+        e = idx[t, j]
+        g, u, a, z = oracle.get().expert_ffn(x[t], si.make_w1_expert(cfg, e),
+                                             si.make_w2_expert(cfg, e))
+        p = plan["pool_row"][t, j]
+        assert np.abs(act[p] - a).max() <= 2e-2 * np.abs(a).max()
+    # padding rows of the pool give zero act
+    pad = plan["row_src"][: plan["P"]] < 0
+    assert np.all(act[pad] == 0)
+    buf.close()
+
+
+def test_back_to_back_layers_reuse_flags():
+    """Three layer calls in a row on the same buffers (flags reset by each plan)."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import assert_layer_close, bf16_dev, f32_dev, i32_dev, to_f64, weights_dev
+    cfg = si.custom("b2b", T=384, H=256, I=256, E=6, k=2, tile=64, seed=99, micro_batches=3)
+    W1, W2 = weights_dev(cfg)
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    outs, ins = [], []
+    for mb in range(3):
+        x = si.make_x(cfg, mb)
+        idx, w = si.make_routing(cfg, mb)
+        ins.append((x, idx, w, bf16_dev(x), i32_dev(idx), f32_dev(w)))
+    for mb in range(3):
+        x, idx, w, dx, di, dw = ins[mb]
+        o = buf.forward(dx, di, dw, W1, W2, moe.moe_config(1, 0, 0, 0))
+        with torch.cuda.stream(buf.compute):
+            outs.append(o.clone())
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(buf.plan)[0] == 0
+    for mb in range(3):
+        x, idx, w = ins[mb][:3]
+        ref = oracle_rows(cfg, x, idx, w, np.arange(cfg.T))
+        assert_layer_close(to_f64(outs[mb]), ref, f"mb{mb}")
+    buf.close()
