@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer hot path (plan -> dispatch -> grouped SwiGLU FFN -> combine).
+
+One step = one full layer call (all micro-batches of the workload) through the C ABI
+(moe_forward) with inputs resident in HBM. Prints one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload deepseek_v3]
+  python bench.py --impl reference ...      # the CPU oracle, timed on the host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent replica of
+the layer on its own tokens (the layer has no exchange step on one GPU: replicas only);
+value = tokens of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = ("MoE layer tokens/sec on 1 B200; dispatch+combine HBM GB/s; "
+          "grouped-GEMM % bf16 peak")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["moe", "reference"], default="moe")
+    ap.add_argument("--workload", default="deepseek_v3")
+    ap.add_argument("--streaming", type=int, default=-1,
+                    help="1: FFN claims tiles while dispatch runs; 0: serial; -1: default")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-tokens", type=int, default=16, help="oracle tokens per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ environment helpers
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, \
+            "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def reduce_max(values, device, world):
+    """Element-wise max over ranks (all_reduce MAX); identity for one rank."""
+    import torch
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.idx)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[5:9]):
+                if val.lower() in ("active", "1"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "combine_moe_plan_03_b200", "csrc"))):
+        h.update(open(os.path.join(ROOT, "combine_moe_plan_03_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if it was taken on the
+    current kernel sources (else None: the counters are stale)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+    except Exception:
+        return None
+    ent = d.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ inputs
+
+def host_weights(cfg):
+    """Full W1 / W2 on the host (bf16 bit patterns)."""
+    return si.make_w1(cfg), (si.make_w2(cfg) if cfg.I > 0 else None)
+
+
+def upload_weights(cfg, dev, rank, world, keep_host: bool):
+    """Rank 0 generates the weights and copies them to its GPU; other ranks receive them by
+    broadcast (setup only, outside the timed region)."""
+    import torch
+    W1 = torch.empty((cfg.E, cfg.H, 2 * cfg.I), dtype=torch.bfloat16, device=dev)
+    W2 = torch.empty((cfg.E, cfg.I, cfg.H), dtype=torch.bfloat16, device=dev)
+    host = None
+    if rank == 0:
+        if keep_host:
+            h1, h2 = host_weights(cfg)
+            W1.copy_(torch.from_numpy(h1.view(np.int16)).view(torch.bfloat16))
+            W2.copy_(torch.from_numpy(h2.view(np.int16)).view(torch.bfloat16))
+            host = (h1, h2)
+        else:
+            n1 = cfg.H * 2 * cfg.I
+            n2 = cfg.I * cfg.H
+            for e in range(cfg.E):
+                h1 = si.normal_bf16(cfg.seed, si.STREAM_W1, e * n1, n1, cfg.w1_sigma())
+                W1[e].copy_(torch.from_numpy(h1.view(np.int16)).view(torch.bfloat16)
+                            .view(cfg.H, 2 * cfg.I))
+                h2 = si.normal_bf16(cfg.seed, si.STREAM_W2, e * n2, n2, cfg.w2_sigma())
+                W2[e].copy_(torch.from_numpy(h2.view(np.int16)).view(torch.bfloat16)
+                            .view(cfg.I, cfg.H))
+    if world > 1:
+        import torch.distributed as dist
+        dist.broadcast(W1, src=0)
+        dist.broadcast(W2, src=0)
+    return W1, W2, host
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_tokens_per_s(cfg, x, idx, w, W1h, W2h, tokens, threads):
+    import oracle
+    orc = oracle.get()
+    W1l = [W1h[e] for e in range(cfg.E)]
+    W2l = [W2h[e] for e in range(cfg.E)]
+    t0 = time.perf_counter()
+    orc.moe_forward(x[tokens], idx[tokens], w[tokens], W1l, W2l, n_threads=threads)
+    return len(tokens) / (time.perf_counter() - t0)
+
+
+def cpu_baseline(cfg, x, idx, w, host, budget_s):
+    """The oracle as it stands on the host cores, on a bounded sample of the workload's tokens."""
+    threads = os.cpu_count() or 1
+    W1h, W2h = host
+    rng = np.random.default_rng(0)
+    probe = np.sort(rng.choice(cfg.T, size=min(cfg.T, threads), replace=False))
+    rate = oracle_tokens_per_s(cfg, x, idx, w, W1h, W2h, probe, threads)
+    n = int(max(threads, min(cfg.T, rate * budget_s)))
+    n = (n // threads) * threads or threads
+    sample = np.sort(rng.choice(cfg.T, size=min(n, cfg.T), replace=False))
+    t0 = time.perf_counter()
+    val = oracle_tokens_per_s(cfg, x, idx, w, W1h, W2h, sample, threads)
+    return {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(sample)} of {cfg.T} tokens of {cfg.name} (seeded), "
+                      f"{time.perf_counter() - t0:.1f} s, fp64 C oracle with OpenMP"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on the host cores (rank 0 only)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    cfg = si.CONFIGS[args.workload]
+    threads = os.cpu_count() or 1
+    orc = oracle.get()
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    rng = np.random.default_rng(1)
+    n = max(1, args.ref_tokens)
+    cache1, cache2 = {}, {}
+
+    def wts(tokens):
+        need = sorted(set(int(e) for e in idx[tokens].reshape(-1) if e >= 0))
+        for e in need:
+            if e not in cache1:
+                if cfg.identity:
+                    continue
+                cache1[e] = si.make_w1_expert(cfg, e)
+                cache2[e] = si.make_w2_expert(cfg, e)
+        return [cache1.get(e) for e in range(cfg.E)], [cache2.get(e) for e in range(cfg.E)]
+
+    def step():
+        tokens = np.sort(rng.choice(cfg.T, size=min(n, cfg.T), replace=False))
+        if cfg.identity:
+            t0 = time.perf_counter()
+            orc.moe_forward_identity(x[tokens], idx[tokens], w[tokens])
+            return len(tokens), time.perf_counter() - t0
+        W1l, W2l = wts(tokens)
+        t0 = time.perf_counter()
+        orc.moe_forward(x[tokens], idx[tokens], w[tokens], W1l, W2l, n_threads=threads)
+        return len(tokens), time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        step()
+    tok = secs = 0.0
+    for _ in range(args.steps):
+        a, b = step()
+        tok += a
+        secs += b
+    val = tok / secs
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(cfg, world),
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"{n} tokens per step of {cfg.name}, {args.steps} steps"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(cfg, world):
+    return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+            "tile": cfg.tile, "micro_batches": cfg.micro_batches, "routing": cfg.routing,
+            "identity_experts": cfg.identity,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2: each step streams the weights and pool (GBs) "
+                  "through the 126 MB L2"}
+
+
+# ------------------------------------------------------------------ the CUDA path
+
+def run_moe(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    import combine_moe_plan_03_b200 as moe
+
+    cfg = si.CONFIGS[args.workload]
+    peaks, peak_src = load_peaks()
+    streaming = 0 if args.streaming < 0 else args.streaming
+    mbs = cfg.micro_batches
+    want_cpu = (world == 1 and rank == 0 and not args.no_cpu_baseline)
+
+    # inputs: each rank takes its own tokens (micro-batch index offset by rank)
+    xs, idxs, ws = [], [], []
+    for m in range(mbs):
+        g = rank * mbs + m
+        xs.append(si.make_x(cfg, g))
+        i_, w_ = si.make_routing(cfg, g)
+        idxs.append(i_)
+        ws.append(w_)
+    if cfg.identity:
+        W1 = W2 = None
+        host = None
+    else:
+        W1, W2, host = upload_weights(cfg, dev, rank, world, keep_host=want_cpu)
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    dx = [dev_bf16(a) for a in xs]
+    didx = [torch.from_numpy(a).to(dev) for a in idxs]
+    dw = [torch.from_numpy(a).to(dev) for a in ws]
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, max(cfg.I, 64), cfg.E, cfg.k, cfg.tile, device=dev,
+                              identity=cfg.identity)
+    calls = args.steps * mbs
+    tev = moe.moe_timing_events_create(7 * calls)
+    import ctypes
+    ev_arrays = [(ctypes.c_void_p * 7)(*tev[7 * c: 7 * c + 7]) for c in range(calls)]
+    cfgs = [moe.moe_config(streaming, 0, 0, 0, ctypes.cast(ev_arrays[c], ctypes.c_void_p))
+            for c in range(calls)]
+    plain = moe.moe_config(streaming, 0, 0, 0, None)
+
+    def step_plain():
+        for m in range(mbs):
+            buf.forward(dx[m], didx[m], dw[m], W1, W2, plain)
+
+    for _ in range(args.warmup):
+        step_plain()
+    torch.cuda.synchronize()
+    code, aux = moe.moe_get_status(buf.plan)
+    if code != 0:
+        raise RuntimeError(f"device status after warm-up: {moe.moe_strerror(code)} ({aux})")
+
+    sampler = ClockSampler(physical_gpu_index(local))
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    c = 0
+    for _ in range(args.steps):
+        for m in range(mbs):
+            buf.forward(dx[m], didx[m], dw[m], W1, W2, cfgs[c])
+            c += 1
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    code, aux = moe.moe_get_status(buf.plan)
+    if code != 0:
+        raise RuntimeError(f"device status after timing: {moe.moe_strerror(code)} ({aux})")
+
+    el = moe.moe_event_elapsed_ms
+    total_ms = el(tev[0], tev[7 * (calls - 1) + 6])
+    ph = {k: 0.0 for k in ("plan", "dispatch", "gemm_a", "gemm_y", "combine")}
+    for c in range(calls):
+        e = tev[7 * c: 7 * c + 7]
+        ph["plan"] += el(e[0], e[1])
+        ph["dispatch"] += el(e[1], e[2])
+        ph["gemm_a"] += el(e[3], e[4])
+        ph["gemm_y"] += el(e[4], e[5])
+        ph["combine"] += el(e[5], e[6])
+    ph = {k: v / calls for k, v in ph.items()}        # ms per launch (per layer call)
+    red = reduce_max([total_ms] + [ph[k] for k in ph], dev, world)
+    total_ms = red[0]
+    ph = dict(zip(ph.keys(), red[1:]))
+
+    tokens_step = cfg.T * mbs
+    ms_step = total_ms / args.steps
+    value = world * tokens_step / (ms_step / 1000.0)
+
+    # ---------------- algorithmic work per layer call (averaged over the micro-batches)
+    pairs = [int((i >= 0).sum()) for i in idxs]
+    Ps = []
+    for i in idxs:
+        cnt = np.bincount(i[i >= 0].reshape(-1), minlength=cfg.E)
+        Ps.append(int(((cnt + cfg.tile - 1) // cfg.tile * cfg.tile).sum()))
+    pairs_m = float(np.mean(pairs))
+    P_m = float(np.mean(Ps))
+    H, I, T = cfg.H, cfg.I, cfg.T
+    disp_bytes = T * H * 2 + P_m * H * 2
+    comb_bytes = pairs_m * H * 2 + T * H * 2 + pairs_m * 8
+    dc_ms = ph["dispatch"] + ph["combine"]
+    dc_gbs = (disp_bytes + comb_bytes) / (dc_ms / 1000.0) / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",
+            "config": config_block(cfg, world), "streaming": streaming,
+            "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
+            "dispatch_combine": {"bytes_per_call": disp_bytes + comb_bytes,
+                                 "gbs": dc_gbs, "frac_hbm": dc_gbs / peaks["hbm_gbs"],
+                                 "dispatch_gbs": disp_bytes / (ph["dispatch"] / 1e3) / 1e9,
+                                 "combine_gbs": comb_bytes / (ph["combine"] / 1e3) / 1e9,
+                                 "padding_bytes": (P_m - pairs_m) * H * 2}}
+    if not cfg.identity:
+        flops_a = pairs_m * 4.0 * H * I
+        flops_y = pairs_m * 2.0 * H * I
+        ffn_ms = ph["gemm_a"] + ph["gemm_y"]
+        ffn_tflops = (flops_a + flops_y) / (ffn_ms / 1e3) / 1e12
+        exec_tflops = P_m * 6.0 * H * I / (ffn_ms / 1e3) / 1e12
+        line["grouped_ffn"] = {"useful_tflops": ffn_tflops,
+                               "frac_bf16_peak": ffn_tflops / peaks["bf16_tflops"],
+                               "executed_tflops": exec_tflops,
+                               "executed_frac_bf16_peak": exec_tflops / peaks["bf16_tflops"],
+                               "weight_gbs": cfg.E * 3 * H * I * 2 / (ffn_ms / 1e3) / 1e9}
+        achieved = flops_a / (ph["gemm_a"] / 1e3) / 1e12
+        line["roofline"] = {"kernel": "ffn_gemm_kernel<0> (GEMM A + SwiGLU)", "bound": "tensor",
+                            "achieved": achieved, "peak": peaks["bf16_tflops"],
+                            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                            "traffic": committed_traffic("ffn_gemm_kernel<0>"),
+                            "peak_source": f"{peak_src} bf16 burst",
+                            "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                            "algorithmic": "useful flops pairs*4*H*I per launch"}
+    else:
+        achieved = disp_bytes / (ph["dispatch"] / 1e3) / 1e9
+        line["roofline"] = {"kernel": "dispatch_kernel", "bound": "hbm", "achieved": achieved,
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": achieved / peaks["hbm_gbs"],
+                            "traffic": committed_traffic("dispatch_kernel"),
+                            "peak_source": f"{peak_src} HBM copy"}
+
+    # ---------------- e2e: pinned host inputs in, result out, copies inside the timed region
+    hx = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in xs]
+    hidx = [torch.from_numpy(a).pin_memory() for a in idxs]
+    hw = [torch.from_numpy(a).pin_memory() for a in ws]
+    hout = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    # two device copies of each input, so the copy of the next call's inputs (comm stream)
+    # never overwrites what the current call's combine (compute stream) still reads
+    bx = [torch.empty_like(dx[0]) for _ in range(2)]
+    bi = [torch.empty_like(didx[0]) for _ in range(2)]
+    bw = [torch.empty_like(dw[0]) for _ in range(2)]
+    ncall = [0]
+
+    def e2e_step():
+        for m in range(mbs):
+            j = ncall[0] & 1
+            ncall[0] += 1
+            with torch.cuda.stream(buf.comm):
+                bx[j].copy_(hx[m], non_blocking=True)
+                bi[j].copy_(hidx[m], non_blocking=True)
+                bw[j].copy_(hw[m], non_blocking=True)
+            buf.forward(bx[j], bi[j], bw[j], W1, W2, plain)
+            with torch.cuda.stream(buf.compute):
+                hout.copy_(buf.out[: cfg.T], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s_ev = torch.cuda.Event(enable_timing=True)
+    e_ev = torch.cuda.Event(enable_timing=True)
+    s_ev.record(buf.comm)
+    for _ in range(args.steps):
+        e2e_step()
+    e_ev.record(buf.compute)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max([s_ev.elapsed_time(e_ev)], dev, world)[0]
+    h2d = mbs * (cfg.T * cfg.H * 2 + cfg.T * cfg.k * 8)
+    d2h = mbs * cfg.T * cfg.H * 2
+    line["e2e"] = {"value": world * tokens_step * args.steps / (e2e_ms / 1000.0),
+                   "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    kernels_per_call = 5 if cfg.identity else 7
+    line["gpu_launches"] = kernels_per_call * calls
+    line["clocks"] = clocks
+    if want_cpu and not cfg.identity:
+        line["cpu_baseline"] = cpu_baseline(cfg, xs[0], idxs[0], ws[0], host,
+                                            args.cpu_baseline_seconds)
+    elif want_cpu:
+        line["cpu_baseline"] = None
+    moe.moe_events_destroy(tev)
+    buf.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_moe(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -44,7 +44,8 @@ class moe_plan_buffers(ctypes.Structure):
 
 class moe_config(ctypes.Structure):
     _fields_ = [("streaming", ctypes.c_int32), ("ffn_ctas", ctypes.c_int32),
-                ("wait_timeout_us", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("wait_timeout_us", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("timing_events", ctypes.c_void_p)]
 
 
 class MoEError(RuntimeError):
@@ -73,6 +74,8 @@ def _load():
         "moe_forward": [P(moe_shape), vp, vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp,
                         P(moe_config), vp, vp, vp, vp],
         "moe_events_create": [P(vp), i32],
+        "moe_timing_events_create": [P(vp), i32],
+        "moe_event_elapsed_ms": [vp, vp, P(ctypes.c_float)],
         "moe_events_destroy": [P(vp), i32],
         "moe_get_status": [P(moe_plan_buffers), P(i32), P(i32)],
         "moe_clear_status": [P(moe_plan_buffers), vp],
@@ -93,8 +96,8 @@ _lib = _load()
 # Names exported by include/moe.h, in declaration order.
 EXPORTS = ["moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
            "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_events_create",
-           "moe_events_destroy", "moe_get_status", "moe_clear_status", "moe_strerror",
-           "moe_version"]
+           "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
+           "moe_get_status", "moe_clear_status", "moe_strerror", "moe_version"]
 
 
 def lib():
@@ -184,6 +187,18 @@ def moe_events_create(n: int) -> list[int]:
     arr = (ctypes.c_void_p * n)()
     _check("moe_events_create", _lib.moe_events_create(arr, n))
     return [int(a) for a in arr]
+
+
+def moe_timing_events_create(n: int) -> list[int]:
+    arr = (ctypes.c_void_p * n)()
+    _check("moe_timing_events_create", _lib.moe_timing_events_create(arr, n))
+    return [int(a) for a in arr]
+
+
+def moe_event_elapsed_ms(start: int, end: int) -> float:
+    ms = ctypes.c_float(0)
+    _check("moe_event_elapsed_ms", _lib.moe_event_elapsed_ms(start, end, ctypes.byref(ms)))
+    return float(ms.value)
 
 
 def moe_events_destroy(events: list[int]) -> None:

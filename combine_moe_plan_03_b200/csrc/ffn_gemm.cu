@@ -395,8 +395,11 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   a.tile = s.tile;
   a.streaming = cfg.streaming;
   a.timeout_ns = timeout_ns;
+  cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(cfg.timing_events);
+  if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t e = launch_one<0>(ta_pool, tb_w1, a, grid, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
 
   FfnParams y = a;
   y.out = static_cast<uint16_t *>(ypool);
@@ -408,7 +411,9 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   y.up_col = 0;
   y.streaming = 0;
   e = launch_one<1>(ta_act, tb_w2, y, cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms, st);
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 }  // namespace moe

@@ -205,17 +205,27 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
     if (cudaEventRecord(evd, comp) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamWaitEvent(comm, evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
   }
+  cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(c.timing_events);
+  if (tev != nullptr && cudaEventRecord(tev[0], comm) != cudaSuccess) return MOE_ERR_CUDA;
   if ((rc = moe_plan(s, topk_idx, p, nullptr, comm)) != MOE_OK) return rc;
   if (cudaEventRecord(evp, comm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[1], comm) != cudaSuccess) return MOE_ERR_CUDA;
   const int signal = (!identity && c.streaming) ? 1 : 0;
   if ((rc = moe_dispatch(s, x, p, pool, signal, comm)) != MOE_OK) return rc;
   if (cudaEventRecord(evd, comm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[2], comm) != cudaSuccess) return MOE_ERR_CUDA;
   if (!identity) {
     if (cudaStreamWaitEvent(comp, c.streaming ? evp : evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
     if ((rc = moe_grouped_ffn(s, pool, W1, W2, p, act, ypool, &c, comp)) != MOE_OK) return rc;
   }
   if (cudaStreamWaitEvent(comp, evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
-  return moe_combine(s, identity ? pool : ypool, topk_w, p, out, comp);
+  if (identity && tev != nullptr) {
+    for (int i = 3; i < 6; ++i)
+      if (cudaEventRecord(tev[i], comp) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if ((rc = moe_combine(s, identity ? pool : ypool, topk_w, p, out, comp)) != MOE_OK) return rc;
+  if (tev != nullptr && cudaEventRecord(tev[6], comp) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 int moe_events_create(void **events, int32_t n) {
@@ -225,6 +235,24 @@ int moe_events_create(void **events, int32_t n) {
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
     events[i] = e;
   }
+  return MOE_OK;
+}
+
+int moe_timing_events_create(void **events, int32_t n) {
+  if (events == nullptr || n < 0) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return MOE_ERR_CUDA;
+    events[i] = e;
+  }
+  return MOE_OK;
+}
+
+int moe_event_elapsed_ms(void *start, void *end, float *ms) {
+  if (start == nullptr || end == nullptr || ms == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cudaEventElapsedTime(ms, static_cast<cudaEvent_t>(start), static_cast<cudaEvent_t>(end)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -97,6 +97,12 @@ typedef struct moe_config {
   int32_t ffn_ctas;        /* persistent FFN CTAs; 0 = number of SMs (streaming: SMs - 16) */
   int32_t wait_timeout_us; /* bound on every device-side wait; 0 = 2,000,000 us */
   int32_t reserved;
+  /* NULL, or 7 cudaEvent_t that moe_forward records at the phase boundaries, each on
+     the stream of the kernels around it: [0] comm before plan, [1] comm after plan,
+     [2] comm after dispatch, [3] compute before the FFN, [4] compute after GEMM A,
+     [5] compute after GEMM Y, [6] compute after combine. moe_grouped_ffn records
+     [3], [4], [5]. For per-kernel timing with cudaEventElapsedTime. */
+  void *const *timing_events;
 } moe_config;
 
 /* Dropless pool bound: T*k + min(E, T*k)*(tile-1), rounded up to a multiple of tile. */
@@ -171,9 +177,17 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
                 void *ypool, void *out, const moe_config *cfg, void *comm_stream,
                 void *compute_stream, void *ev_plan, void *ev_dispatch);
 
-/* Create / destroy n cudaEvent_t (timing disabled) for moe_forward. */
+/* Create / destroy n cudaEvent_t (timing disabled) for moe_forward's ordering. */
 int moe_events_create(void **events, int32_t n);
 int moe_events_destroy(void **events, int32_t n);
+
+/* Create n cudaEvent_t with timing enabled (for moe_config.timing_events); destroy
+ * them with moe_events_destroy. */
+int moe_timing_events_create(void **events, int32_t n);
+
+/* Milliseconds between two recorded timing events (cudaEventElapsedTime; the end
+ * event must have completed, else MOE_ERR_CUDA). */
+int moe_event_elapsed_ms(void *start, void *end, float *ms);
 
 /* Read the status word (synchronous: waits for work already queued that writes it). */
 int moe_get_status(const moe_plan_buffers *p, int32_t *code, int32_t *aux);
