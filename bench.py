@@ -82,6 +82,11 @@ def reduce_max(values, device, world):
     return t.tolist()
 
 
+def whole_job_tokens_per_s(world, tokens_per_step, ms_per_step):
+    """All ranks' tokens per step over the slowest rank's time per step."""
+    return world * tokens_per_step / (ms_per_step / 1000.0)
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -396,7 +401,7 @@ def run_moe(args):
 
     tokens_step = cfg.T * mbs
     ms_step = total_ms / args.steps
-    value = world * tokens_step / (ms_step / 1000.0)
+    value = whole_job_tokens_per_s(world, tokens_step, ms_step)
 
     # ---------------- algorithmic work per layer call (averaged over the micro-batches)
     pairs = [int((i >= 0).sum()) for i in idxs]

@@ -1,0 +1,78 @@
+"""bench.py's multi-rank host logic on CPU with gloo (world size 2): max-over-ranks timing,
+the whole-job value, and the reference arm running on rank 0 only."""
+import io
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r measured (10 + r) ms for the timed region and 2 + 3r ms for one phase
+        red = bench.reduce_max([10.0 + rank, 2.0 + 3 * rank], torch.device("cpu"), world)
+        bench.barrier(world)
+        val = bench.whole_job_tokens_per_s(world, tokens_per_step=8192, ms_per_step=red[0])
+        q.put((rank, red, val))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_max_and_value_over_two_gloo_ranks():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, red, val in res:
+        assert red == [11.0, 5.0]                        # max over ranks, element-wise
+        assert val == pytest.approx(2 * 8192 / 0.011)   # all ranks' tokens / max time
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"])
+    assert rc == 0 and buf.getvalue() == ""
+
+
+def test_reference_arm_line_on_rank_zero(monkeypatch):
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "2",
+                         "--warmup", "1", "--ref-tokens", "8"])
+    line = json.loads(buf.getvalue())
+    assert rc == 0 and line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
