@@ -25,6 +25,8 @@ MOE_ERR_UNSUPPORTED_SHAPE = -2
 MOE_ERR_MISALIGNED = -3
 MOE_ERR_CUDA = -4
 MOE_ERR_NO_DEVICE = -5
+MOE_ERR_SCRATCH_LIMIT = -6
+MOE_PLAN_NOALLOC_SCRATCH_INTS = (1 << 19) + 64
 MOE_ERR_BAD_INDEX = -10
 MOE_ERR_FLAG_TIMEOUT = -11
 MOE_ERR_POOL_OVERFLOW = -12
@@ -79,6 +81,7 @@ def _load():
         "moe_events_destroy": [P(vp), i32],
         "moe_get_status": [P(moe_plan_buffers), P(i32), P(i32)],
         "moe_clear_status": [P(moe_plan_buffers), vp],
+        "moe_plan_noalloc": [P(moe_shape), vp, P(moe_plan_buffers), vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -97,7 +100,8 @@ _lib = _load()
 EXPORTS = ["moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
            "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
-           "moe_get_status", "moe_clear_status", "moe_strerror", "moe_version"]
+           "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
+           "moe_version"]
 
 
 def lib():
@@ -148,6 +152,15 @@ def moe_plan(shape, topk_idx_ptr: int, plan: moe_plan_buffers, host_P_ptr: int =
              stream: int = 0) -> None:
     _check("moe_plan", _lib.moe_plan(ctypes.byref(_shape(shape)), topk_idx_ptr,
                                      ctypes.byref(plan), host_P_ptr or None, stream or None))
+
+
+def moe_plan_noalloc(shape, topk_idx_ptr: int, plan: moe_plan_buffers, host_P_ptr: int = 0,
+                     stream: int = 0) -> None:
+    """moe_plan without caller-provided scratch (for callers that cannot allocate device
+    memory): the library's static 2 MiB device buffer holds it, plan.workspace is ignored."""
+    _check("moe_plan_noalloc", _lib.moe_plan_noalloc(ctypes.byref(_shape(shape)), topk_idx_ptr,
+                                                     ctypes.byref(plan), host_P_ptr or None,
+                                                     stream or None))
 
 
 def moe_dispatch(shape, x_ptr: int, plan: moe_plan_buffers, pool_ptr: int,

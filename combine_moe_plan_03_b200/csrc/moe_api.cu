@@ -289,6 +289,8 @@ const char *moe_strerror(int code) {
     case MOE_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
     case MOE_ERR_CUDA: return "CUDA call failed";
     case MOE_ERR_NO_DEVICE: return "current device is not sm_100";
+    case MOE_ERR_SCRATCH_LIMIT:
+      return "shape needs more plan scratch than moe_plan_noalloc's static buffer holds";
     case MOE_ERR_BAD_INDEX: return "topk_idx value outside [-1, E)";
     case MOE_ERR_FLAG_TIMEOUT: return "streaming FFN timed out waiting for a pool tile";
     case MOE_ERR_POOL_OVERFLOW: return "pool rows exceeded the dropless bound";

@@ -62,6 +62,7 @@ extern "C" {
 #define MOE_ERR_MISALIGNED (-3)        /* a tensor pointer not 16-byte aligned */
 #define MOE_ERR_CUDA (-4)              /* a CUDA runtime / driver call failed */
 #define MOE_ERR_NO_DEVICE (-5)         /* current device is not sm_100 */
+#define MOE_ERR_SCRATCH_LIMIT (-6)     /* moe_plan_noalloc: shape needs more than its static scratch */
 /* device-side errors, reported through the status word (moe_get_status) */
 #define MOE_ERR_BAD_INDEX (-10)     /* topk_idx value outside [-1, E); aux = pair id */
 #define MOE_ERR_FLAG_TIMEOUT (-11)  /* streaming FFN gave up waiting on a tile flag; aux = tile */
@@ -197,6 +198,32 @@ int moe_clear_status(const moe_plan_buffers *p, void *stream);
 
 /* Text for an error code. */
 const char *moe_strerror(int code);
+
+/*
+ * moe_plan_noalloc - moe_plan for callers that cannot allocate device memory.
+ * The paper has no counterpart; this is a convenience of this library.
+ *
+ * Same inputs, outputs and results as moe_plan (bit for bit), but the plan's
+ * scratch lives in a static device buffer inside the library, so p->workspace is
+ * ignored (it may be NULL) and the caller never sizes or allocates scratch. Meant
+ * for code whose host framework owns all device memory and gives it no allocator
+ * (an inference engine's plugin hook, for instance), or loops that cannot afford
+ * a cudaMalloc's device synchronisation or its failure under a fixed budget.
+ *   - Maximum: E * max(1, ceil(T*k/256)) + 8 <= MOE_PLAN_NOALLOC_SCRATCH_INTS
+ *     (2 MiB + 256 B of int32; e.g. E = 256 with up to 524,288 pairs). Larger
+ *     shapes return MOE_ERR_SCRATCH_LIMIT and launch nothing. Every GPU that loads
+ *     the library holds this buffer until the process exits.
+ *   - All calls on a device share the buffer and it keeps the last call's
+ *     contents; each call rewrites what it reads and zeroes its counter first, so
+ *     back-to-back calls are independent, but calls that overlap on the GPU
+ *     (issued on concurrent streams) race on it.
+ *   - The first call on a device (with that device current) looks up the
+ *     buffer's device address; make it before any stream capture.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define MOE_PLAN_NOALLOC_SCRATCH_INTS ((1 << 19) + 64)
+int moe_plan_noalloc(const moe_shape *s, const int32_t *topk_idx, const moe_plan_buffers *p,
+                     int32_t *host_P, void *stream);
 
 /* Library version string. */
 const char *moe_version(void);
