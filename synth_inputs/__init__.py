@@ -15,6 +15,7 @@ pages describe; the sizes follow the DeepSeek-V3 / Qwen3-235B-A22B families and 
   decode_microbatch 3 x T=128, H=7168, I=2048, E=256, k=8, tile=128, Zipf(1.2) routing
   dc_sweep_T{1024,4096,16384,65536}_{uniform,zipf}
                     H=7168, E=256, k=8, tile=128, identity experts
+  deepseek_v3_e32   T=1024, H=7168, I=2048, E=32, k=8, tile=128 (profiling size)
 """
 from __future__ import annotations
 
@@ -194,6 +195,11 @@ def _cfg_list():
     out["decode_microbatch"] = MoEConfig("decode_microbatch", T=128, H=7168, I=2048, E=256, k=8,
                                          tile=128, seed=SEED_BASE + 3, routing="zipf", alpha=1.2,
                                          micro_batches=3)
+    # the DeepSeek-V3 expert shape at 32 experts: ~256 rows per expert like the full layer,
+    # about 3 GB on the device (for detailed kernel profiles)
+    out["deepseek_v3_e32"] = MoEConfig("deepseek_v3_e32", T=1024, H=7168, I=2048, E=32, k=8,
+                                       tile=128, seed=SEED_BASE + 5, routing="softmax_bias",
+                                       bias_sigma=0.5)
     for T in (1024, 4096, 16384, 65536):
         for r in ("uniform", "zipf"):
             nm = f"dc_sweep_T{T}_{r}"
