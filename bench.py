@@ -39,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["moe", "reference"], default="moe")
     ap.add_argument("--workload", default="deepseek_v3")
@@ -96,7 +96,7 @@ def barrier(world):
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 100 ms while the timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
@@ -105,6 +105,14 @@ class ClockSampler:
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
+
+    def mark(self, begin: bool):
+        """Host wall time of the start / end of the timed region (samples outside are dropped)."""
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
 
     def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -127,14 +135,21 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, smax, reasons = [], [], set()
+        sm, smax, power, reasons = [], [], [], set()
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            if ts is not None and self.t0 is not None and not (self.t0 <= ts <= self.t1):
+                continue
+            try:
                 sm.append(float(parts[1]))
                 smax.append(float(parts[2]))
+                power.append(float(parts[3]))
             except ValueError:
                 continue
             for name, val in zip(self.REASONS, parts[5:9]):
@@ -143,7 +158,8 @@ class ClockSampler:
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_median": statistics.median(power) if power else None}
 
 
 def physical_gpu_index(local_rank: int) -> int:
@@ -372,12 +388,14 @@ def run_moe(args):
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
+    sampler.mark(True)
     c = 0
     for _ in range(args.steps):
         for m in range(mbs):
             buf.forward(dx[m], didx[m], dw[m], W1, W2, cfgs[c])
             c += 1
     torch.cuda.synchronize()
+    sampler.mark(False)
     barrier(world)
     clocks = sampler.stop()
     code, aux = moe.moe_get_status(buf.plan)
@@ -410,6 +428,7 @@ def run_moe(args):
         cnt = np.bincount(i[i >= 0].reshape(-1), minlength=cfg.E)
         Ps.append(int(((cnt + cfg.tile - 1) // cfg.tile * cfg.tile).sum()))
     pairs_m = float(np.mean(pairs))
+    n_live_experts = float(np.mean([len(np.unique(i[i >= 0])) for i in idxs]))
     P_m = float(np.mean(Ps))
     H, I, T = cfg.H, cfg.I, cfg.T
     disp_bytes = T * H * 2 + P_m * H * 2
@@ -422,6 +441,8 @@ def run_moe(args):
             "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",
             "config": config_block(cfg, world), "streaming": streaming,
             "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
+            "phases_mcycles_per_call": ({k: round(v * clocks["sm_mhz"] / 1000.0, 4)
+                                         for k, v in ph.items()} if clocks.get("sm_mhz") else None),
             "dispatch_combine": {"bytes_per_call": disp_bytes + comb_bytes,
                                  "gbs": dc_gbs, "frac_hbm": dc_gbs / peaks["hbm_gbs"],
                                  "dispatch_gbs": disp_bytes / (ph["dispatch"] / 1e3) / 1e9,
@@ -437,14 +458,22 @@ def run_moe(args):
                                "frac_bf16_peak": ffn_tflops / peaks["bf16_tflops"],
                                "executed_tflops": exec_tflops,
                                "executed_frac_bf16_peak": exec_tflops / peaks["bf16_tflops"],
-                               "weight_gbs": cfg.E * 3 * H * I * 2 / (ffn_ms / 1e3) / 1e9}
+                               "weight_gbs": n_live_experts * 3 * H * I * 2 / (ffn_ms / 1e3)
+                                             / 1e9,
+                               "weight_frac_hbm": n_live_experts * 3 * H * I * 2
+                                                  / (ffn_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        line["grouped_ffn"]["frac_bf16_sustained"] = ffn_tflops / peaks["bf16_tflops_sustained"]
         achieved = flops_a / (ph["gemm_a"] / 1e3) / 1e12
+        # The timed loop runs back to back at the power cap (see "clocks"), so the kernel is
+        # compared with cuBLAS's sustained bf16 rate under the same cap; burst beside it.
         line["roofline"] = {"kernel": "ffn_gemm_kernel<0> (GEMM A + SwiGLU)", "bound": "tensor",
-                            "achieved": achieved, "peak": peaks["bf16_tflops"],
-                            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                            "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                            "unit": "TFLOP/s",
+                            "frac": achieved / peaks["bf16_tflops_sustained"],
                             "traffic": committed_traffic("ffn_gemm_kernel<0>"),
-                            "peak_source": f"{peak_src} bf16 burst",
-                            "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                            "peak_source": f"{peak_src} bf16 sustained (timed inside a long "
+                                           "loop at the power cap)",
+                            "frac_of_burst": achieved / peaks["bf16_tflops"],
                             "algorithmic": "useful flops pairs*4*H*I per launch"}
     else:
         achieved = disp_bytes / (ph["dispatch"] / 1e3) / 1e9

@@ -3,25 +3,39 @@
 // sm_100a tensor cores:
 //   GEMM A: act[p, n]   = bf16( silu(pool[p] . W1[e][:, n]) * (pool[p] . W1[e][:, I + n]) )
 //   GEMM Y: ypool[p, m] = bf16( act[p] . W2[e][:, m] )
-// for the rows p of each 128-row block of expert e (the plan's row-block table).
+// for the live rows p of expert e (pool rows past an expert's count are padding and
+// are not computed; combine never reads them).
 //
-// One persistent kernel per GEMM, one CTA per SM, 6 warps:
-//   warp 0      TMA producer: per k-step, one 128x64 A box (K-major, 128-byte
-//               swizzle) and N/64 B boxes of 64(k) x 64(n) (the weights stay in
-//               their [K, N] layout: an MN-major operand) into a 4-stage ring.
-//               In streaming mode it first waits (bounded, acquire) until the
-//               tile flags of the block's pool rows are full.
+// Orientation: the weights are the MMA's M operand and the pool rows its N operand
+// (D^T = W^T X^T). A work unit is (row chunk of one expert: up to 256 live rows,
+// block of weight columns). Its N is the chunk's live rows rounded up to 16, so the
+// tile padding of the pool costs (almost) no tensor work, and a chunk of 256 rows
+// uses each weight tile it loads 256 times. Each unit has two 128-row weight tiles
+// and two TMEM accumulators (128 lanes x N columns each):
+//   GEMM A: tile 0 = 128 gate columns, tile 1 = the same 128 up columns, so lane f
+//           of the epilogue holds gate and up of output column f for every row;
+//   GEMM Y: tiles 0 and 1 = two adjacent blocks of 128 output columns.
+//
+// One persistent kernel per GEMM, one CTA per SM, 10 warps:
+//   warp 0      TMA producer: per k-step two weight tiles of 128 columns x 64 k
+//               (two 64x64 boxes each; weights stay in their [K, N] layout, read as
+//               an MN-major operand, 128-byte swizzle) and ceil(N/32) boxes of
+//               32 pool rows x 64 k (K-major, 128-byte swizzle), into a 3-stage
+//               ring of 64 KB stages. In streaming mode it first waits (bounded,
+//               acquire) until the tile flags of the chunk's pool rows are full.
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (M=128, N=256 or 128, K=16; bf16 in, fp32 accumulate) into one of
-//               two 256-column TMEM accumulators and commits the stage back to
-//               the producer and the finished accumulator to the epilogue.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//               32*(w%4)...), SwiGLU (GEMM A) or plain conversion (GEMM Y), bf16
-//               stores, then release the accumulator, so the epilogue of one
-//               unit overlaps the main loop of the next.
-// Work unit = (row block, N block); units are dealt round-robin over the CTAs,
-// N block fastest, so the CTAs working at one time share the same A rows and the
-// same expert's weights through L2.
+//               (M=128, N<=256, K=16; bf16 in, fp32 accumulate), two per 16 k (one
+//               per accumulator), commits each stage back to the producer and the
+//               finished unit to the epilogue.
+//   warps 2-9   epilogue: two warps per TMEM lane quadrant (warp w reads lanes
+//               32*(w%4)... and every other group of 32 pool rows), tcgen05.ld,
+//               SwiGLU (GEMM A) or conversion (GEMM Y) to bf16, a 32x32 turn in
+//               shared memory, and 16-byte stores along the output rows.
+// Units are handed out in order (row chunk, then weight block) from a global ticket
+// counter as CTAs free up, so the CTAs working at one time share the same pool rows
+// and the same expert's weights through L2, and uneven units balance out. The
+// producer takes the ticket and passes the unit id to the MMA thread and the
+// epilogue through a 4-slot ring in shared memory.
 //
 // Every wait is bounded (global timer). The tile-flag wait, furthest upstream,
 // gets the configured budget; the pipeline waits downstream of it get two (TMA
@@ -35,33 +49,40 @@
 
 namespace moe {
 
-constexpr int kBM = 128;
-constexpr int kBK = 64;
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kBK * 2;        // 16 KB
-constexpr int kChunkBytes = 64 * kBK * 2;     // 8 KB: 64 columns x 64 k-rows
-constexpr int kBBytesMax = 4 * kChunkBytes;   // N <= 256
-constexpr int kStageBytes = kABytes + kBBytesMax;
+constexpr int kBM = 128;                              // weight columns per tile (MMA M)
+constexpr int kBK = 64;                               // k per stage
+constexpr int kMaxN = kGemmBlockM;                    // pool rows per unit (MMA N <= 256)
+constexpr int kStages = 3;
+constexpr int kChunkBytes = 64 * kBK * 2;             // 8 KB: 64 weight columns x 64 k
+constexpr int kWTileBytes = 2 * kChunkBytes;          // 16 KB: one 128-column weight tile
+constexpr int kRowBox = 32;                           // pool rows per TMA box
+constexpr int kRowBoxBytes = kRowBox * kBK * 2;       // 4 KB
+constexpr int kStageBytes = 2 * kWTileBytes + kMaxN * kBK * 2;  // 64 KB
 constexpr int kTmemCols = 512;
 constexpr int kAccStride = 256;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr int kSchedSlots = 4;                        // unit ids in flight inside a CTA
 constexpr int kBarrierBytes = 256;
-constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+constexpr int kXposeBytes = 32 * 32 * 2;              // per epilogue warp: 32 rows x 32 columns bf16
+constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kEpiWarps * kXposeBytes + 1024;
 
 struct FfnParams {
-  const int32_t *mblk;     // row blocks {row_start, expert, rows}
-  const int32_t *meta;     // meta[2] = number of row blocks
+  const int32_t *mblk;     // row chunks {row_start, expert, live rows <= 256}
+  const int32_t *meta;     // meta[2] = number of row chunks
   const uint32_t *flags;   // pool tile flags (streaming)
   int32_t *status;
   uint16_t *out;           // act (GEMM A) or ypool (GEMM Y)
   int64_t out_ld;          // elements per row of out
   int32_t K;               // reduction length
-  int32_t n_blocks;        // N blocks per row block
-  int32_t bn;              // GEMM A: columns of act per block (gate and up each); GEMM Y: N
-  int32_t k_rows;          // rows per expert in the B tensor map (H for W1, I for W2)
-  int32_t up_col;          // GEMM A: first up column of W1 (= I)
+  int32_t n_blocks;        // weight-column blocks per row chunk
+  int32_t col_step;        // weight columns per block (GEMM A 128, GEMM Y 256)
+  int32_t col1_off;        // first column of tile 1 inside the block's weights (I or 128)
+  int32_t n_out;           // output columns (I or H): masks a ragged last block
+  int32_t k_rows;          // rows per expert in the weight tensor map (H for W1, I for W2)
   int32_t tile;            // pool tile rows
   int32_t streaming;
+  int32_t *sched;          // {next unit ticket, CTAs done}: zero at launch, zeroed again at exit
   uint64_t timeout_ns;
 };
 
@@ -71,19 +92,31 @@ __device__ __forceinline__ void raise_abort(volatile int *abort, int32_t *status
   *abort = 1;
 }
 
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  __nv_bfloat16 b = __float2bfloat16_rn(v);
+  return *reinterpret_cast<uint16_t *>(&b);
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
-    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                    const __grid_constant__ CUtensorMap tm_b, const FfnParams prm) {
+    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_x, const FfnParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
   uint64_t *empty = full + kStages;
-  uint64_t *acc_full = empty + kStages;
-  uint64_t *acc_empty = acc_full + 2;
-  uint64_t *drain = acc_empty + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *acc_full = empty + kStages;  // the unit's accumulators are complete
+  uint64_t *acc_empty = acc_full + 1;    // the epilogue has read them
+  uint64_t *drain = acc_empty + 1;
+  uint64_t *sched_full = drain + 1;          // [kSchedSlots] a unit id was written
+  uint64_t *sched_empty = sched_full + kSchedSlots;  // [kSchedSlots] MMA + epilogue read it
+  int32_t *sched = reinterpret_cast<int32_t *>(sched_empty + kSchedSlots);  // unit ids, -1 = end
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched + kSchedSlots);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   int *never = abort_flag + 1;  // stays 0: waits that must not be cut short by an abort
 
@@ -95,19 +128,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, 128);
-    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiWarps * 32);
     mbar_init(drain, 1);
+    for (int i = 0; i < kSchedSlots; ++i) {
+      mbar_init(sched_full + i, 1);
+      mbar_init(sched_empty + i, 1 + kEpiWarps);
+    }
     *abort_flag = 0;
     *never = 0;
     fence_mbarrier_init();
     fence_proxy_async_shared();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -119,10 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   volatile int *abort = abort_flag;
 
-  const int64_t n_units = (int64_t)prm.meta[2] * prm.n_blocks;
-  const int mma_n = kMode == 0 ? 2 * prm.bn : prm.bn;
-  const int n_chunks = mma_n / 64;
-  const uint32_t stage_tx = (uint32_t)(kABytes + n_chunks * kChunkBytes);
+  const int32_t n_units = prm.meta[2] * prm.n_blocks;
   const int kb_count = prm.K / kBK;
 
   if (warp == 0) {
@@ -130,12 +162,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ TMA producer
       uint32_t stage = 0, phase = 0;
       uint32_t issued = 0, last_parity = 0;  // per stage: ever issued, parity of last issue
-      for (int64_t u = blockIdx.x; u < n_units && !*abort; u += gridDim.x) {
+      uint32_t sslot = 0, sphase = 0;
+      for (;;) {
+        // take the next unit (tickets are handed out in unit order) and publish it
+        if (!mbar_wait(sched_empty + sslot, sphase ^ 1u, 2 * prm.timeout_ns, abort)) {
+          raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+          break;
+        }
+        const int32_t ticket = atomicAdd(prm.sched + 0, 1);
+        const int64_t u = (ticket < n_units && !*abort) ? ticket : -1;
+        sched[sslot] = (int32_t)u;
+        mbar_arrive(sched_full + sslot);
+        if (++sslot == kSchedSlots) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (u < 0) break;
         const int mb = (int)(u / prm.n_blocks);
         const int nb = (int)(u % prm.n_blocks);
         const int32_t row0 = prm.mblk[3 * mb + 0];
         const int32_t e = prm.mblk[3 * mb + 1];
         const int32_t rows = prm.mblk[3 * mb + 2];
+        const int nbox = (rows + kRowBox - 1) / kRowBox;
         if (kMode == 0 && prm.streaming) {
           const int32_t t_end = (row0 + rows - 1) / prm.tile;
           for (int32_t t = row0 / prm.tile; t <= t_end && !*abort; ++t) {
@@ -151,28 +199,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_global();
           if (*abort) break;
         }
-        const int32_t brow = e * prm.k_rows;
+        const int32_t wcol0 = nb * prm.col_step;
+        const int32_t wcol1 = wcol0 + prm.col1_off;
+        const uint32_t tx = (uint32_t)(2 * kWTileBytes + nbox * kRowBoxBytes);
         for (int kb = 0; kb < kb_count; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1u, 2 * prm.timeout_ns, abort)) {
             raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, (int32_t)u);
             break;
           }
-          uint8_t *sa = smem + stage * kStageBytes;
-          uint8_t *sb = sa + kABytes;
-          mbar_arrive_expect_tx(full + stage, stage_tx);
-          tma_load_2d(sa, &tm_a, full + stage, kb * kBK, row0);
-          const int32_t krow = brow + kb * kBK;
-          if (kMode == 0) {
-            const int half = n_chunks / 2;
-            for (int c = 0; c < half; ++c)
-              tma_load_2d(sb + c * kChunkBytes, &tm_b, full + stage, nb * prm.bn + c * 64, krow);
-            for (int c = 0; c < half; ++c)
-              tma_load_2d(sb + (half + c) * kChunkBytes, &tm_b, full + stage,
-                          prm.up_col + nb * prm.bn + c * 64, krow);
-          } else {
-            for (int c = 0; c < n_chunks; ++c)
-              tma_load_2d(sb + c * kChunkBytes, &tm_b, full + stage, nb * prm.bn + c * 64, krow);
-          }
+          uint8_t *sw0 = smem + stage * kStageBytes;
+          uint8_t *sw1 = sw0 + kWTileBytes;
+          uint8_t *sx = sw0 + 2 * kWTileBytes;
+          const int32_t krow = e * prm.k_rows + kb * kBK;
+          mbar_arrive_expect_tx(full + stage, tx);
+          tma_load_2d(sw0, &tm_w, full + stage, wcol0, krow);
+          tma_load_2d(sw0 + kChunkBytes, &tm_w, full + stage, wcol0 + 64, krow);
+          tma_load_2d(sw1, &tm_w, full + stage, wcol1, krow);
+          tma_load_2d(sw1 + kChunkBytes, &tm_w, full + stage, wcol1 + 64, krow);
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d(sx + i * kRowBoxBytes, &tm_x, full + stage, kb * kBK, row0 + i * kRowBox);
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -186,23 +231,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s)
           if (issued & (1u << s))
             mbar_wait(full + s, (last_parity >> s) & 1u, prm.timeout_ns, never);
+      } else {
+        // Every CTA has taken its end ticket before it counts itself done, so the last
+        // one may zero the counters for the next launch.
+        __threadfence();
+        if (atomicAdd(prm.sched + 1, 1) == (int)gridDim.x - 1) {
+          atomicExch(prm.sched + 0, 0);
+          atomicExch(prm.sched + 1, 0);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(kBM, (uint32_t)mma_n, true);
       uint32_t stage = 0, phase = 0, local = 0;
-      for (int64_t u = blockIdx.x; u < n_units && !*abort; u += gridDim.x, ++local) {
-        const uint32_t b = local & 1u;
-        const uint32_t acc_phase = (local >> 1) & 1u;
-        if (!mbar_wait(acc_empty + b, acc_phase ^ 1u, 2 * prm.timeout_ns, abort)) {
+      uint32_t sslot = 0, sphase = 0;
+      bool ok = true;
+      for (;; ++local) {
+        if (!mbar_wait(sched_full + sslot, sphase, 2 * prm.timeout_ns, abort)) {
+          raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+          break;
+        }
+        const int32_t u = sched[sslot];
+        mbar_arrive(sched_empty + sslot);
+        if (++sslot == kSchedSlots) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (u < 0) break;
+        const int mb = u / prm.n_blocks;
+        const int32_t rows = prm.mblk[3 * mb + 2];
+        const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32_ab(kBM, n_mma, /*a_mn=*/true, /*b_mn=*/false);
+        // The accumulators may be overwritten once the epilogue read the previous unit
+        // (parity of the previous unit; a fresh barrier passes parity 1).
+        if (!mbar_wait(acc_empty, (local + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
           raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, (int32_t)u);
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + b * kAccStride;
-        bool ok = true;
         for (int kb = 0; kb < kb_count; ++kb) {
           if (!mbar_wait(full + stage, phase, 2 * prm.timeout_ns, abort)) {
             raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, (int32_t)u);
@@ -210,15 +277,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-          const uint32_t sb = sa + kABytes;
+          const uint32_t sw0 = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sw1 = sw0 + kWTileBytes;
+          const uint32_t sx = sw0 + 2 * kWTileBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            // A: K-major, 128-byte rows, 8-row groups 1024 B apart; +32 B per 16 k.
-            const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
-            // B: MN-major, 64-column chunks kChunkBytes apart, 8 k-rows per 1024 B; +2048 B per 16 k.
-            const uint64_t bdesc = smem_desc_sw128(sb + kk * 2048, kChunkBytes, 1024);
-            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            // weights: MN-major, 64-column chunks kChunkBytes apart, 8 k-rows per 1024 B;
+            // +2048 B per 16 k. Pool rows: K-major, 128-byte rows, 8-row groups 1024 B
+            // apart; +32 B per 16 k.
+            const uint64_t xdesc = smem_desc_sw128(sx + kk * 32, 16, 1024);
+            const uint64_t w0 = smem_desc_sw128(sw0 + kk * 2048, kChunkBytes, 1024);
+            const uint64_t w1 = smem_desc_sw128(sw1 + kk * 2048, kChunkBytes, 1024);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            tc_mma_bf16(tmem_base, w0, xdesc, idesc, acc);
+            tc_mma_bf16(tmem_base + kAccStride, w1, xdesc, idesc, acc);
           }
           tc_commit(empty + stage);
           if (++stage == kStages) {
@@ -227,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit(acc_full + b);
+        tc_commit(acc_full);
       }
       // Wait for every MMA issued by this thread before the TMEM is released.
       tc_commit(drain);
@@ -235,70 +307,88 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // accumulator row = TMEM lane
+    // Lane f of a warp holds output column f of its 32-column group for 32 pool rows
+    // at a time; the warp turns that 32x32 block around in shared memory so that
+    // every global store writes 16 contiguous bytes of one pool row.
+    const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+    const int half = (warp - 2) >> 2;          // which 32-row groups it takes
+    const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
+    uint16_t *xp = reinterpret_cast<uint16_t *>(smem + kStages * kStageBytes + kBarrierBytes) +
+                   (warp - 2) * (kXposeBytes / 2);
     uint32_t local = 0;
-    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
-      const int mb = (int)(u / prm.n_blocks);
-      const int nb = (int)(u % prm.n_blocks);
+    uint32_t sslot = 0, sphase = 0;
+    for (;; ++local) {
+      int32_t u = -1;
+      int got = 1;
+      if (lane == 0) {
+        got = mbar_wait(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort) ? 1 : 0;
+        if (got) {
+          u = sched[sslot];
+          mbar_arrive(sched_empty + sslot);
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (++sslot == kSchedSlots) {
+        sslot = 0;
+        sphase ^= 1u;
+      }
+      if (!got) {
+        if (lane == 0) raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+        break;
+      }
+      if (u < 0) break;
+      const int mb = u / prm.n_blocks;
+      const int nb = u % prm.n_blocks;
       const int32_t row0 = prm.mblk[3 * mb + 0];
       const int32_t rows = prm.mblk[3 * mb + 2];
-      const uint32_t b = local & 1u;
-      const uint32_t acc_phase = (local >> 1) & 1u;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(acc_full + b, acc_phase, 3 * prm.timeout_ns, abort) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait(acc_full, local & 1u, 3 * prm.timeout_ns, abort) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, (int32_t)u);
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + b * kAccStride;
-      const bool row_ok = r < rows;
-      uint16_t *orow = prm.out + (size_t)(row0 + r) * prm.out_ld + (size_t)nb * prm.bn;
-      if (kMode == 0) {
-        for (int c = 0; c < prm.bn; c += 32) {
-          uint32_t g[32], v[32];
+      // first output column of this warp's group for accumulator 0 / 1
+      const int32_t cb0 = nb * prm.col_step + quad * 32;
+      const int32_t cb1 = cb0 + prm.col1_off;
+      const bool ok0 = cb0 < prm.n_out;
+      const bool ok1 = kMode == 1 && cb1 < prm.n_out;
+      for (int c = half * 32; c < rows; c += 64) {
+        uint32_t a0[32], a1[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tq + c, a0);
+        tmem_ld_32x32b_x32(tq + kAccStride + c, a1);
+        tmem_ld_wait();
+        const int lim = min(32, rows - c);
+        for (int j = 0; j < (kMode == 0 ? 1 : 2); ++j) {
+          if (!(j == 0 ? ok0 : ok1)) continue;  // uniform across the warp
           __syncwarp();
-          tmem_ld_32x32b_x32(taddr + c, g);
-          tmem_ld_32x32b_x32(taddr + prm.bn + c, v);
-          tmem_ld_wait();
-          if (row_ok) {
-            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-              const float u0 = __uint_as_float(v[2 * i]), u1 = __uint_as_float(v[2 * i + 1]);
-              const float a0 = g0 / (1.0f + __expf(-g0)) * u0;
-              const float a1 = g1 / (1.0f + __expf(-g1)) * u1;
-              pk[i] = pack_bf16x2(a0, a1);
-            }
-            uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 32; ++i) {
+            const float v = kMode == 0
+                                ? silu_mul(__uint_as_float(a0[i]), __uint_as_float(a1[i]))
+                                : __uint_as_float(j == 0 ? a0[i] : a1[i]);
+            xp[i * 32 + lane] = bf16_bits(v);
           }
-        }
-      } else {
-        for (int c = 0; c < prm.bn; c += 32) {
-          uint32_t y[32];
           __syncwarp();
-          tmem_ld_32x32b_x32(taddr + c, y);
-          tmem_ld_wait();
-          if (row_ok) {
-            uint32_t pk[16];
+          const int32_t cb = j == 0 ? cb0 : cb1;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
-            uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int q = 0; q < 4; ++q) {
+            const int v = lane + 32 * q;
+            const int r = v >> 2;         // pool row inside the 32-row group
+            const int part = v & 3;       // 8-column part of the 32 columns
+            if (r < lim) {
+              const uint4 val = *reinterpret_cast<const uint4 *>(xp + r * 32 + part * 8);
+              *reinterpret_cast<uint4 *>(prm.out + (size_t)(row0 + c + r) * prm.out_ld + cb +
+                                         part * 8) = val;
+            }
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(acc_empty + b);
+      mbar_arrive(acc_empty);
     }
   }
 
@@ -347,7 +437,7 @@ static bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t
 }
 
 template <int kMode>
-static cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const FfnParams &prm,
+static cudaError_t launch_one(const CUtensorMap &tw, const CUtensorMap &tx, const FfnParams &prm,
                               int grid, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -359,7 +449,7 @@ static cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, cons
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  ffn_gemm_kernel<kMode><<<grid, kThreads, kSmemBytes, st>>>(ta, tb, prm);
+  ffn_gemm_kernel<kMode><<<grid, kThreads, kSmemBytes, st>>>(tw, tx, prm);
   return cudaGetLastError();
 }
 
@@ -368,11 +458,11 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
                int num_sms, cudaStream_t st) {
   const PlanGeom g = plan_geom(s);
   if (g.pmax == 0) return MOE_OK;
-  CUtensorMap ta_pool, tb_w1, ta_act, tb_w2;
-  if (!make_tmap(&ta_pool, pool, (uint64_t)s.H, (uint64_t)g.pmax, kBM) ||
-      !make_tmap(&tb_w1, W1, 2ull * s.I, (uint64_t)s.E * s.H, kBK) ||
-      !make_tmap(&ta_act, act, (uint64_t)s.I, (uint64_t)g.pmax, kBM) ||
-      !make_tmap(&tb_w2, W2, (uint64_t)s.H, (uint64_t)s.E * s.I, kBK))
+  CUtensorMap tw1, tx_pool, tw2, tx_act;
+  if (!make_tmap(&tw1, W1, 2ull * s.I, (uint64_t)s.E * s.H, kBK) ||
+      !make_tmap(&tx_pool, pool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
+      !make_tmap(&tw2, W2, (uint64_t)s.H, (uint64_t)s.E * s.I, kBK) ||
+      !make_tmap(&tx_act, act, (uint64_t)s.I, (uint64_t)g.pmax, kRowBox))
     return MOE_ERR_CUDA;
 
   int grid = cfg.ffn_ctas > 0 ? cfg.ffn_ctas : (cfg.streaming ? num_sms - 16 : num_sms);
@@ -388,16 +478,18 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   a.out = static_cast<uint16_t *>(act);
   a.out_ld = s.I;
   a.K = s.H;
-  a.bn = (s.I % 128 == 0) ? 128 : 64;
-  a.n_blocks = s.I / a.bn;
+  a.col_step = kBM;                       // 128 gate columns and the same 128 up columns
+  a.col1_off = s.I;
+  a.n_blocks = (s.I + kBM - 1) / kBM;
+  a.n_out = s.I;
   a.k_rows = s.H;
-  a.up_col = s.I;
   a.tile = s.tile;
   a.streaming = cfg.streaming;
+  a.sched = p.meta + 4;
   a.timeout_ns = timeout_ns;
   cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(cfg.timing_events);
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t e = launch_one<0>(ta_pool, tb_w1, a, grid, st);
+  cudaError_t e = launch_one<0>(tw1, tx_pool, a, grid, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -405,12 +497,14 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   y.out = static_cast<uint16_t *>(ypool);
   y.out_ld = s.H;
   y.K = s.I;
-  y.bn = (s.H % 256 == 0) ? 256 : ((s.H % 128 == 0) ? 128 : 64);
-  y.n_blocks = s.H / y.bn;
+  y.col_step = 2 * kBM;                   // two adjacent 128-column blocks of W2
+  y.col1_off = kBM;
+  y.n_blocks = (s.H + 2 * kBM - 1) / (2 * kBM);
+  y.n_out = s.H;
   y.k_rows = s.I;
-  y.up_col = 0;
   y.streaming = 0;
-  e = launch_one<1>(ta_act, tb_w2, y, cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms, st);
+  y.sched = p.meta + 6;
+  e = launch_one<1>(tw2, tx_act, y, cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;

@@ -61,7 +61,7 @@ void plan_sizes(const moe_shape &s, size_t words[10]) {
   words[3] = (size_t)g.pmax;
   words[4] = (size_t)g.n_tiles;
   words[5] = 3 * (size_t)g.n_tiles;
-  words[6] = 4;
+  words[6] = 8;
   words[7] = (size_t)g.n_tiles;
   words[8] = plan_workspace_ints(s);
   words[9] = 4;

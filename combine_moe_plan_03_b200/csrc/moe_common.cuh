@@ -203,12 +203,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, A K-major, B MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bool b_mn_major) {
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D; A / B K-major or MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(uint32_t M, uint32_t N, bool a_mn_major,
+                                                         bool b_mn_major) {
   return (1u << 4)                              // D format: f32
          | (1u << 7)                            // A format: bf16
          | (1u << 10)                           // B format: bf16
-         | (0u << 15)                           // A major: K
+         | ((a_mn_major ? 1u : 0u) << 15)       // A major
          | ((b_mn_major ? 1u : 0u) << 16)       // B major
          | ((N >> 3) << 17)                     // N / 8
          | ((M >> 4) << 24);                    // M / 16

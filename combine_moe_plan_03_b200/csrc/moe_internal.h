@@ -14,7 +14,15 @@ constexpr int kPlanChunk = 256;
 constexpr int kPlanWarps = 8;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
-constexpr int kGemmBlockM = 128;
+constexpr int kGemmBlockM = 256;  // most live rows of one expert in one grouped-GEMM unit
+
+// Rows per grouped-GEMM chunk for an expert with c live rows: the rows are cut into
+// ceil(c / 256) chunks of equal size, rounded up to a multiple of 16 (the MMA's N step).
+__host__ __device__ inline int32_t gemm_chunk_rows(int32_t c) {
+  if (c <= 0) return kGemmBlockM;
+  const int32_t n = (c + kGemmBlockM - 1) / kGemmBlockM;
+  return ((c + n - 1) / n + 15) & ~15;
+}
 
 struct PlanGeom {
   int64_t pairs;     // T * k

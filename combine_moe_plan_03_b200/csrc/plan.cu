@@ -10,7 +10,10 @@
 //                      chunks (the chunk's base inside the expert), counts[e].
 //                      The last block to finish pads the counts to the tile,
 //                      scans them into offsets, and writes tile_expert, the GEMM
-//                      row-block table and meta.
+//                      row-chunk table and meta. An expert's live rows are cut into
+//                      ceil(count/256) chunks of equal size (a multiple of 16), so
+//                      the grouped GEMM's units of one expert run at the same pace
+//                      and share each weight tile through L2.
 //   plan_rank_kernel   each warp walks its chunk again 32 pairs at a time;
 //                      __match_any_sync groups lanes with the same expert and the
 //                      rank inside the group is the popcount of lower lanes, so
@@ -143,7 +146,8 @@ __global__ void __launch_bounds__(256)
     const int32_t c = __ldcg(counts + x);
     const int32_t pad = (c + tile - 1) / tile * tile;
     my_rows += pad;
-    my_blk += (pad + kGemmBlockM - 1) / kGemmBlockM;
+    const int32_t chunk = gemm_chunk_rows(c);
+    if (c > 0) my_blk += (c + chunk - 1) / chunk;
   }
   int32_t tot_rows, tot_blk;
   int32_t row = block_excl_scan(my_rows, warp_sums, &tot_rows);
@@ -153,10 +157,11 @@ __global__ void __launch_bounds__(256)
     const int32_t pad = (c + tile - 1) / tile * tile;
     offsets[x] = row;
     for (int32_t r = 0; r < pad; r += tile) tile_expert[(row + r) / tile] = x;
-    for (int32_t r = 0; r < pad; r += kGemmBlockM) {
+    const int32_t chunk = gemm_chunk_rows(c);
+    for (int32_t r = 0; r < c; r += chunk) {  // live rows only: padding is not computed
       mblk[3 * blk + 0] = row + r;
       mblk[3 * blk + 1] = x;
-      mblk[3 * blk + 2] = min(kGemmBlockM, pad - r);
+      mblk[3 * blk + 2] = min(chunk, c - r);
       ++blk;
     }
     row += pad;
@@ -167,6 +172,7 @@ __global__ void __launch_bounds__(256)
     meta[1] = tot_rows;
     meta[2] = tot_blk;
     meta[3] = 0;
+    for (int i = 4; i < 8; ++i) meta[i] = 0;  // grouped-GEMM unit counters
     if ((int64_t)tot_rows > pmax) report(status, MOE_ERR_POOL_OVERFLOW, tot_rows);
   }
 }

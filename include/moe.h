@@ -83,8 +83,9 @@ typedef struct moe_plan_buffers {
   int32_t *pool_row;    /* [T * k]      pool row of pair f, -1 for a dropped pair */
   int32_t *row_src;     /* [P_max]      pair id of pool row p, -1 for padding */
   int32_t *tile_expert; /* [P_max/tile] expert of pool tile i, -1 past P/tile */
-  int32_t *mblk;        /* [3 * P_max/tile] GEMM row blocks: {row_start, expert, rows} */
-  int32_t *meta;        /* [4]          num_tiles, P, num_mblk, 0 */
+  int32_t *mblk;        /* [3 * P_max/tile] GEMM row chunks: {row_start, expert, live rows <= 256} */
+  int32_t *meta;        /* [8]          num_tiles, P, number of row chunks, 0, and four
+                                        grouped-GEMM unit counters (zeroed by moe_plan) */
   uint32_t *tile_flags; /* [P_max/tile] rows landed per tile (streaming) */
   int32_t *workspace;   /* plan scratch: per-(expert, 256-pair chunk) counts + 1 counter */
   int32_t *status;      /* [4]          code, aux, 0, 0 (first device error wins) */
@@ -146,7 +147,8 @@ int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, v
  * compute kernels": grouped GEMM A then grouped GEMM Y), tcgen05 tensor cores:
  *   act[p]   = bf16( silu(pool[p] W1[e]_gate) * (pool[p] W1[e]_up) )   (fp32 accumulate)
  *   ypool[p] = bf16( act[p] W2[e] )                                     (fp32 accumulate)
- * for every row p < P, e = the expert of p's tile. Padding rows give zeros.
+ * for every live row p (a row that holds a routed pair), e = the expert of p's
+ * segment. Padding rows of act and ypool are not written (combine never reads them).
  * With cfg->streaming the first GEMM waits (bounded) until tile_flags[tile] == tile
  * for each tile it reads, so it may be launched while moe_dispatch is still running
  * on another stream; otherwise it must be ordered after moe_dispatch.

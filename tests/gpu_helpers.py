@@ -63,13 +63,17 @@ def check_plan_exact(buf, ref, T, k):
                                   ref["tile_expert"])
     meta = buf.plan_view("meta")[:4].cpu().numpy()
     assert meta[0] == P // buf.shape.tile and meta[1] == P
-    # GEMM row blocks: 128-row blocks covering each expert's padded segment, in order
+    # GEMM row chunks: an expert's live rows in ceil(c/256) equal chunks (multiples of 16)
     mb = buf.plan_view("mblk")[: 3 * meta[2]].cpu().numpy().reshape(-1, 3)
     want = []
     for e in range(E):
-        a, b = ref["offsets"][e], ref["offsets"][e + 1]
-        for r in range(a, b, 128):
-            want.append((r, e, min(128, b - r)))
+        a, c = int(ref["offsets"][e]), int(ref["counts"][e])
+        if c == 0:
+            continue
+        n = -(-c // 256)
+        step = (-(-c // n) + 15) // 16 * 16
+        for r in range(a, a + c, step):
+            want.append((r, e, min(step, a + c - r)))
     np.testing.assert_array_equal(mb, np.array(want, np.int64).reshape(-1, 3))
 
 

@@ -39,6 +39,8 @@ SHAPES = [
     ("H128-I192", 150, 128, 192, 5, 3, 128),    # GEMM Y N=128, GEMM A half width 64
     ("one-expert", 130, 320, 384, 1, 1, 128),
     ("deep-K", 64, 1024, 256, 2, 2, 64),
+    ("pairs-tile64", 500, 128, 128, 3, 2, 64),     # 256-row units plus 64/128/192-row tails
+    ("pairs-tile128", 700, 256, 128, 3, 2, 128),   # pair units and single 128-row units
 ]
 
 
@@ -76,9 +78,9 @@ def test_tiny_config_all_tokens_and_act():
                                              si.make_w2_expert(cfg, e))
         p = plan["pool_row"][t, j]
         assert np.abs(act[p] - a).max() <= 2e-2 * np.abs(a).max()
-    # padding rows of the pool give zero act
-    pad = plan["row_src"][: plan["P"]] < 0
-    assert np.all(act[pad] == 0)
+    # every live row of act is finite (padding rows are not computed)
+    live = plan["row_src"][: plan["P"]] >= 0
+    assert np.isfinite(act[live]).all()
     buf.close()
 
 
