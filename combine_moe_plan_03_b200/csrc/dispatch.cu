@@ -4,94 +4,178 @@
 // tile's flag counts the rows that have landed (release order), so the grouped
 // GEMM can claim a tile as soon as its flag reaches the tile height.
 //
-// One block of 128 threads per work item, grid-stride over E + T items:
-//   item e < E    zero the padding rows of expert e (all in its last tile)
-//   item E + t    read x[t] once (16-byte vectors, no L1 allocation) and write it
-//                 to the k pool rows of token t
+// Rows move as whole-row bulk copies staged in shared memory: one bulk load of
+// x[t] (H*2 bytes) into a shared buffer, then one bulk store of that buffer per
+// pool row of the token; padding rows are bulk-stored from a zeroed shared row.
+// Each block is one warp: lane j reads the token's j-th pool row id, lane 0 issues
+// the copies; two staging buffers let the load of the block's next token overlap
+// the stores of the current one.
+// Work items, grid-stride over E + T:
+//   item e < E    the padding rows of expert e (all in its last tile)
+//   item E + t    token t
 // HBM traffic per call: T*H*2 read + (live pairs + padding rows)*H*2 written.
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
 namespace moe {
 
-constexpr int kDispThreads = 128;
-constexpr int kDispVec = 8;  // 16-byte vectors per thread held in registers per pass
-
-__device__ __forceinline__ uint4 ld_stream_v4(const uint4 *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+__device__ __forceinline__ void bulk_load_row(void *dst_smem, const void *src, uint32_t bytes,
+                                              uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst_smem)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
-__global__ void __launch_bounds__(kDispThreads)
-    dispatch_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ pool_row,
+__device__ __forceinline__ void bulk_store_row(void *dst, const void *src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src_smem)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// All but the newest `n` committed groups have finished reading their shared sources.
+template <int n>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(n) : "memory");
+}
+
+// All committed groups are complete (their global writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(32)
+    dispatch_kernel(const uint8_t *__restrict__ x, const int32_t *__restrict__ pool_row,
                     const int32_t *__restrict__ offsets, const int32_t *__restrict__ counts,
-                    uint4 *__restrict__ pool, uint32_t *__restrict__ flags, int32_t T, int32_t k,
-                    int32_t E, int32_t hv, int32_t tile, int32_t signal) {
-  __shared__ int32_t s_rows[kMaxTopK];
-  const int tid = threadIdx.x;
+                    uint8_t *__restrict__ pool, uint32_t *__restrict__ flags, int32_t T, int32_t k,
+                    int32_t E, uint32_t row_bytes, int32_t tile, int32_t signal,
+                    uint64_t timeout_ns, int32_t *__restrict__ status) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint8_t *zeros = sm + 2 * row_bytes;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 3 * row_bytes);
+  int *never = reinterpret_cast<int *>(bar + 2);
+  const int lane = threadIdx.x;
+
+  for (uint32_t i = lane * 16; i < row_bytes; i += 32 * 16)
+    *reinterpret_cast<uint4 *>(zeros + i) = make_uint4(0u, 0u, 0u, 0u);
+  if (lane == 0) {
+    mbar_init(bar + 0, 1);
+    mbar_init(bar + 1, 1);
+    *never = 0;
+    fence_mbarrier_init();
+  }
+  fence_proxy_async_shared();  // the zeros and barriers, written by threads, are read by bulk copies
+  __syncwarp();
+
   const int64_t items = (int64_t)E + T;
-  for (int64_t w = blockIdx.x; w < items; w += gridDim.x) {
+  const int64_t G = gridDim.x;
+  // Lane 0 issues every copy. Token loads alternate between two staging buffers; the
+  // load of the block's next token is issued before the current token's stores.
+  uint32_t uses[2] = {0u, 0u};     // loads issued into each buffer so far
+  uint32_t cur = 0;                // buffer holding the current token (if prefetched)
+  bool have = false;               // the current token's load was already issued
+  bool failed = false;
+  for (int64_t w = blockIdx.x; w < items && !failed; w += G) {
     if (w < E) {
-      const int e = (int)w;
-      const int32_t start = offsets[e] + counts[e];
-      const int32_t end = offsets[e + 1];
-      const int32_t npad = end - start;
-      if (npad <= 0) continue;  // uniform across the block
-      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-      for (int32_t r = 0; r < npad; ++r) {
-        uint4 *dst = pool + (size_t)(start + r) * hv;
-        for (int v = tid; v < hv; v += kDispThreads) dst[v] = z;
-      }
-      if (signal) {
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) red_release_gpu_add(flags + (end - 1) / tile, (uint32_t)npad);
-      }
-    } else {
-      const int64_t t = w - E;
-      if (tid < k) s_rows[tid] = pool_row[t * k + tid];
-      __syncthreads();
-      const uint4 *src = x + (size_t)t * hv;
-      for (int v0 = 0; v0 < hv; v0 += kDispThreads * kDispVec) {
-        uint4 buf[kDispVec];
-#pragma unroll
-        for (int i = 0; i < kDispVec; ++i) {
-          const int v = v0 + i * kDispThreads + tid;
-          if (v < hv) buf[i] = ld_stream_v4(src + v);
-        }
-        for (int j = 0; j < k; ++j) {
-          const int32_t p = s_rows[j];
-          if (p < 0) continue;
-          uint4 *dst = pool + (size_t)p * hv;
-#pragma unroll
-          for (int i = 0; i < kDispVec; ++i) {
-            const int v = v0 + i * kDispThreads + tid;
-            if (v < hv) dst[v] = buf[i];
+      if (lane == 0) {
+        const int e = (int)w;
+        const int32_t start = offsets[e] + counts[e];
+        const int32_t end = offsets[e + 1];
+        if (end > start) {
+          for (int32_t r = start; r < end; ++r)
+            bulk_store_row(pool + (size_t)r * row_bytes, zeros, row_bytes);
+          bulk_commit();
+          if (signal) {
+            bulk_wait_all();
+            fence_proxy_async_global();
+            red_release_gpu_add(flags + (end - 1) / tile, (uint32_t)(end - start));
           }
         }
       }
-      if (signal) {
-        __threadfence();
-        __syncthreads();
-        if (tid < k && s_rows[tid] >= 0) red_release_gpu_add(flags + s_rows[tid] / tile, 1u);
+      continue;
+    }
+    const int64_t t = w - E;
+    const int32_t my_row = lane < k ? pool_row[t * k + lane] : -1;
+    if (lane == 0) {
+      if (!have) {
+        bulk_wait_read<0>();  // nothing may still read the buffer that is about to be filled
+        mbar_arrive_expect_tx(bar + cur, row_bytes);
+        bulk_load_row(sm + cur * row_bytes, x + (size_t)t * row_bytes, row_bytes, bar + cur);
+        ++uses[cur];
+      }
+      const int64_t wn = w + G;
+      const uint32_t nxt = cur ^ 1u;
+      const bool prefetch = wn < items && wn >= E;
+      if (prefetch) {
+        bulk_wait_read<0>();  // the previous token's stores have read the other buffer
+        mbar_arrive_expect_tx(bar + nxt, row_bytes);
+        bulk_load_row(sm + nxt * row_bytes, x + (size_t)(wn - E) * row_bytes, row_bytes,
+                      bar + nxt);
+        ++uses[nxt];
+      }
+      if (!mbar_wait(bar + cur, (uses[cur] - 1u) & 1u, timeout_ns, never)) {
+        report(status, MOE_ERR_PIPE_TIMEOUT, (int32_t)t);
+        failed = true;
+      }
+      have = prefetch;
+    }
+    failed = __shfl_sync(0xffffffffu, failed ? 1 : 0, 0) != 0;
+    if (failed) break;
+    for (int j = 0; j < k; ++j) {
+      const int32_t p = __shfl_sync(0xffffffffu, my_row, j);
+      if (lane == 0 && p >= 0)
+        bulk_store_row(pool + (size_t)p * row_bytes, sm + cur * row_bytes, row_bytes);
+    }
+    if (lane == 0) bulk_commit();
+    if (signal) {
+      // the rows must have landed before their tiles are counted (by the thread that
+      // issued and waited for the writes)
+      if (lane == 0) {
+        bulk_wait_all();
+        fence_proxy_async_global();
+      }
+      for (int j = 0; j < k; ++j) {
+        const int32_t p = __shfl_sync(0xffffffffu, my_row, j);
+        if (lane == 0 && p >= 0) red_release_gpu_add(flags + p / tile, 1u);
       }
     }
-    __syncthreads();  // s_rows is rewritten by the next item
+    cur ^= 1u;
+  }
+  if (lane == 0) {
+    // a prefetched load that was never consumed must land before the block exits
+    if (have) mbar_wait(bar + cur, (uses[cur] - 1u) & 1u, timeout_ns, never);
+    bulk_wait_all();
   }
 }
 
 cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_buffers &p,
                             void *pool, int signal, int num_sms, cudaStream_t st) {
+  const uint32_t row_bytes = (uint32_t)s.H * 2;
+  const size_t smem = 3 * (size_t)row_bytes + 2 * sizeof(uint64_t) + 16;
+  static size_t attr_smem[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (attr_smem[dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(dispatch_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_smem[dev] = smem;
+  }
+  const int per_sm = (int)(200 * 1024 / smem) > 0 ? (int)(200 * 1024 / smem) : 1;
   const int64_t items = (int64_t)s.E + s.T;
-  int64_t grid = (int64_t)num_sms * 8;
+  int64_t grid = (int64_t)num_sms * (per_sm < 16 ? per_sm : 16);
   if (grid > items) grid = items;
   if (grid < 1) grid = 1;
-  dispatch_kernel<<<(int)grid, kDispThreads, 0, st>>>(
-      static_cast<const uint4 *>(x), p.pool_row, p.offsets, p.counts, static_cast<uint4 *>(pool),
-      p.tile_flags, s.T, s.k, s.E, s.H / 8, s.tile, signal);
+  dispatch_kernel<<<(int)grid, 32, smem, st>>>(
+      static_cast<const uint8_t *>(x), p.pool_row, p.offsets, p.counts,
+      static_cast<uint8_t *>(pool), p.tile_flags, s.T, s.k, s.E, row_bytes, s.tile, signal,
+      2000000000ull, p.status);
   return cudaGetLastError();
 }
 
