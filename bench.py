@@ -487,7 +487,13 @@ def run_moe(args):
     hx = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in xs]
     hidx = [torch.from_numpy(a).pin_memory() for a in idxs]
     hw = [torch.from_numpy(a).pin_memory() for a in ws]
-    hout = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    hout = [torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    # results go back on a copy stream from two device output buffers, so the copy of one
+    # call's result overlaps the next call
+    dout = [torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    copy_stream = torch.cuda.Stream(dev)
+    done_ev = [torch.cuda.Event() for _ in range(2)]
+    copied_ev = [torch.cuda.Event() for _ in range(2)]
     # two device copies of each input, so the copy of the next call's inputs (comm stream)
     # never overwrites what the current call's combine (compute stream) still reads
     bx = [torch.empty_like(dx[0]) for _ in range(2)]
@@ -503,9 +509,13 @@ def run_moe(args):
                 bx[j].copy_(hx[m], non_blocking=True)
                 bi[j].copy_(hidx[m], non_blocking=True)
                 bw[j].copy_(hw[m], non_blocking=True)
-            buf.forward(bx[j], bi[j], bw[j], W1, W2, plain)
-            with torch.cuda.stream(buf.compute):
-                hout.copy_(buf.out[: cfg.T], non_blocking=True)
+            buf.compute.wait_event(copied_ev[j])   # dout[j] was copied out two calls ago
+            buf.forward(bx[j], bi[j], bw[j], W1, W2, plain, out=dout[j])
+            done_ev[j].record(buf.compute)
+            copy_stream.wait_event(done_ev[j])
+            with torch.cuda.stream(copy_stream):
+                hout[j].copy_(dout[j], non_blocking=True)
+            copied_ev[j].record(copy_stream)
 
     for _ in range(2):
         e2e_step()
@@ -516,6 +526,7 @@ def run_moe(args):
     s_ev.record(buf.comm)
     for _ in range(args.steps):
         e2e_step()
+    buf.compute.wait_stream(copy_stream)
     e_ev.record(buf.compute)
     torch.cuda.synchronize()
     e2e_ms = reduce_max([s_ev.elapsed_time(e_ev)], dev, world)[0]

@@ -65,10 +65,14 @@ class MoELayerBuffers:
 
     def forward(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
                 W1: torch.Tensor | None, W2: torch.Tensor | None,
-                cfg: moe_config | None = None) -> torch.Tensor:
+                cfg: moe_config | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
         """Enqueue the layer (plan + dispatch on comm, FFN + combine on compute).
-        Returns ``out`` [T, H]; it is ready once the compute stream reaches this point."""
+        Writes ``out`` [T, H] bf16 (default: this object's own buffer) and returns it; it is
+        ready once the compute stream reaches this point."""
         s = self.shape
+        if out is None:
+            out = self.out[: s.T]
+        assert out.dtype == torch.bfloat16 and tuple(out.shape) == (s.T, s.H) and out.is_contiguous()
         assert x.dtype == torch.bfloat16 and tuple(x.shape) == (s.T, s.H) and x.is_contiguous()
         assert topk_idx.dtype == torch.int32 and tuple(topk_idx.shape) == (s.T, s.k)
         assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (s.T, s.k)
@@ -80,7 +84,7 @@ class MoELayerBuffers:
             w1, w2 = W1.data_ptr(), W2.data_ptr()
             act, ypool = self.act.data_ptr(), self.ypool.data_ptr()
         moe_forward(s, x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), w1, w2, self.plan,
-                    self.pool.data_ptr(), act, ypool, self.out.data_ptr(), cfg,
+                    self.pool.data_ptr(), act, ypool, out.data_ptr(), cfg,
                     self.comm.cuda_stream, self.compute.cuda_stream, self.events[0],
                     self.events[1])
-        return self.out[: s.T]
+        return out
