@@ -46,7 +46,7 @@ class moe_plan_buffers(ctypes.Structure):
 
 class moe_config(ctypes.Structure):
     _fields_ = [("streaming", ctypes.c_int32), ("ffn_ctas", ctypes.c_int32),
-                ("wait_timeout_us", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("wait_timeout_us", ctypes.c_int32), ("packed_weights", ctypes.c_int32),
                 ("timing_events", ctypes.c_void_p)]
 
 
@@ -82,6 +82,8 @@ def _load():
         "moe_get_status": [P(moe_plan_buffers), P(i32), P(i32)],
         "moe_clear_status": [P(moe_plan_buffers), vp],
         "moe_plan_noalloc": [P(moe_shape), vp, P(moe_plan_buffers), vp, vp],
+        "moe_packed_weight_bytes": [P(moe_shape), P(ctypes.c_size_t), P(ctypes.c_size_t)],
+        "moe_pack_weights": [P(moe_shape), vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -97,7 +99,7 @@ def _load():
 _lib = _load()
 
 # Names exported by include/moe.h, in declaration order.
-EXPORTS = ["moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
+EXPORTS = ["moe_packed_weight_bytes", "moe_pack_weights", "moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
            "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
            "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
@@ -125,6 +127,19 @@ def moe_strerror(code: int) -> str:
 
 def moe_version() -> str:
     return _lib.moe_version().decode()
+
+
+def moe_packed_weight_bytes(shape) -> tuple[int, int]:
+    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check("moe_packed_weight_bytes", _lib.moe_packed_weight_bytes(ctypes.byref(_shape(shape)),
+                                                                   ctypes.byref(a), ctypes.byref(b)))
+    return int(a.value), int(b.value)
+
+
+def moe_pack_weights(shape, w1_ptr: int, w2_ptr: int, w1p_ptr: int, w2p_ptr: int,
+                     stream: int = 0) -> None:
+    _check("moe_pack_weights", _lib.moe_pack_weights(ctypes.byref(_shape(shape)), w1_ptr, w2_ptr,
+                                                     w1p_ptr, w2p_ptr, stream or None))
 
 
 def moe_pool_rows_max(shape) -> int:

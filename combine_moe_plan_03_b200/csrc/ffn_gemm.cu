@@ -31,6 +31,8 @@
 //               32*(w%4)... and every other group of 32 pool rows), tcgen05.ld,
 //               SwiGLU (GEMM A) or conversion (GEMM Y) to bf16, a 32x32 turn in
 //               shared memory, and 16-byte stores along the output rows.
+// With prepacked weights (moe_pack_weights) each weight tile is one contiguous 16 KB
+// box, so a unit streams contiguous HBM.
 // Units are handed out in order (row chunk, then weight block) from a global ticket
 // counter as CTAs free up, so the CTAs working at one time share the same pool rows
 // and the same expert's weights through L2, and uneven units balance out. The
@@ -83,6 +85,8 @@ struct FfnParams {
   int32_t tile;            // pool tile rows
   int32_t streaming;
   int32_t *sched;          // {next unit ticket, CTAs done}: zero at launch, zeroed again at exit
+  int32_t packed;          // weights are moe_pack_weights tiles (one 16 KB box per tile)
+  int32_t pk_e, pk_j, pk_nb;  // packed tile index = e*pk_e + j*pk_j + nb*pk_nb + kb
   uint64_t timeout_ns;
 };
 
@@ -212,10 +216,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t *sx = sw0 + 2 * kWTileBytes;
           const int32_t krow = e * prm.k_rows + kb * kBK;
           mbar_arrive_expect_tx(full + stage, tx);
-          tma_load_2d(sw0, &tm_w, full + stage, wcol0, krow);
-          tma_load_2d(sw0 + kChunkBytes, &tm_w, full + stage, wcol0 + 64, krow);
-          tma_load_2d(sw1, &tm_w, full + stage, wcol1, krow);
-          tma_load_2d(sw1 + kChunkBytes, &tm_w, full + stage, wcol1 + 64, krow);
+          if (prm.packed) {
+            const int32_t t0 = e * prm.pk_e + nb * prm.pk_nb + kb;
+            tma_load_2d(sw0, &tm_w, full + stage, 0, t0 * 128);
+            tma_load_2d(sw1, &tm_w, full + stage, 0, (t0 + prm.pk_j) * 128);
+          } else {
+            tma_load_2d(sw0, &tm_w, full + stage, wcol0, krow);
+            tma_load_2d(sw0 + kChunkBytes, &tm_w, full + stage, wcol0 + 64, krow);
+            tma_load_2d(sw1, &tm_w, full + stage, wcol1, krow);
+            tma_load_2d(sw1 + kChunkBytes, &tm_w, full + stage, wcol1 + 64, krow);
+          }
           for (int i = 0; i < nbox; ++i)
             tma_load_2d(sx + i * kRowBoxBytes, &tm_x, full + stage, kb * kBK, row0 + i * kRowBox);
           issued |= 1u << stage;
@@ -459,9 +469,17 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   const PlanGeom g = plan_geom(s);
   if (g.pmax == 0) return MOE_OK;
   CUtensorMap tw1, tx_pool, tw2, tx_act;
-  if (!make_tmap(&tw1, W1, 2ull * s.I, (uint64_t)s.E * s.H, kBK) ||
-      !make_tmap(&tx_pool, pool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
-      !make_tmap(&tw2, W2, (uint64_t)s.H, (uint64_t)s.E * s.I, kBK) ||
+  const PackGeom pg = pack_geom(s);
+  bool ok;
+  if (cfg.packed_weights) {
+    // packed tiles: an array of 128-byte rows, one 128-row box per tile
+    ok = make_tmap(&tw1, W1, 64, (uint64_t)pg.tiles1 * 128, 128) &&
+         make_tmap(&tw2, W2, 64, (uint64_t)pg.tiles2 * 128, 128);
+  } else {
+    ok = make_tmap(&tw1, W1, 2ull * s.I, (uint64_t)s.E * s.H, kBK) &&
+         make_tmap(&tw2, W2, (uint64_t)s.H, (uint64_t)s.E * s.I, kBK);
+  }
+  if (!ok || !make_tmap(&tx_pool, pool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
       !make_tmap(&tx_act, act, (uint64_t)s.I, (uint64_t)g.pmax, kRowBox))
     return MOE_ERR_CUDA;
 
@@ -486,6 +504,10 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   a.tile = s.tile;
   a.streaming = cfg.streaming;
   a.sched = p.meta + 4;
+  a.packed = cfg.packed_weights ? 1 : 0;
+  a.pk_e = 2 * pg.nb1 * pg.kb1;           // gate tiles of expert e, then its up tiles
+  a.pk_j = pg.nb1 * pg.kb1;
+  a.pk_nb = pg.kb1;
   a.timeout_ns = timeout_ns;
   cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(cfg.timing_events);
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -504,6 +526,9 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   y.k_rows = s.I;
   y.streaming = 0;
   y.sched = p.meta + 6;
+  y.pk_e = pg.nb2 * pg.kb2;               // 128-column blocks of expert e, k fastest
+  y.pk_j = pg.kb2;
+  y.pk_nb = 2 * pg.kb2;
   e = launch_one<1>(tw2, tx_act, y, cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;

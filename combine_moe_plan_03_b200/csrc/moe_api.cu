@@ -73,6 +73,32 @@ size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
 extern "C" {
 
+int moe_packed_weight_bytes(const moe_shape *s, size_t *w1p_bytes, size_t *w2p_bytes) {
+  int rc = check_shape(s, true);
+  if (rc != MOE_OK) return rc;
+  if (w1p_bytes == nullptr || w2p_bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  const PackGeom g = pack_geom(*s);
+  *w1p_bytes = (size_t)g.tiles1 * 128 * 64 * 2;
+  *w2p_bytes = (size_t)g.tiles2 * 128 * 64 * 2;
+  return MOE_OK;
+}
+
+int moe_pack_weights(const moe_shape *s, const void *W1, const void *W2, void *W1p, void *W2p,
+                     void *stream) {
+  int rc = check_shape(s, true);
+  if (rc != MOE_OK) return rc;
+  if (!W1 || !W2 || !W1p || !W2p) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(W1) || !aligned16(W2) || !aligned16(W1p) || !aligned16(W2p))
+    return MOE_ERR_MISALIGNED;
+  const PackGeom g = pack_geom(*s);
+  if ((g.tiles1 + g.tiles2) * 128 > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  if (launch_pack(*s, W1, W2, W1p, W2p, nsm, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 int moe_pool_rows_max(const moe_shape *s, int64_t *rows_out) {
   int rc = check_shape(s, false);
   if (rc != MOE_OK) return rc;

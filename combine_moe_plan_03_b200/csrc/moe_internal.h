@@ -32,6 +32,16 @@ struct PlanGeom {
 };
 
 PlanGeom plan_geom(const moe_shape &s);
+
+// Prepacked weight tiles (pack.cu): 128 rows of 64 bf16 (16 KB) per tile.
+struct PackGeom {
+  int32_t nb1, kb1;  // W1: 128-column blocks of each of gate / up, 64-row k blocks
+  int32_t nb2, kb2;  // W2: 128-column blocks (even count), 64-row k blocks
+  int64_t tiles1, tiles2;
+};
+PackGeom pack_geom(const moe_shape &s);
+cudaError_t launch_pack(const moe_shape &s, const void *W1, const void *W2, void *W1p, void *W2p,
+                        int num_sms, cudaStream_t st);
 size_t plan_workspace_ints(const moe_shape &s);
 
 cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_plan_buffers &p,

@@ -8,8 +8,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (moe_config, moe_events_create, moe_events_destroy, moe_forward, moe_plan_arena_bytes,
-               moe_plan_bind, moe_pool_rows_max, moe_shape)
+from . import (moe_config, moe_events_create, moe_events_destroy, moe_forward, moe_pack_weights,
+               moe_packed_weight_bytes, moe_plan_arena_bytes, moe_plan_bind, moe_pool_rows_max,
+               moe_shape)
 
 _PLAN_FIELDS = ("counts", "offsets", "pool_row", "row_src", "tile_expert", "mblk", "meta",
                 "tile_flags", "workspace", "status")
@@ -63,6 +64,20 @@ class MoELayerBuffers:
                if i + 1 < len(_PLAN_FIELDS) else self.arena.numel())
         return self.arena[off:end].view(torch.int32)
 
+    def pack_weights(self, W1: torch.Tensor, W2: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+        """One-time prepack of W1 [E,H,2I] / W2 [E,I,H] into the GEMMs' tile layout
+        (moe_pack_weights). Use the results with ``moe_config(packed_weights=1)``."""
+        s = self.shape
+        assert tuple(W1.shape) == (s.E, s.H, 2 * s.I) and W1.dtype == torch.bfloat16
+        assert tuple(W2.shape) == (s.E, s.I, s.H) and W2.dtype == torch.bfloat16
+        b1, b2 = moe_packed_weight_bytes(s)
+        W1p = torch.empty(b1 // 2, dtype=torch.bfloat16, device=self.device)
+        W2p = torch.empty(b2 // 2, dtype=torch.bfloat16, device=self.device)
+        moe_pack_weights(s, W1.data_ptr(), W2.data_ptr(), W1p.data_ptr(), W2p.data_ptr(),
+                         self.compute.cuda_stream)
+        self.compute.synchronize()
+        return W1p, W2p
+
     def forward(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
                 W1: torch.Tensor | None, W2: torch.Tensor | None,
                 cfg: moe_config | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
@@ -79,8 +94,13 @@ class MoELayerBuffers:
         w1 = w2 = act = ypool = 0
         if not self.identity:
             assert W1 is not None and W2 is not None
-            assert tuple(W1.shape) == (s.E, s.H, 2 * s.I) and W1.dtype == torch.bfloat16
-            assert tuple(W2.shape) == (s.E, s.I, s.H) and W2.dtype == torch.bfloat16
+            assert W1.dtype == torch.bfloat16 and W2.dtype == torch.bfloat16
+            if cfg is not None and cfg.packed_weights:
+                b1, b2 = moe_packed_weight_bytes(s)
+                assert W1.numel() * 2 >= b1 and W2.numel() * 2 >= b2
+            else:
+                assert tuple(W1.shape) == (s.E, s.H, 2 * s.I)
+                assert tuple(W2.shape) == (s.E, s.I, s.H)
             w1, w2 = W1.data_ptr(), W2.data_ptr()
             act, ypool = self.act.data_ptr(), self.ypool.data_ptr()
         moe_forward(s, x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), w1, w2, self.plan,

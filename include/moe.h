@@ -98,7 +98,8 @@ typedef struct moe_config {
                               orders the FFN after dispatch. */
   int32_t ffn_ctas;        /* persistent FFN CTAs; 0 = number of SMs (streaming: SMs - 16) */
   int32_t wait_timeout_us; /* bound on every device-side wait; 0 = 2,000,000 us */
-  int32_t reserved;
+  int32_t packed_weights;  /* 1: W1 / W2 passed to moe_grouped_ffn / moe_forward are the
+                              tiles written by moe_pack_weights, not [E,H,2I] / [E,I,H] */
   /* NULL, or 7 cudaEvent_t that moe_forward records at the phase boundaries, each on
      the stream of the kernels around it: [0] comm before plan, [1] comm after plan,
      [2] comm after dispatch, [3] compute before the FFN, [4] compute after GEMM A,
@@ -106,6 +107,19 @@ typedef struct moe_config {
      [3], [4], [5]. For per-kernel timing with cudaEventElapsedTime. */
   void *const *timing_events;
 } moe_config;
+
+/*
+ * Weight prepack (a layout copy made once, e.g. when the model is loaded; not part of
+ * the pages' method). The grouped GEMMs read each expert's weights as tiles of 64 k-rows
+ * x 128 columns; from [E,H,2I] / [E,I,H] every such tile is 64 pieces of 128 bytes at the
+ * matrix's row pitch. moe_pack_weights stores each tile as one contiguous 16 KB block in
+ * the order the GEMM's shared-memory tile takes, so the weight stream reads contiguous
+ * HBM. Packed sizes (bytes) from moe_packed_weight_bytes; columns past I / H are zero.
+ * W1p and W2p are caller-owned device buffers, 16-byte aligned; the copy runs on `stream`.
+ */
+int moe_packed_weight_bytes(const moe_shape *s, size_t *w1p_bytes, size_t *w2p_bytes);
+int moe_pack_weights(const moe_shape *s, const void *W1, const void *W2, void *W1p, void *W2p,
+                     void *stream);
 
 /* Dropless pool bound: T*k + min(E, T*k)*(tile-1), rounded up to a multiple of tile. */
 int moe_pool_rows_max(const moe_shape *s, int64_t *rows_out);

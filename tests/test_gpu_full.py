@@ -21,9 +21,11 @@ def _weights(cfg):
     return h1, h2, W1, W2
 
 
-@pytest.mark.parametrize("name,streaming", [("qwen3_235b_a22b", 0), ("qwen3_235b_a22b", 1),
-                                            ("deepseek_v3", 1), ("decode_microbatch", 1)])
-def test_full_layer(name, streaming):
+@pytest.mark.parametrize("name,streaming,packed", [("qwen3_235b_a22b", 0, 0),
+                                                   ("qwen3_235b_a22b", 1, 1),
+                                                   ("deepseek_v3", 0, 1), ("deepseek_v3", 1, 0),
+                                                   ("decode_microbatch", 1, 1)])
+def test_full_layer(name, streaming, packed):
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import (assert_layer_close, bf16_dev, check_plan_exact, f32_dev, i32_dev,
                              sample_tokens, to_f64)
@@ -31,13 +33,15 @@ def test_full_layer(name, streaming):
     h1, h2, W1, W2 = _weights(cfg)
     buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
     buf.pool.view(torch.int16).fill_(0x7FC0)
+    if packed:                                   # the layout the benchmark times
+        W1, W2 = buf.pack_weights(W1, W2)
     W1l = [h1[e] for e in range(cfg.E)]
     W2l = [h2[e] for e in range(cfg.E)]
     for mb in range(cfg.micro_batches):
         x = si.make_x(cfg, mb)
         idx, w = si.make_routing(cfg, mb)
         out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2,
-                          moe.moe_config(streaming, 0, 0, 0, None))
+                          moe.moe_config(streaming, 0, 0, packed, None))
         torch.cuda.synchronize()
         code, aux = moe.moe_get_status(buf.plan)
         assert code == 0, (moe.moe_strerror(code), aux)
