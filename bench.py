@@ -173,9 +173,18 @@ def physical_gpu_index(local_rank: int) -> int:
     return local_rank
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "ffn_gemm_kernel<0>": ("ffn_gemm.cu", "moe_common.cuh", "moe_internal.h"),
+    "ffn_gemm_kernel<1>": ("ffn_gemm.cu", "moe_common.cuh", "moe_internal.h"),
+    "dispatch_kernel": ("dispatch.cu", "moe_common.cuh", "moe_internal.h"),
+}
+
+
+def kernel_source_hash(kernel: str = "ffn_gemm_kernel<0>") -> str:
+    """Hash of the source files a kernel is built from (its committed counters are only
+    used while this matches)."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "combine_moe_plan_03_b200", "csrc"))):
+    for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, "combine_moe_plan_03_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -189,7 +198,7 @@ def committed_traffic(kernel: str):
     except Exception:
         return None
     ent = d.get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 

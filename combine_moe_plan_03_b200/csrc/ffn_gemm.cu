@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int32_t u = -1;
       int got = 1;
       if (lane == 0) {
-        got = mbar_wait(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort) ? 1 : 0;
+        got = mbar_wait_sleepy(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort, 1024) ? 1 : 0;
         if (got) {
           u = sched[sslot];
           mbar_arrive(sched_empty + sslot);
@@ -353,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t row0 = prm.mblk[3 * mb + 0];
       const int32_t rows = prm.mblk[3 * mb + 2];
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(acc_full, local & 1u, 3 * prm.timeout_ns, abort) ? 1 : 0;
+      if (lane == 0)
+        ok = mbar_wait_sleepy(acc_full, local & 1u, 3 * prm.timeout_ns, abort, 1024) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) raise_abort(abort, prm.status, MOE_ERR_PIPE_TIMEOUT, (int32_t)u);

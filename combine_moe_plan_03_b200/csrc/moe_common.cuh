@@ -110,6 +110,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
   }
 }
 
+// Same as mbar_wait, for waits that usually last long (a whole GEMM unit): between polls
+// the thread sleeps, backing off from 32 ns to max_sleep_ns, so it spends few issue
+// slots (and little power) while it waits.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity,
+                                                 uint64_t timeout_ns, const volatile int *abort,
+                                                 uint32_t max_sleep_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t sleep_ns = 32;
+  for (;;) {
+    __nanosleep(sleep_ns);
+    if (sleep_ns < max_sleep_ns) sleep_ns <<= 1;
+    if (mbar_try_wait(a, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
 // ---- TMA --------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
