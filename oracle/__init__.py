@@ -56,6 +56,8 @@ class Oracle:
         L.oracle_moe_forward_identity.restype = ctypes.c_int
         L.oracle_combine.argtypes = [i64, i32, i32, vp, vp, vp, vp]
         L.oracle_combine.restype = ctypes.c_int
+        L.oracle_route.argtypes = [i64, i32, i32, vp, vp, vp, vp]
+        L.oracle_route.restype = ctypes.c_int
         self.L = L
 
     # ---- plan -------------------------------------------------------------------------
@@ -156,6 +158,19 @@ class Oracle:
         if rc != 0:
             raise OracleError(rc)
         return y
+
+
+    def route(self, logits: np.ndarray, k: int, bias: Optional[np.ndarray] = None):
+        """Router: (topk_idx [T, k] int32, topk_w [T, k] float64) from fp32 logits [T, E]."""
+        lg = np.ascontiguousarray(logits, np.float32)
+        T, E = lg.shape
+        b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+        idx = np.empty((T, k), np.int32)
+        w = np.empty((T, k), np.float64)
+        rc = self.L.oracle_route(T, E, k, _p(lg), 0 if b is None else _p(b), _p(idx), _p(w))
+        if rc != 0:
+            raise OracleError(rc)
+        return idx, w
 
 
 class OracleError(RuntimeError):

@@ -26,7 +26,10 @@
  *   - padding rows of the pool are all-zero;
  *   - topk_idx == -1 marks a dropped pair (no pool row, no contribution);
  *     any other index outside [0, E) is an error;
- *   - silu(v) = v / (1 + exp(-v)).
+ *   - silu(v) = v / (1 + exp(-v));
+ *   - the router's choice (oracle_route) is taken on the fp32 scores logit + bias
+ *     (one fp32 addition), the precision the GPU decides in; ties go to the lower
+ *     expert index; the renormalised weights are computed in double.
  *
  * Pins (tests/test_oracle_pins.py): a hand-worked example, a stable-sort brute
  * force of the plan, invariants, a dense all-experts brute force of the layer,
@@ -256,5 +259,48 @@ int oracle_combine(int64_t T, int32_t H, int32_t k, const int32_t *pool_row,
       y[t * H + m] = acc;
     }
   }
+  return ORACLE_OK;
+}
+
+/*
+ * Router (the inputs of the StreamEP call: topk_idx / topk_weights from the gate's
+ * softmax; "softmax top-k, renormalised"), per token t over E experts:
+ *   v_e   = logits[t][e] + bias[e]            (fp32; bias may be NULL)
+ *   chosen = the k largest v_e, largest first, equal v_e: lower e first
+ *   w_j   = p_j / sum_{chosen i} p_i with p = softmax(v) over all E experts,
+ *           which equals exp(v_j - m) / sum_{chosen i} exp(v_i - m), m = max_e v_e
+ * idx [T, k] int32, w [T, k] double.
+ */
+int oracle_route(int64_t T, int32_t E, int32_t k, const float *logits, const float *bias,
+                 int32_t *idx, double *w) {
+  if (T < 0 || E <= 0 || k <= 0 || k > E) return ORACLE_ERR_ARG;
+  float *v = (float *)malloc(sizeof(float) * (size_t)E);
+  unsigned char *taken = (unsigned char *)malloc((size_t)E);
+  if (!v || !taken) {
+    free(v);
+    free(taken);
+    return ORACLE_ERR_ARG;
+  }
+  for (int64_t t = 0; t < T; ++t) {
+    float m = -INFINITY;
+    for (int32_t e = 0; e < E; ++e) {
+      v[e] = bias ? logits[t * E + e] + bias[e] : logits[t * E + e];
+      taken[e] = 0;
+      if (v[e] > m) m = v[e];
+    }
+    double sum = 0.0;
+    for (int32_t j = 0; j < k; ++j) {
+      int32_t best = -1;
+      for (int32_t e = 0; e < E; ++e)
+        if (!taken[e] && (best < 0 || v[e] > v[best])) best = e;
+      taken[best] = 1;
+      idx[t * k + j] = best;
+      w[t * k + j] = exp((double)v[best] - (double)m);
+      sum += w[t * k + j];
+    }
+    for (int32_t j = 0; j < k; ++j) w[t * k + j] /= sum;
+  }
+  free(v);
+  free(taken);
   return ORACLE_OK;
 }

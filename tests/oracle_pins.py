@@ -304,9 +304,56 @@ def pin_combine_gather(orc):
                                orc.moe_forward_identity(x, idx, w), rtol=1e-15, atol=0)
 
 
+# ---------------------------------------------------------------- router ---------------
+
+def route_bruteforce(logits, k, bias=None):
+    """np.lexsort on (-score, index) of the fp32 scores; softmax over all experts in double,
+    renormalised over the chosen ones."""
+    v = logits.astype(np.float32) + (bias.astype(np.float32) if bias is not None else np.float32(0))
+    T, E = v.shape
+    idx = np.empty((T, k), np.int64)
+    w = np.empty((T, k))
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -v[t].astype(np.float64)))
+        idx[t] = order[:k]
+        p = np.exp(v[t].astype(np.float64) - v[t].max())
+        p /= p.sum()
+        w[t] = p[order[:k]] / p[order[:k]].sum()
+    return idx, w
+
+
+def pin_route_bruteforce(orc):
+    rng = _rng(11)
+    for (T, E, k, with_bias) in [(50, 8, 2, False), (40, 64, 8, True), (10, 256, 8, True),
+                                 (7, 5, 5, False), (9, 33, 1, True)]:
+        lg = rng.standard_normal((T, E)).astype(np.float32)
+        b = (rng.standard_normal(E) * 0.5).astype(np.float32) if with_bias else None
+        idx, w = orc.route(lg, k, b)
+        ridx, rw = route_bruteforce(lg, k, b)
+        np.testing.assert_array_equal(idx, ridx)
+        np.testing.assert_allclose(w, rw, rtol=1e-12, atol=0)
+
+
+def pin_route_special_cases(orc):
+    rng = _rng(12)
+    lg = rng.standard_normal((6, 16)).astype(np.float32)
+    idx, w = orc.route(lg, 1)
+    np.testing.assert_array_equal(idx[:, 0], np.argmax(lg, axis=1))
+    assert np.all(w == 1.0)                                       # k = 1: weight exactly 1
+    idx, w = orc.route(lg, 16)                                    # k = E: the full softmax
+    sm = np.exp(lg.astype(np.float64) - lg.max(1, keepdims=True))
+    sm /= sm.sum(1, keepdims=True)
+    np.testing.assert_allclose(w, np.take_along_axis(sm, idx.astype(np.int64), 1), rtol=1e-12)
+    tie = np.zeros((1, 6), np.float32)
+    tie[0, [1, 4]] = 2.0                                          # exact tie: lower index first
+    idx, w = orc.route(tie, 3)
+    assert idx.tolist() == [[1, 4, 0]]
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-15)
+
+
 ALL_PINS = [
     pin_plan_worked, pin_plan_bruteforce, pin_plan_invariants, pin_plan_bad_index,
     pin_pool_gather, pin_ffn_worked, pin_ffn_dense_bruteforce, pin_ffn_textbook_torch,
     pin_ffn_closed_form, pin_ffn_linearity, pin_ffn_permutation, pin_identity_closed_form,
-    pin_combine_gather,
+    pin_combine_gather, pin_route_bruteforce, pin_route_special_cases,
 ]

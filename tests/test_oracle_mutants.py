@@ -37,6 +37,14 @@ MUTANTS = {
     "identity_counts_dropped": ("if (topk_idx[t * k + j] >= 0)\n          acc +=", "acc +="),
     "bad_index_accepted": ("if (e < -1 || e >= E) return ORACLE_ERR_BAD_INDEX;\n  }\n  for (int32_t e = 0; e < E; ++e) counts[e] = 0;",
                            "if (e < -1 || e >= E) e = 0;\n  }\n  for (int32_t e = 0; e < E; ++e) counts[e] = 0;"),
+    "route_tie_to_higher_index": ("if (!taken[e] && (best < 0 || v[e] > v[best])) best = e;",
+                                  "if (!taken[e] && (best < 0 || v[e] >= v[best])) best = e;"),
+    "route_no_renorm": ("for (int32_t j = 0; j < k; ++j) w[t * k + j] /= sum;",
+                        "for (int32_t j = 0; j < k; ++j) w[t * k + j] /= sum + 1.0;"),
+    "route_smallest_first": ("if (!taken[e] && (best < 0 || v[e] > v[best])) best = e;",
+                             "if (!taken[e] && (best < 0 || v[e] < v[best])) best = e;"),
+    "route_bias_ignored": ("v[e] = bias ? logits[t * E + e] + bias[e] : logits[t * E + e];",
+                           "v[e] = logits[t * E + e];"),
 }
 
 
