@@ -502,6 +502,40 @@ def run_moe(args):
                             "traffic": committed_traffic("dispatch_kernel"),
                             "peak_source": f"{peak_src} HBM copy"}
 
+    # ---------------- router on the device (not part of the layer step: the layer takes
+    # topk_idx / topk_w as inputs); timed on its own with the workload's logits
+    if cfg.routing in ("softmax", "softmax_bias") and rank == 0:
+        lg = si.normal_f32(cfg.seed, si.STREAM_LOGITS, 0, cfg.T * cfg.E).reshape(cfg.T, cfg.E)
+        dl = torch.from_numpy(lg).to(dev)
+        db = None
+        if cfg.routing == "softmax_bias":
+            db = torch.from_numpy(si.normal_f32(cfg.seed, si.STREAM_BIAS, 0, cfg.E,
+                                                cfg.bias_sigma)).to(dev)
+        ri = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+        rw = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+        rb = moe.MoELayerBuffers(cfg.T, 64, 64, cfg.E, cfg.k, cfg.tile, device=dev,
+                                 identity=True)
+        st = torch.cuda.current_stream().cuda_stream
+
+        def rp():
+            moe.moe_route_plan(rb.shape, dl.data_ptr(), db.data_ptr() if db is not None else 0,
+                               ri.data_ptr(), rw.data_ptr(), rb.plan, 0, st)
+        for _ in range(5):
+            rp()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(50):
+            rp()
+        s1.record()
+        torch.cuda.synchronize()
+        rp_ms = s0.elapsed_time(s1) / 50
+        line["router"] = {"route_plan_ms": rp_ms,
+                          "kernels": 3 if 256 % cfg.k == 0 else 4,
+                          "logits_gbs": cfg.T * cfg.E * 4 / (rp_ms / 1e3) / 1e9,
+                          "matches_host_router": bool(np.array_equal(ri.cpu().numpy(), idxs[0])
+                                                      if rank == 0 and mbs == 1 else True)}
+        rb.close()
+
     # ---------------- e2e: pinned host inputs in, result out, copies inside the timed region
     hx = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in xs]
     hidx = [torch.from_numpy(a).pin_memory() for a in idxs]

@@ -82,6 +82,8 @@ def _load():
         "moe_get_status": [P(moe_plan_buffers), P(i32), P(i32)],
         "moe_clear_status": [P(moe_plan_buffers), vp],
         "moe_plan_noalloc": [P(moe_shape), vp, P(moe_plan_buffers), vp, vp],
+        "moe_route": [P(moe_shape), vp, vp, vp, vp, vp],
+        "moe_route_plan": [P(moe_shape), vp, vp, vp, vp, P(moe_plan_buffers), vp, vp],
         "moe_packed_weight_bytes": [P(moe_shape), P(ctypes.c_size_t), P(ctypes.c_size_t)],
         "moe_pack_weights": [P(moe_shape), vp, vp, vp, vp, vp],
     }
@@ -99,7 +101,7 @@ def _load():
 _lib = _load()
 
 # Names exported by include/moe.h, in declaration order.
-EXPORTS = ["moe_packed_weight_bytes", "moe_pack_weights", "moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
+EXPORTS = ["moe_route", "moe_route_plan", "moe_packed_weight_bytes", "moe_pack_weights", "moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
            "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
            "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
@@ -176,6 +178,20 @@ def moe_plan_noalloc(shape, topk_idx_ptr: int, plan: moe_plan_buffers, host_P_pt
     _check("moe_plan_noalloc", _lib.moe_plan_noalloc(ctypes.byref(_shape(shape)), topk_idx_ptr,
                                                      ctypes.byref(plan), host_P_ptr or None,
                                                      stream or None))
+
+
+def moe_route(shape, logits_ptr: int, bias_ptr: int, topk_idx_ptr: int, topk_w_ptr: int,
+              stream: int = 0) -> None:
+    _check("moe_route", _lib.moe_route(ctypes.byref(_shape(shape)), logits_ptr, bias_ptr or None,
+                                       topk_idx_ptr, topk_w_ptr, stream or None))
+
+
+def moe_route_plan(shape, logits_ptr: int, bias_ptr: int, topk_idx_ptr: int, topk_w_ptr: int,
+                   plan: moe_plan_buffers, host_P_ptr: int = 0, stream: int = 0) -> None:
+    _check("moe_route_plan", _lib.moe_route_plan(ctypes.byref(_shape(shape)), logits_ptr,
+                                                 bias_ptr or None, topk_idx_ptr, topk_w_ptr,
+                                                 ctypes.byref(plan), host_P_ptr or None,
+                                                 stream or None))
 
 
 def moe_dispatch(shape, x_ptr: int, plan: moe_plan_buffers, pool_ptr: int,

@@ -163,6 +163,39 @@ int moe_plan(const moe_shape *s, const int32_t *topk_idx, const moe_plan_buffers
   return MOE_OK;
 }
 
+int moe_route(const moe_shape *s, const float *logits, const float *bias, int32_t *topk_idx,
+              float *topk_w, void *stream) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if (s->k > s->E) return MOE_ERR_INVALID_ARG;
+  if (s->T > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  if (launch_route(*s, logits, bias, topk_idx, topk_w, nullptr, nsm,
+                   static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_route_plan(const moe_shape *s, const float *logits, const float *bias, int32_t *topk_idx,
+                   float *topk_w, const moe_plan_buffers *p, int32_t *host_P, void *stream) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (s->k > s->E) return MOE_ERR_INVALID_ARG;
+  if (s->T > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (launch_route(*s, logits, bias, topk_idx, topk_w, p, nsm, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (host_P != nullptr &&
+      cudaMemcpyAsync(host_P, p->meta + 1, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, void *pool,
                  int32_t signal_flags, void *stream) {
   int rc = check_shape(s, false);

@@ -46,6 +46,13 @@ size_t plan_workspace_ints(const moe_shape &s);
 
 cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_plan_buffers &p,
                         cudaStream_t st);
+// The plan's second and third launches (per-expert scan + tables, stable rank), after
+// ws[e][chunk] holds the per-chunk counts (written by plan_hist_kernel or the router).
+cudaError_t launch_plan_scan_rank(const moe_shape &s, const int32_t *topk_idx,
+                                  const moe_plan_buffers &p, cudaStream_t st);
+cudaError_t launch_route(const moe_shape &s, const float *logits, const float *bias,
+                         int32_t *topk_idx, float *topk_w, const moe_plan_buffers *p,
+                         int num_sms, cudaStream_t st);
 cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_buffers &p,
                             void *pool, int signal, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const moe_shape &s, const void *ypool, const float *topk_w,

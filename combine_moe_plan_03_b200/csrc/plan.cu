@@ -225,6 +225,16 @@ cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_p
       p.tile_flags, g.n_tiles, p.status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
+  return launch_plan_scan_rank(s, topk_idx, p, st);
+}
+
+cudaError_t launch_plan_scan_rank(const moe_shape &s, const int32_t *topk_idx,
+                                  const moe_plan_buffers &p, cudaStream_t st) {
+  const PlanGeom g = plan_geom(s);
+  const size_t smem = sizeof(int32_t) * kPlanWarps * (size_t)s.E;
+  int32_t *done = p.workspace + (size_t)s.E * (size_t)(g.n_chunks > 0 ? g.n_chunks : 1);
+  const int nblk = g.n_chunks > 0 ? (g.n_chunks + kPlanWarps - 1) / kPlanWarps : 0;
+  cudaError_t err;
   plan_scan_kernel<<<s.E, 256, 0, st>>>(p.workspace, g.n_chunks, s.E, s.tile, done, p.counts,
                                          p.offsets, p.tile_expert, p.mblk, p.meta, g.pmax,
                                          p.status);

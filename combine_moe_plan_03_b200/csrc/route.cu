@@ -1,0 +1,158 @@
+// Router on the device: per token, the softmax over E experts of the fp32 scores
+// logit + bias, the k largest (ties: lower expert index), renormalised over the k
+// chosen (the topk_idx / topk_weights the StreamEP call takes as inputs). Because
+// the softmax is monotonic and its denominator cancels in the renormalisation, the
+// choice is made on the scores themselves and w_j = exp(v_j - m) / sum over the
+// chosen exp(v_i - m), m = the largest score.
+//
+// One warp per token: lane l holds the scores of experts l, l+32, ...; each of the
+// k rounds is a warp argmax (shuffle butterfly) over the experts not chosen yet.
+// With a plan to fill (and k dividing 256), each warp routes the tokens of exactly
+// one 256-pair plan chunk and counts its pairs per expert in shared memory, so the
+// plan's histogram launch is not needed (the plan's scan and rank launches follow).
+#include <float.h>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+constexpr int kRoutePerLane = kMaxExperts / 32;
+
+// Route token t; lane j < k returns the j-th chosen expert in *e_out and its weight in
+// *w_out (other lanes: -1, 0).
+__device__ __forceinline__ void route_token(const float *__restrict__ row,
+                                            const float *__restrict__ bias, int E, int k,
+                                            int lane, int32_t *e_out, float *w_out) {
+  float v[kRoutePerLane];
+  const int nper = (E + 31) >> 5;
+#pragma unroll
+  for (int i = 0; i < kRoutePerLane; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = -FLT_MAX;
+    if (i < nper && e < E) v[i] = bias ? row[e] + bias[e] : row[e];
+  }
+  uint32_t taken = 0;
+  int32_t my_e = -1;
+  float my_v = 0.0f, m = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -FLT_MAX;
+    int32_t be = INT32_MAX;
+#pragma unroll
+    for (int i = 0; i < kRoutePerLane; ++i) {
+      const int e = lane + 32 * i;
+      if (i < nper && e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int32_t oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (j == 0) m = bv;
+    if (lane == j) {
+      my_e = be;
+      my_v = bv;
+    }
+  }
+  const float ex = lane < k ? expf(my_v - m) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  *e_out = my_e;
+  *w_out = lane < k ? ex / sum : 0.0f;
+}
+
+__global__ void __launch_bounds__(256)
+    route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int32_t T,
+                 int32_t E, int32_t k, int32_t *__restrict__ topk_idx,
+                 float *__restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
+       t += warps) {
+    int32_t e;
+    float w;
+    route_token(logits + t * E, bias, E, k, lane, &e, &w);
+    if (lane < k) {
+      topk_idx[t * k + lane] = e;
+      topk_w[t * k + lane] = w;
+    }
+  }
+}
+
+// Routing fused with the plan's first launch: warp = one 256-pair chunk.
+__global__ void __launch_bounds__(kPlanWarps * 32)
+    route_hist_kernel(const float *__restrict__ logits, const float *__restrict__ bias,
+                      int32_t T, int32_t E, int32_t k, int32_t *__restrict__ topk_idx,
+                      float *__restrict__ topk_w, int32_t n_chunks, int32_t *__restrict__ ws,
+                      int32_t *__restrict__ done_counter, int32_t *__restrict__ row_src,
+                      int64_t pmax, int32_t *__restrict__ tile_expert,
+                      uint32_t *__restrict__ flags, int64_t n_tiles) {
+  extern __shared__ int32_t hist[];  // [kPlanWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kPlanWarps * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int chunk = blockIdx.x * kPlanWarps + warp;
+  if (chunk < n_chunks) {
+    int32_t *h = hist + warp * E;
+    const int per = kPlanChunk / k;  // tokens per chunk
+    const int64_t t0 = (int64_t)chunk * per;
+    for (int i = 0; i < per; ++i) {
+      const int64_t t = t0 + i;
+      if (t >= T) break;
+      int32_t e;
+      float w;
+      route_token(logits + t * E, bias, E, k, lane, &e, &w);
+      if (lane < k) {
+        topk_idx[t * k + lane] = e;
+        topk_w[t * k + lane] = w;
+        atomicAdd(&h[e], 1);
+      }
+    }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) ws[(int64_t)e * n_chunks + chunk] = h[e];
+  }
+  const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t gsz = (int64_t)gridDim.x * blockDim.x;
+  if (gtid == 0) *done_counter = 0;
+  for (int64_t i = gtid; i < pmax; i += gsz) row_src[i] = -1;
+  for (int64_t i = gtid; i < n_tiles; i += gsz) {
+    tile_expert[i] = -1;
+    flags[i] = 0;
+  }
+}
+
+cudaError_t launch_route(const moe_shape &s, const float *logits, const float *bias,
+                         int32_t *topk_idx, float *topk_w, const moe_plan_buffers *p,
+                         int num_sms, cudaStream_t st) {
+  if (p == nullptr || (kPlanChunk % s.k) != 0) {
+    if (s.T > 0) {
+      const int64_t blocks = ((int64_t)s.T + 7) / 8;
+      const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
+      route_kernel<<<grid, 256, 0, st>>>(logits, bias, s.T, s.E, s.k, topk_idx, topk_w);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess || p == nullptr) return e;
+    }
+    return launch_plan(s, topk_idx, *p, st);
+  }
+  const PlanGeom g = plan_geom(s);
+  const size_t smem = sizeof(int32_t) * kPlanWarps * (size_t)s.E;
+  int32_t *done = p->workspace + (size_t)s.E * (size_t)(g.n_chunks > 0 ? g.n_chunks : 1);
+  const int nblk = g.n_chunks > 0 ? (g.n_chunks + kPlanWarps - 1) / kPlanWarps : 1;
+  route_hist_kernel<<<nblk, kPlanWarps * 32, smem, st>>>(
+      logits, bias, s.T, s.E, s.k, topk_idx, topk_w, g.n_chunks, p->workspace, done, p->row_src,
+      g.pmax, p->tile_expert, p->tile_flags, g.n_tiles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_plan_scan_rank(s, topk_idx, *p, st);
+}
+
+}  // namespace moe

@@ -147,6 +147,25 @@ int moe_plan(const moe_shape *s, const int32_t *topk_idx, const moe_plan_buffers
              int32_t *host_P, void *stream);
 
 /*
+ * Router on the device (the topk_idx / topk_weights inputs of the StreamEP call: the
+ * gate's softmax, top-k, renormalised). For each token t of fp32 logits [T, E] and an
+ * optional fp32 bias [E] (NULL for none): scores v = logit + bias (fp32); the k largest
+ * scores, largest first, equal scores by lower expert index, go to topk_idx [T, k];
+ * topk_w [T, k] = their softmax probabilities renormalised over the k chosen (fp32,
+ * expf). Requires k <= E. Logits must be finite.
+ */
+int moe_route(const moe_shape *s, const float *logits, const float *bias, int32_t *topk_idx,
+              float *topk_w, void *stream);
+
+/*
+ * moe_route followed by moe_plan, with the router and the plan's per-expert histogram
+ * in one kernel when k divides 256 (each warp routes one 256-pair plan chunk); same
+ * outputs as the two calls. host_P as in moe_plan.
+ */
+int moe_route_plan(const moe_shape *s, const float *logits, const float *bias, int32_t *topk_idx,
+                   float *topk_w, const moe_plan_buffers *p, int32_t *host_P, void *stream);
+
+/*
  * Dispatch (StreamEP README, How it works, "Pool-layout dispatch" and "Per-tile
  * streaming"): pool[pool_row[t*k+j]] = x[t] for every live pair, padding rows of
  * each expert's segment set to zero, and (signal_flags != 0) tile_flags[p / tile]
