@@ -7,7 +7,7 @@
 //
 // One warp per token: lane l holds the scores of experts l, l+32, ...; each of the
 // k rounds is a warp argmax (shuffle butterfly) over the experts not chosen yet.
-// With a plan to fill (and k dividing 256), each warp routes the tokens of exactly
+// With a plan to fill (and k dividing 256), each block routes the tokens of exactly
 // one 256-pair plan chunk and counts its pairs per expert in shared memory, so the
 // plan's histogram launch is not needed (the plan's scan and rank launches follow).
 #include <float.h>
@@ -17,20 +17,18 @@
 
 namespace moe {
 
-constexpr int kRoutePerLane = kMaxExperts / 32;
-
 // Route token t; lane j < k returns the j-th chosen expert in *e_out and its weight in
-// *w_out (other lanes: -1, 0).
+// *w_out (other lanes: -1, 0). kPer = scores held per lane (E <= 32 * kPer).
+template <int kPer>
 __device__ __forceinline__ void route_token(const float *__restrict__ row,
                                             const float *__restrict__ bias, int E, int k,
                                             int lane, int32_t *e_out, float *w_out) {
-  float v[kRoutePerLane];
-  const int nper = (E + 31) >> 5;
+  float v[kPer];
 #pragma unroll
-  for (int i = 0; i < kRoutePerLane; ++i) {
+  for (int i = 0; i < kPer; ++i) {
     const int e = lane + 32 * i;
     v[i] = -FLT_MAX;
-    if (i < nper && e < E) v[i] = bias ? row[e] + bias[e] : row[e];
+    if (e < E) v[i] = bias ? row[e] + bias[e] : row[e];
   }
   uint32_t taken = 0;
   int32_t my_e = -1;
@@ -39,9 +37,9 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row,
     float bv = -FLT_MAX;
     int32_t be = INT32_MAX;
 #pragma unroll
-    for (int i = 0; i < kRoutePerLane; ++i) {
+    for (int i = 0; i < kPer; ++i) {
       const int e = lane + 32 * i;
-      if (i < nper && e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
+      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
         bv = v[i];
         be = e;
       }
@@ -70,6 +68,7 @@ __device__ __forceinline__ void route_token(const float *__restrict__ row,
   *w_out = lane < k ? ex / sum : 0.0f;
 }
 
+template <int kPer>
 __global__ void __launch_bounds__(256)
     route_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int32_t T,
                  int32_t E, int32_t k, int32_t *__restrict__ topk_idx,
@@ -80,7 +79,7 @@ __global__ void __launch_bounds__(256)
        t += warps) {
     int32_t e;
     float w;
-    route_token(logits + t * E, bias, E, k, lane, &e, &w);
+    route_token<kPer>(logits + t * E, bias, E, k, lane, &e, &w);
     if (lane < k) {
       topk_idx[t * k + lane] = e;
       topk_w[t * k + lane] = w;
@@ -88,7 +87,9 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Routing fused with the plan's first launch: warp = one 256-pair chunk.
+// Routing fused with the plan's first launch: block = one 256-pair chunk, its 8 warps
+// route the chunk's tokens in turn and count them in one shared histogram.
+template <int kPer>
 __global__ void __launch_bounds__(kPlanWarps * 32)
     route_hist_kernel(const float *__restrict__ logits, const float *__restrict__ bias,
                       int32_t T, int32_t E, int32_t k, int32_t *__restrict__ topk_idx,
@@ -96,30 +97,30 @@ __global__ void __launch_bounds__(kPlanWarps * 32)
                       int32_t *__restrict__ done_counter, int32_t *__restrict__ row_src,
                       int64_t pmax, int32_t *__restrict__ tile_expert,
                       uint32_t *__restrict__ flags, int64_t n_tiles) {
-  extern __shared__ int32_t hist[];  // [kPlanWarps][E]
+  extern __shared__ int32_t hist[];  // [E] for this block's chunk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kPlanWarps * E; i += blockDim.x) hist[i] = 0;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  const int chunk = blockIdx.x * kPlanWarps + warp;
+  const int chunk = blockIdx.x;
   if (chunk < n_chunks) {
-    int32_t *h = hist + warp * E;
     const int per = kPlanChunk / k;  // tokens per chunk
     const int64_t t0 = (int64_t)chunk * per;
-    for (int i = 0; i < per; ++i) {
+    for (int i = warp; i < per; i += kPlanWarps) {
       const int64_t t = t0 + i;
       if (t >= T) break;
       int32_t e;
       float w;
-      route_token(logits + t * E, bias, E, k, lane, &e, &w);
+      route_token<kPer>(logits + t * E, bias, E, k, lane, &e, &w);
       if (lane < k) {
         topk_idx[t * k + lane] = e;
         topk_w[t * k + lane] = w;
-        atomicAdd(&h[e], 1);
+        atomicAdd(&hist[e], 1);
       }
     }
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) ws[(int64_t)e * n_chunks + chunk] = h[e];
   }
+  __syncthreads();
+  if (chunk < n_chunks)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) ws[(int64_t)e * n_chunks + chunk] = hist[e];
   const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t gsz = (int64_t)gridDim.x * blockDim.x;
   if (gtid == 0) *done_counter = 0;
@@ -130,29 +131,42 @@ __global__ void __launch_bounds__(kPlanWarps * 32)
   }
 }
 
-cudaError_t launch_route(const moe_shape &s, const float *logits, const float *bias,
-                         int32_t *topk_idx, float *topk_w, const moe_plan_buffers *p,
-                         int num_sms, cudaStream_t st) {
+template <int kPer>
+static cudaError_t launch_route_t(const moe_shape &s, const float *logits, const float *bias,
+                                  int32_t *topk_idx, float *topk_w, const moe_plan_buffers *p,
+                                  int num_sms, cudaStream_t st) {
   if (p == nullptr || (kPlanChunk % s.k) != 0) {
     if (s.T > 0) {
       const int64_t blocks = ((int64_t)s.T + 7) / 8;
       const int grid = (int)(blocks < (int64_t)num_sms * 8 ? blocks : (int64_t)num_sms * 8);
-      route_kernel<<<grid, 256, 0, st>>>(logits, bias, s.T, s.E, s.k, topk_idx, topk_w);
+      route_kernel<kPer><<<grid, 256, 0, st>>>(logits, bias, s.T, s.E, s.k, topk_idx, topk_w);
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess || p == nullptr) return e;
     }
     return launch_plan(s, topk_idx, *p, st);
   }
   const PlanGeom g = plan_geom(s);
-  const size_t smem = sizeof(int32_t) * kPlanWarps * (size_t)s.E;
+  const size_t smem = sizeof(int32_t) * (size_t)s.E;
   int32_t *done = p->workspace + (size_t)s.E * (size_t)(g.n_chunks > 0 ? g.n_chunks : 1);
-  const int nblk = g.n_chunks > 0 ? (g.n_chunks + kPlanWarps - 1) / kPlanWarps : 1;
-  route_hist_kernel<<<nblk, kPlanWarps * 32, smem, st>>>(
+  const int nblk = g.n_chunks > 0 ? g.n_chunks : 1;
+  route_hist_kernel<kPer><<<nblk, kPlanWarps * 32, smem, st>>>(
       logits, bias, s.T, s.E, s.k, topk_idx, topk_w, g.n_chunks, p->workspace, done, p->row_src,
       g.pmax, p->tile_expert, p->tile_flags, g.n_tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_plan_scan_rank(s, topk_idx, *p, st);
+}
+
+cudaError_t launch_route(const moe_shape &s, const float *logits, const float *bias,
+                         int32_t *topk_idx, float *topk_w, const moe_plan_buffers *p,
+                         int num_sms, cudaStream_t st) {
+  const int per = (s.E + 31) / 32;
+  if (per <= 1) return launch_route_t<1>(s, logits, bias, topk_idx, topk_w, p, num_sms, st);
+  if (per <= 2) return launch_route_t<2>(s, logits, bias, topk_idx, topk_w, p, num_sms, st);
+  if (per <= 4) return launch_route_t<4>(s, logits, bias, topk_idx, topk_w, p, num_sms, st);
+  if (per <= 8) return launch_route_t<8>(s, logits, bias, topk_idx, topk_w, p, num_sms, st);
+  if (per <= 16) return launch_route_t<16>(s, logits, bias, topk_idx, topk_w, p, num_sms, st);
+  return launch_route_t<32>(s, logits, bias, topk_idx, topk_w, p, num_sms, st);
 }
 
 }  // namespace moe

@@ -159,7 +159,7 @@ int moe_route(const moe_shape *s, const float *logits, const float *bias, int32_
 
 /*
  * moe_route followed by moe_plan, with the router and the plan's per-expert histogram
- * in one kernel when k divides 256 (each warp routes one 256-pair plan chunk); same
+ * in one kernel when k divides 256 (each block routes one 256-pair plan chunk); same
  * outputs as the two calls. host_P as in moe_plan.
  */
 int moe_route_plan(const moe_shape *s, const float *logits, const float *bias, int32_t *topk_idx,
