@@ -47,6 +47,8 @@ def parse_args(argv=None):
                     help="1: FFN claims tiles while dispatch runs; 0: serial; -1: default")
     ap.add_argument("--packed", type=int, default=1,
                     help="1: prepack the weights once before timing (moe_pack_weights)")
+    ap.add_argument("--ffn-kernel", type=int, default=0,
+                    help="grouped-GEMM kernel: 1 one CTA per unit, 2 SM pairs; 0: default")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=16, help="oracle tokens per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -174,8 +176,12 @@ def physical_gpu_index(local_rank: int) -> int:
 
 
 KERNEL_SOURCES = {
-    "ffn_gemm_kernel<0>": ("ffn_gemm.cu", "moe_common.cuh", "moe_internal.h"),
-    "ffn_gemm_kernel<1>": ("ffn_gemm.cu", "moe_common.cuh", "moe_internal.h"),
+    "ffn_gemm_kernel<0>": ("ffn_gemm.cu", "ffn_gemm.cuh", "moe_common.cuh", "moe_internal.h"),
+    "ffn_gemm_kernel<1>": ("ffn_gemm.cu", "ffn_gemm.cuh", "moe_common.cuh", "moe_internal.h"),
+    "ffn_gemm_pair_kernel<0>": ("ffn_gemm_pair.cu", "ffn_gemm.cuh", "moe_common.cuh",
+                                "moe_internal.h"),
+    "ffn_gemm_pair_kernel<1>": ("ffn_gemm_pair.cu", "ffn_gemm.cuh", "moe_common.cuh",
+                                "moe_internal.h"),
     "dispatch_kernel": ("dispatch.cu", "moe_common.cuh", "moe_internal.h"),
 }
 
@@ -377,6 +383,7 @@ def run_moe(args):
     buf = moe.MoELayerBuffers(cfg.T, cfg.H, max(cfg.I, 64), cfg.E, cfg.k, cfg.tile, device=dev,
                               identity=cfg.identity)
     packed = 1 if (args.packed and not cfg.identity) else 0
+    ffn_kernel = args.ffn_kernel
     if packed:
         # one-time layout copy (as at model load), outside every timed region
         W1, W2 = buf.pack_weights(W1, W2)
@@ -385,9 +392,10 @@ def run_moe(args):
     tev = moe.moe_timing_events_create(7 * calls)
     import ctypes
     ev_arrays = [(ctypes.c_void_p * 7)(*tev[7 * c: 7 * c + 7]) for c in range(calls)]
-    cfgs = [moe.moe_config(streaming, 0, 0, packed, ctypes.cast(ev_arrays[c], ctypes.c_void_p))
+    cfgs = [moe.moe_config(streaming, 0, 0, packed, ffn_kernel,
+                           ctypes.cast(ev_arrays[c], ctypes.c_void_p))
             for c in range(calls)]
-    plain = moe.moe_config(streaming, 0, 0, packed, None)
+    plain = moe.moe_config(streaming, 0, 0, packed, ffn_kernel, None)
 
     def step_plain():
         for m in range(mbs):
@@ -458,7 +466,7 @@ def run_moe(args):
             "config": dict(config_block(cfg, world),
                            weights="prepacked tiles (moe_pack_weights, once before timing)"
                            if packed else "as given: W1 [E,H,2I], W2 [E,I,H]"),
-            "streaming": streaming,
+            "streaming": streaming, "ffn_kernel": ffn_kernel,
             "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
             "phases_mcycles_per_call": ({k: round(v * clocks["sm_mhz"] / 1000.0, 4)
                                          for k, v in ph.items()} if clocks.get("sm_mhz") else None),
@@ -485,11 +493,14 @@ def run_moe(args):
         achieved = flops_a / (ph["gemm_a"] / 1e3) / 1e12
         # The timed loop runs back to back at the power cap (see "clocks"), so the kernel is
         # compared with cuBLAS's sustained bf16 rate under the same cap; burst beside it.
-        line["roofline"] = {"kernel": "ffn_gemm_kernel<0> (GEMM A + SwiGLU)", "bound": "tensor",
+        kname = ("ffn_gemm_pair_kernel<0>"
+                 if (ffn_kernel or moe.MOE_FFN_DEFAULT) == moe.MOE_FFN_SM_PAIR
+                 else "ffn_gemm_kernel<0>")
+        line["roofline"] = {"kernel": f"{kname} (GEMM A + SwiGLU)", "bound": "tensor",
                             "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                             "unit": "TFLOP/s",
                             "frac": achieved / peaks["bf16_tflops_sustained"],
-                            "traffic": committed_traffic("ffn_gemm_kernel<0>"),
+                            "traffic": committed_traffic(kname),
                             "peak_source": f"{peak_src} bf16 sustained (timed inside a long "
                                            "loop at the power cap)",
                             "frac_of_burst": achieved / peaks["bf16_tflops"],

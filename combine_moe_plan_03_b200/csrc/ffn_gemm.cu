@@ -46,8 +46,7 @@
 // MOE_ERR_PIPE_TIMEOUT / MOE_ERR_FLAG_TIMEOUT in the status word and raises a
 // CTA-wide abort flag; the roles then leave their loops, the producer waits for
 // the loads it has in flight, the MMA thread for its MMAs, and the TMEM is freed.
-#include "moe_common.cuh"
-#include "moe_internal.h"
+#include "ffn_gemm.cuh"
 
 namespace moe {
 
@@ -69,40 +68,10 @@ constexpr int kBarrierBytes = 256;
 constexpr int kXposeBytes = 32 * 32 * 2;              // per epilogue warp: 32 rows x 32 columns bf16
 constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kEpiWarps * kXposeBytes + 1024;
 
-struct FfnParams {
-  const int32_t *mblk;     // row chunks {row_start, expert, live rows <= 256}
-  const int32_t *meta;     // meta[2] = number of row chunks
-  const uint32_t *flags;   // pool tile flags (streaming)
-  int32_t *status;
-  uint16_t *out;           // act (GEMM A) or ypool (GEMM Y)
-  int64_t out_ld;          // elements per row of out
-  int32_t K;               // reduction length
-  int32_t n_blocks;        // weight-column blocks per row chunk
-  int32_t col_step;        // weight columns per block (GEMM A 128, GEMM Y 256)
-  int32_t col1_off;        // first column of tile 1 inside the block's weights (I or 128)
-  int32_t n_out;           // output columns (I or H): masks a ragged last block
-  int32_t k_rows;          // rows per expert in the weight tensor map (H for W1, I for W2)
-  int32_t tile;            // pool tile rows
-  int32_t streaming;
-  int32_t *sched;          // {next unit ticket, CTAs done}: zero at launch, zeroed again at exit
-  int32_t packed;          // weights are moe_pack_weights tiles (one 16 KB box per tile)
-  int32_t pk_e, pk_j, pk_nb;  // packed tile index = e*pk_e + j*pk_j + nb*pk_nb + kb
-  uint64_t timeout_ns;
-};
-
 __device__ __forceinline__ void raise_abort(volatile int *abort, int32_t *status, int32_t code,
                                             int32_t aux) {
   if (!*abort) report(status, code, aux);
   *abort = 1;
-}
-
-__device__ __forceinline__ float silu_mul(float g, float u) {
-  return __fdividef(g, 1.0f + __expf(-g)) * u;
-}
-
-__device__ __forceinline__ uint16_t bf16_bits(float v) {
-  __nv_bfloat16 b = __float2bfloat16_rn(v);
-  return *reinterpret_cast<uint16_t *>(&b);
 }
 
 template <int kMode>
@@ -431,10 +400,8 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [outer, inner] viewed as a 2-D tensor; box {64, box_outer},
-// 128-byte swizzle (the canonical layout tcgen05 descriptors read).
-static bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-                      uint32_t box_outer) {
+bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+               uint32_t box_outer) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -484,8 +451,17 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
       !make_tmap(&tx_act, act, (uint64_t)s.I, (uint64_t)g.pmax, kRowBox))
     return MOE_ERR_CUDA;
 
+  const bool pair = (cfg.ffn_kernel != 0 ? cfg.ffn_kernel : MOE_FFN_DEFAULT) == MOE_FFN_SM_PAIR;
   int grid = cfg.ffn_ctas > 0 ? cfg.ffn_ctas : (cfg.streaming ? num_sms - 16 : num_sms);
   if (grid < 1) grid = 1;
+  int grid_y = cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms;
+  if (pair) {
+    // clusters of two CTAs: as many as fit at once, at most half the requested CTAs
+    const int fit0 = ffn_pair_max_clusters(0), fit1 = ffn_pair_max_clusters(1);
+    if (fit0 < 1 || fit1 < 1) return MOE_ERR_CUDA;
+    grid = grid / 2 < 1 ? 1 : (grid / 2 < fit0 ? grid / 2 : fit0);
+    grid_y = grid_y / 2 < 1 ? 1 : (grid_y / 2 < fit1 ? grid_y / 2 : fit1);
+  }
   const uint64_t timeout_ns =
       (uint64_t)(cfg.wait_timeout_us > 0 ? cfg.wait_timeout_us : 2000000) * 1000ull;
 
@@ -509,10 +485,18 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   a.pk_e = 2 * pg.nb1 * pg.kb1;           // gate tiles of expert e, then its up tiles
   a.pk_j = pg.nb1 * pg.kb1;
   a.pk_nb = pg.kb1;
+  a.pk_v = 0;
+  if (pair) {                             // 256 gate and 256 up columns per unit
+    a.col_step = 2 * kBM;
+    a.n_blocks = (s.I + 2 * kBM - 1) / (2 * kBM);
+    a.pk_nb = 2 * pg.kb1;
+    a.pk_v = pg.kb1;
+  }
   a.timeout_ns = timeout_ns;
   cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(cfg.timing_events);
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t e = launch_one<0>(tw1, tx_pool, a, grid, st);
+  cudaError_t e = pair ? launch_ffn_pair(0, tw1, tx_pool, a, grid, st)
+                       : launch_one<0>(tw1, tx_pool, a, grid, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -530,7 +514,16 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   y.pk_e = pg.nb2 * pg.kb2;               // 128-column blocks of expert e, k fastest
   y.pk_j = pg.kb2;
   y.pk_nb = 2 * pg.kb2;
-  e = launch_one<1>(tw2, tx_act, y, cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms, st);
+  if (pair) {                             // two adjacent blocks of 256 columns per unit
+    y.col_step = 4 * kBM;
+    y.col1_off = 2 * kBM;
+    y.n_blocks = (s.H + 4 * kBM - 1) / (4 * kBM);
+    y.pk_j = 2 * pg.kb2;
+    y.pk_nb = 4 * pg.kb2;
+    y.pk_v = pg.kb2;
+  }
+  e = pair ? launch_ffn_pair(1, tw2, tx_act, y, grid_y, st)
+           : launch_one<1>(tw2, tx_act, y, grid_y, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;

@@ -1,0 +1,53 @@
+// Parameters and helpers shared by the two grouped-GEMM kernels (one CTA per unit in
+// ffn_gemm.cu, an SM pair per unit in ffn_gemm_pair.cu).
+#pragma once
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+struct FfnParams {
+  const int32_t *mblk;     // row chunks {row_start, expert, live rows <= 256}
+  const int32_t *meta;     // meta[2] = number of row chunks
+  const uint32_t *flags;   // pool tile flags (streaming)
+  int32_t *status;
+  uint16_t *out;           // act (GEMM A) or ypool (GEMM Y)
+  int64_t out_ld;          // elements per row of out
+  int32_t K;               // reduction length
+  int32_t n_blocks;        // weight-column blocks per row chunk
+  int32_t col_step;        // weight columns per block
+  int32_t col1_off;        // first column of accumulator 1 inside the block's weights
+  int32_t n_out;           // output columns (I or H): masks a ragged last block
+  int32_t k_rows;          // rows per expert in the weight tensor map (H for W1, I for W2)
+  int32_t tile;            // pool tile rows
+  int32_t streaming;
+  int32_t *sched;          // {next unit ticket, CTAs done}: zero at launch, zeroed again at exit
+  int32_t packed;          // weights are moe_pack_weights tiles (one 16 KB box per tile)
+  // packed tile index = e*pk_e + nb*pk_nb + rank*pk_v + j*pk_j + kb
+  // (rank = CTA of an SM pair, j = accumulator)
+  int32_t pk_e, pk_j, pk_nb, pk_v;
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  __nv_bfloat16 b = __float2bfloat16_rn(v);
+  return *reinterpret_cast<uint16_t *>(&b);
+}
+
+// Row-major bf16 matrix [outer, inner] as a 2-D TMA tensor map, box {64, box_outer},
+// 128-byte swizzle (the canonical layout tcgen05 descriptors read). ffn_gemm.cu.
+bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+               uint32_t box_outer);
+
+// Pair-kernel launch (ffn_gemm_pair.cu): grid = 2 * clusters CTAs, clusters of two.
+cudaError_t launch_ffn_pair(int mode, const CUtensorMap &tw, const CUtensorMap &tx,
+                            const FfnParams &prm, int clusters, cudaStream_t st);
+// Clusters of two of the pair kernel that fit on the device at once (0 on error).
+int ffn_pair_max_clusters(int mode);
+
+}  // namespace moe

@@ -1,0 +1,522 @@
+// Grouped SwiGLU FFN on SM pairs: the same two GEMMs as ffn_gemm.cu (StreamEP README,
+// How it works, "CuTeDSL compute kernels": grouped GEMM A then grouped GEMM Y), with
+// each work unit computed by a cluster of two CTAs on two SMs through tcgen05's
+// cta_group::2 MMA (M = 256):
+//   GEMM A: act[p, n]   = bf16( silu(pool[p] . W1[e][:, n]) * (pool[p] . W1[e][:, I + n]) )
+//   GEMM Y: ypool[p, m] = bf16( act[p] . W2[e][:, m] )
+// for the live rows p of expert e.
+//
+// A unit is (row chunk of one expert: up to 256 live rows, block of weight columns).
+// Weights are the MMA's M operand, the chunk's rows its N operand (N = live rows rounded
+// up to 16). Each CTA of the pair holds 128 of the 256 weight columns of each MMA and
+// half of the N pool rows; each CTA's TMEM receives the accumulator rows of its own
+// 128 weight columns for all N pool rows. Two accumulators per unit:
+//   GEMM A: 256 gate columns and the same 256 up columns (block of 256 act columns;
+//           CTA r writes act columns 128 r ... 128 r + 127 of the block);
+//   GEMM Y: two adjacent blocks of 256 output columns (block of 512 columns).
+// Against one CTA per unit this halves each SM's share of the pool-row loads (per
+// k-step a CTA loads 32 KB of weights and at most 16 KB of pool rows instead of 32 +
+// 32 KB), so the 4-stage ring fits where the one-CTA kernel has 3 stages.
+//
+// Roles (10 warps per CTA, one CTA per SM):
+//   warp 0  TMA producer (both CTAs): its CTA's two weight tiles and its half of the
+//           pool rows per k-step. The first CTA's producer takes the unit tickets,
+//           writes each unit id into both CTAs' 4-slot rings, and sets the expected
+//           bytes of both CTAs' loads on its own full barrier, which the loads of
+//           both CTAs complete (cta_group::2 form of the TMA load).
+//   warp 1  both CTAs allocate 512 TMEM columns (cta_group::2). In the first CTA one
+//           thread issues the MMAs and commits each stage to the empty barriers of
+//           both CTAs and each finished unit to both CTAs' accumulator barriers.
+//   2-9     epilogue (both CTAs), as in the one-CTA kernel, over the CTA's own TMEM;
+//           a warp reports the accumulators read on the first CTA's barrier.
+// Every wait is bounded as in the one-CTA kernel (flag T, producer / MMA 2T,
+// epilogue 3T); a wait that runs out raises the abort flag of both CTAs. Both CTAs
+// leave through two cluster barriers (with a grace period between them after an
+// abort, for loads still in flight) so that neither exits while the other may still
+// write to its shared memory or barriers, and then free the TMEM.
+#include "ffn_gemm.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;                              // weight columns per CTA per accumulator
+constexpr int kBK = 64;                               // k per stage
+constexpr int kStages = 4;
+constexpr int kChunkBytes = 64 * kBK * 2;             // 8 KB: 64 weight columns x 64 k
+constexpr int kWTileBytes = 2 * kChunkBytes;          // 16 KB: one 128-column weight tile
+constexpr int kRowBox = 32;                           // pool rows per TMA box
+constexpr int kRowBoxBytes = kRowBox * kBK * 2;       // 4 KB
+constexpr int kHalfRows = kGemmBlockM / 2;            // pool rows per CTA (N / 2 <= 128)
+constexpr int kStageBytes = 2 * kWTileBytes + kHalfRows * kBK * 2;  // 48 KB
+constexpr int kTmemCols = 512;
+constexpr int kAccStride = 256;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr int kSchedSlots = 4;
+// readers of a unit id, all counted on the first CTA's sched_empty: its MMA thread and
+// epilogue warps, the second CTA's producer and epilogue warps
+constexpr int kSchedReaders = 1 + kEpiWarps + 1 + kEpiWarps;
+constexpr int kBarrierBytes = 256;
+constexpr int kXposeBytes = 32 * 32 * 2;
+constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kEpiWarps * kXposeBytes + 1024;
+constexpr uint64_t kAbortGraceNs = 1000000;           // after an abort: loads in flight land
+
+__device__ __forceinline__ void raise_abort_pair(volatile int *abort, uint32_t peer_abort,
+                                                 int32_t *status, int32_t code, int32_t aux) {
+  if (!*abort) report(status, code, aux);
+  *abort = 1;
+  st_cluster_u32(peer_abort, 1u);
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
+                         const __grid_constant__ CUtensorMap tm_x, const FfnParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  // The same offsets in both CTAs (the MMA reads both CTAs' operands at one address).
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+  uint64_t *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages;
+  uint64_t *acc_empty = acc_full + 1;
+  uint64_t *drain = acc_empty + 1;
+  uint64_t *sched_full = drain + 1;
+  uint64_t *sched_empty = sched_full + kSchedSlots;
+  int32_t *sched = reinterpret_cast<int32_t *>(sched_empty + kSchedSlots);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched + kSchedSlots);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  int *never = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const bool lead = rank == 0;
+  const uint32_t peer_abort = cluster_map(smem_u32(abort_flag), peer);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * kEpiWarps);
+    mbar_init(drain, 1);
+    for (int i = 0; i < kSchedSlots; ++i) {
+      mbar_init(sched_full + i, 1);
+      mbar_init(sched_empty + i, kSchedReaders);
+    }
+    *abort_flag = 0;
+    *never = 0;
+    fence_mbarrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  // Barriers of both CTAs are initialised and both TMEMs allocated before either CTA
+  // touches the other's.
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  volatile int *abort = abort_flag;
+
+  const int32_t n_units = prm.meta[2] * prm.n_blocks;
+  const int kb_count = prm.K / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued = 0, last_parity = 0;  // first CTA: stages whose bytes it expects
+      uint32_t sslot = 0, sphase = 0;
+      for (;;) {
+        int32_t u;
+        if (lead) {
+          if (!mbar_wait<true>(sched_empty + sslot, sphase ^ 1u, 2 * prm.timeout_ns, abort)) {
+            raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+            break;
+          }
+          const int32_t ticket = atomicAdd(prm.sched + 0, 1);
+          u = (ticket < n_units && !*abort) ? ticket : -1;
+          sched[sslot] = u;
+          st_cluster_u32(cluster_map(smem_u32(sched + sslot), peer), (uint32_t)u);
+          mbar_arrive(sched_full + sslot);
+          mbar_arrive_cluster(cluster_map(smem_u32(sched_full + sslot), peer));
+        } else {
+          if (!mbar_wait<true>(sched_full + sslot, sphase, 2 * prm.timeout_ns, abort)) {
+            raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+            break;
+          }
+          u = sched[sslot];
+          mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
+        }
+        if (++sslot == kSchedSlots) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (u < 0) break;
+        const int mb = u / prm.n_blocks;
+        const int nb = u % prm.n_blocks;
+        const int32_t row0 = prm.mblk[3 * mb + 0];
+        const int32_t e = prm.mblk[3 * mb + 1];
+        const int32_t rows = prm.mblk[3 * mb + 2];
+        const int32_t half_rows = ((rows + 15) & ~15) >> 1;   // N / 2
+        const int nbox = (half_rows + kRowBox - 1) / kRowBox;  // same in both CTAs
+        const int32_t xrow0 = row0 + (int32_t)rank * half_rows;
+        if (kMode == 0 && prm.streaming) {
+          const int32_t t_end = (row0 + rows - 1) / prm.tile;
+          for (int32_t t = row0 / prm.tile; t <= t_end && !*abort; ++t) {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t it = 0;
+            while (ld_acquire_gpu(prm.flags + t) < (uint32_t)prm.tile) {
+              if ((++it & 63u) == 0 && (*abort || globaltimer_ns() - t0 > prm.timeout_ns)) {
+                raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_FLAG_TIMEOUT, t);
+                break;
+              }
+            }
+          }
+          fence_proxy_async_global();
+          if (*abort) break;
+        }
+        const int32_t wcol0 = nb * prm.col_step + (int32_t)rank * kBM;
+        const int32_t wcol1 = wcol0 + prm.col1_off;
+        const uint32_t tx = 2u * (uint32_t)(2 * kWTileBytes + nbox * kRowBoxBytes);
+        for (int kb = 0; kb < kb_count; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1u, 2 * prm.timeout_ns, abort)) {
+            raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+            break;
+          }
+          uint8_t *sw0 = smem + stage * kStageBytes;
+          uint8_t *sw1 = sw0 + kWTileBytes;
+          uint8_t *sx = sw0 + 2 * kWTileBytes;
+          const uint32_t fb = cluster_map(smem_u32(full + stage), 0);
+          if (lead) {
+            mbar_arrive_expect_tx(full + stage, tx);
+            issued |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          if (prm.packed) {
+            const int32_t t0 =
+                e * prm.pk_e + nb * prm.pk_nb + (int32_t)rank * prm.pk_v + kb;
+            tma_load_2d_pair(sw0, &tm_w, fb, 0, t0 * 128);
+            tma_load_2d_pair(sw1, &tm_w, fb, 0, (t0 + prm.pk_j) * 128);
+          } else {
+            const int32_t krow = e * prm.k_rows + kb * kBK;
+            tma_load_2d_pair(sw0, &tm_w, fb, wcol0, krow);
+            tma_load_2d_pair(sw0 + kChunkBytes, &tm_w, fb, wcol0 + 64, krow);
+            tma_load_2d_pair(sw1, &tm_w, fb, wcol1, krow);
+            tma_load_2d_pair(sw1 + kChunkBytes, &tm_w, fb, wcol1 + 64, krow);
+          }
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d_pair(sx + i * kRowBoxBytes, &tm_x, fb, kb * kBK, xrow0 + i * kRowBox);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort) {
+        if (lead)
+          for (int s = 0; s < kStages; ++s)
+            if (issued & (1u << s))
+              mbar_wait(full + s, (last_parity >> s) & 1u, prm.timeout_ns, never);
+      } else if (lead) {
+        // Every cluster has taken its end ticket before it counts itself done, so the
+        // last one may zero the counters for the next launch.
+        __threadfence();
+        if (atomicAdd(prm.sched + 1, 1) == (int)(gridDim.x >> 1) - 1) {
+          atomicExch(prm.sched + 0, 0);
+          atomicExch(prm.sched + 1, 0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && lead) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t stage = 0, phase = 0, local = 0;
+      uint32_t sslot = 0, sphase = 0;
+      bool ok = true;
+      for (;; ++local) {
+        if (!mbar_wait(sched_full + sslot, sphase, 2 * prm.timeout_ns, abort)) {
+          raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+          break;
+        }
+        const int32_t u = sched[sslot];
+        mbar_arrive(sched_empty + sslot);
+        if (++sslot == kSchedSlots) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (u < 0) break;
+        const int mb = u / prm.n_blocks;
+        const int32_t rows = prm.mblk[3 * mb + 2];
+        const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32_ab(2 * kBM, n_mma, /*a_mn=*/true, /*b_mn=*/false);
+        // Both CTAs' epilogues have read the previous unit's accumulators.
+        if (!mbar_wait<true>(acc_empty, (local + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
+          raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < kb_count; ++kb) {
+          if (!mbar_wait(full + stage, phase, 2 * prm.timeout_ns, abort)) {
+            raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sw0 = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sw1 = sw0 + kWTileBytes;
+          const uint32_t sx = sw0 + 2 * kWTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            // weights: MN-major, 64-column chunks kChunkBytes apart, +2048 B per 16 k;
+            // pool rows: K-major 128-byte rows, 8-row groups 1024 B apart, +32 B per 16 k
+            const uint64_t xdesc = smem_desc_sw128(sx + kk * 32, 16, 1024);
+            const uint64_t w0 = smem_desc_sw128(sw0 + kk * 2048, kChunkBytes, 1024);
+            const uint64_t w1 = smem_desc_sw128(sw1 + kk * 2048, kChunkBytes, 1024);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            tc_mma_bf16_pair(tmem_base, w0, xdesc, idesc, acc);
+            tc_mma_bf16_pair(tmem_base + kAccStride, w1, xdesc, idesc, acc);
+          }
+          tc_commit_pair_mc(empty + stage, 0x3);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(acc_full, 0x3);
+      }
+      // Wait for every MMA issued by this thread before either TMEM is released.
+      tc_commit_pair_mc(drain, 0x1);
+      mbar_wait(drain, 0, prm.timeout_ns, never);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
+    uint16_t *xp = reinterpret_cast<uint16_t *>(smem + kStages * kStageBytes + kBarrierBytes) +
+                   (warp - 2) * (kXposeBytes / 2);
+    const uint32_t acc_empty_lead = cluster_map(smem_u32(acc_empty), 0);
+    uint32_t local = 0;
+    uint32_t sslot = 0, sphase = 0;
+    for (;; ++local) {
+      int32_t u = -1;
+      int got = 1;
+      if (lane == 0) {
+        got = mbar_wait_sleepy<true>(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort, 1024)
+                  ? 1
+                  : 0;
+        if (got) {
+          u = sched[sslot];
+          if (lead)
+            mbar_arrive(sched_empty + sslot);
+          else
+            mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (++sslot == kSchedSlots) {
+        sslot = 0;
+        sphase ^= 1u;
+      }
+      if (!got) {
+        if (lane == 0) raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+        break;
+      }
+      if (u < 0) break;
+      const int mb = u / prm.n_blocks;
+      const int nb = u % prm.n_blocks;
+      const int32_t row0 = prm.mblk[3 * mb + 0];
+      const int32_t rows = prm.mblk[3 * mb + 2];
+      int ok = 1;
+      if (lane == 0)
+        ok = mbar_wait_sleepy(acc_full, local & 1u, 3 * prm.timeout_ns, abort, 1024) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+        break;
+      }
+      tc_fence_after();
+      const int32_t cb0 = nb * prm.col_step + (int32_t)rank * kBM + quad * 32;
+      const int32_t cb1 = cb0 + prm.col1_off;
+      const bool ok0 = cb0 < prm.n_out;
+      const bool ok1 = kMode == 1 && cb1 < prm.n_out;
+      // First the warp's whole share of both accumulators (at most four 32-row groups)
+      // into registers as bf16 pairs (rows 2i, 2i+1 of a group in pk[.][i]), and the TMEM
+      // back to the MMA thread; then the slower turn through shared memory and the
+      // global stores, while the next unit's MMAs already run.
+      constexpr int kOuts = kMode == 0 ? 1 : 2;  // output tiles per 32-row group
+      uint32_t pk[4 * kOuts][16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int c = half * 32 + g * 64;
+        if (c < rows) {  // uniform across the warp
+          __syncwarp();
+          if (kMode == 0) {
+            uint32_t a0[32], a1[32];
+            tmem_ld_32x32b_x32(tq + c, a0);
+            tmem_ld_32x32b_x32(tq + kAccStride + c, a1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[g][i] = pack_bf16x2(
+                  silu_mul(__uint_as_float(a0[2 * i]), __uint_as_float(a1[2 * i])),
+                  silu_mul(__uint_as_float(a0[2 * i + 1]), __uint_as_float(a1[2 * i + 1])));
+          } else {
+            // one accumulator at a time: 128 registers of pairs stay live at the end
+#pragma unroll
+            for (int j = 0; j < kOuts; ++j) {
+              uint32_t a[32];
+              tmem_ld_32x32b_x32(tq + j * kAccStride + c, a);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[kOuts * g + j][i] =
+                    pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (lead)
+          mbar_arrive(acc_empty);
+        else
+          mbar_arrive_cluster(acc_empty_lead);
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int c = half * 32 + g * 64;
+        if (c < rows) {
+          const int lim = min(32, rows - c);
+#pragma unroll
+          for (int j = 0; j < kOuts; ++j) {
+            if (!(j == 0 ? ok0 : ok1)) continue;  // uniform across the warp
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint32_t v = pk[kOuts * g + j][i];
+              xp[(2 * i) * 32 + lane] = (uint16_t)(v & 0xFFFFu);
+              xp[(2 * i + 1) * 32 + lane] = (uint16_t)(v >> 16);
+            }
+            __syncwarp();
+            const int32_t cb = j == 0 ? cb0 : cb1;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int v = lane + 32 * q;
+              const int r = v >> 2;
+              const int part = v & 3;
+              if (r < lim) {
+                const uint4 val = *reinterpret_cast<const uint4 *>(xp + r * 32 + part * 8);
+                *reinterpret_cast<uint4 *>(prm.out + (size_t)(row0 + c + r) * prm.out_ld + cb +
+                                           part * 8) = val;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  // After an abort in either CTA, loads that one CTA issued may still be landing in its
+  // shared memory and on the first CTA's barriers: give them time before both exit.
+  if (threadIdx.x == 0 && (*abort || ld_cluster_u32(peer_abort) != 0u)) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kAbortGraceNs) __nanosleep(1000);
+  }
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+template <int kMode>
+cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnParams &prm,
+                        int clusters, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3(2 * clusters, 1, 1);
+  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.dynamicSmemBytes = kSmemBytes;
+  lc.stream = st;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&lc, ffn_gemm_pair_kernel<kMode>, tw, tx, prm);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int kMode>
+int max_clusters_mode() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return 0;
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    lc.gridDim = dim3(2, 1, 1);
+    lc.blockDim = dim3(kThreads, 1, 1);
+    lc.dynamicSmemBytes = kSmemBytes;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, ffn_gemm_pair_kernel<kMode>, &lc) != cudaSuccess)
+      return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_pair(int mode, const CUtensorMap &tw, const CUtensorMap &tx,
+                            const FfnParams &prm, int clusters, cudaStream_t st) {
+  return mode == 0 ? launch_mode<0>(tw, tx, prm, clusters, st)
+                   : launch_mode<1>(tw, tx, prm, clusters, st);
+}
+
+int ffn_pair_max_clusters(int mode) {
+  return mode == 0 ? max_clusters_mode<0>() : max_clusters_mode<1>();
+}
+
+}  // namespace moe

@@ -52,6 +52,13 @@ int check_plan(const moe_plan_buffers *p) {
   return MOE_OK;
 }
 
+int check_config(const moe_config &c) {
+  if (c.ffn_kernel != 0 && c.ffn_kernel != MOE_FFN_ONE_SM && c.ffn_kernel != MOE_FFN_SM_PAIR)
+    return MOE_ERR_INVALID_ARG;
+  if (c.ffn_ctas < 0 || c.wait_timeout_us < 0) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
 // Sizes (in 4-byte words) of the plan buffers, in moe_plan_buffers field order.
 void plan_sizes(const moe_shape &s, size_t words[10]) {
   const PlanGeom g = plan_geom(s);
@@ -221,10 +228,11 @@ int moe_grouped_ffn(const moe_shape *s, const void *pool, const void *W1, const 
   if (!aligned16(pool) || !aligned16(W1) || !aligned16(W2) || !aligned16(act) ||
       !aligned16(ypool))
     return MOE_ERR_MISALIGNED;
-  int nsm;
-  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
   moe_config c{};
   if (cfg != nullptr) c = *cfg;
+  if ((rc = check_config(c)) != MOE_OK) return rc;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
   return launch_ffn(*s, pool, W1, W2, *p, act, ypool, c, nsm, static_cast<cudaStream_t>(stream));
 }
 
@@ -255,6 +263,7 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
   if ((W1 == nullptr) != (W2 == nullptr)) return MOE_ERR_INVALID_ARG;
   moe_config c{};
   if (cfg != nullptr) c = *cfg;
+  if ((rc = check_config(c)) != MOE_OK) return rc;
   cudaStream_t comm = static_cast<cudaStream_t>(comm_stream);
   cudaStream_t comp = static_cast<cudaStream_t>(compute_stream);
   cudaEvent_t evp = static_cast<cudaEvent_t>(ev_plan);

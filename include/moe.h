@@ -91,6 +91,10 @@ typedef struct moe_plan_buffers {
   int32_t *status;      /* [4]          code, aux, 0, 0 (first device error wins) */
 } moe_plan_buffers;
 
+#define MOE_FFN_ONE_SM 1
+#define MOE_FFN_SM_PAIR 2
+#define MOE_FFN_DEFAULT MOE_FFN_SM_PAIR /* the kernel that moe_config.ffn_kernel = 0 selects */
+
 /* FFN launch options (all fields 0 = defaults). */
 typedef struct moe_config {
   int32_t streaming;       /* 1: the FFN claims pool tiles as their flags fill (dispatch may
@@ -100,6 +104,9 @@ typedef struct moe_config {
   int32_t wait_timeout_us; /* bound on every device-side wait; 0 = 2,000,000 us */
   int32_t packed_weights;  /* 1: W1 / W2 passed to moe_grouped_ffn / moe_forward are the
                               tiles written by moe_pack_weights, not [E,H,2I] / [E,I,H] */
+  int32_t ffn_kernel;      /* grouped-GEMM kernel: MOE_FFN_ONE_SM (one CTA per work unit,
+                              MMA M = 128) or MOE_FFN_SM_PAIR (a cluster of two CTAs on two
+                              SMs per unit, cta_group::2 MMA with M = 256); 0 = default */
   /* NULL, or 7 cudaEvent_t that moe_forward records at the phase boundaries, each on
      the stream of the kernels around it: [0] comm before plan, [1] comm after plan,
      [2] comm after dispatch, [3] compute before the FFN, [4] compute after GEMM A,

@@ -65,3 +65,25 @@ def test_misaligned_and_null_rejected_without_device():
         moe.moe_combine(s, 1 << 20, 1 << 21, bad, 1 << 22)
     assert ei.value.code == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_strerror(-11).startswith("streaming FFN")
+
+
+def test_ffn_kernel_constants_and_config_layout():
+    """The binding's constants and moe_config layout match include/moe.h; an unknown
+    grouped-GEMM kernel is rejected on the host."""
+    import combine_moe_plan_03_b200 as moe
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    defs = dict(re.findall(r"^#define (MOE_FFN_\w+) (\w+)", src, re.M))
+    assert int(defs["MOE_FFN_ONE_SM"]) == moe.MOE_FFN_ONE_SM
+    assert int(defs["MOE_FFN_SM_PAIR"]) == moe.MOE_FFN_SM_PAIR
+    assert getattr(moe, defs["MOE_FFN_DEFAULT"]) == moe.MOE_FFN_DEFAULT
+    body = re.search(r"typedef struct moe_config \{(.*?)\} moe_config;", src, re.S).group(1)
+    fields = re.findall(r"^\s*(?:int32_t|void \*const \*)\s*(\w+);", body, re.M)
+    assert fields == [f for f, _ in moe.moe_config._fields_]
+    assert moe.moe_config.timing_events.offset == 24 and ctypes.sizeof(moe.moe_config) == 32
+    s = moe.moe_shape(16, 128, 128, 8, 2, 64)
+    p = moe.moe_plan_bind(s, 1 << 20)
+    for bad in (3, -1):
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_grouped_ffn(s, 1 << 20, 1 << 21, 1 << 21, p, 1 << 22, 1 << 23,
+                                moe.moe_config(0, 0, 0, 0, bad))
+        assert ei.value.code == moe.MOE_ERR_INVALID_ARG

@@ -28,7 +28,8 @@ def test_bad_index_reported_and_pair_dropped():
     buf.close()
 
 
-def test_streaming_wait_times_out_then_context_is_usable():
+@pytest.mark.parametrize("ffn_kernel", [1, 2], ids=["one_sm", "sm_pair"])
+def test_streaming_wait_times_out_then_context_is_usable(ffn_kernel):
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import bf16_dev, f32_dev, i32_dev, weights_dev
     cfg = si.custom("to", T=128, H=128, I=128, E=4, k=2, tile=64, seed=3)
@@ -40,13 +41,14 @@ def test_streaming_wait_times_out_then_context_is_usable():
     # no dispatch: the tile flags stay 0, the streaming FFN must give up after ~1 ms
     moe.moe_grouped_ffn(buf.shape, buf.pool.data_ptr(), W1.data_ptr(), W2.data_ptr(), buf.plan,
                         buf.act.data_ptr(), buf.ypool.data_ptr(),
-                        moe.moe_config(1, 0, 1000, 0), 0)
+                        moe.moe_config(1, 0, 1000, 0, ffn_kernel), 0)
     torch.cuda.synchronize()
     code, aux = moe.moe_get_status(buf.plan)
     assert code == moe.MOE_ERR_FLAG_TIMEOUT and aux >= 0
     # the context still works: a full layer afterwards is correct
     moe.moe_clear_status(buf.plan, 0)
-    out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2)
+    out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2,
+                      moe.moe_config(0, 0, 0, 0, ffn_kernel))
     torch.cuda.synchronize()
     assert moe.moe_get_status(buf.plan)[0] == 0
     assert torch.isfinite(out.float()).all()

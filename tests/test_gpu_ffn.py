@@ -10,7 +10,7 @@ import synth_inputs as si
 pytestmark = pytest.mark.gpu
 
 
-def run_layer(cfg, streaming=0, mb=0, W=None):
+def run_layer(cfg, streaming=0, mb=0, W=None, ffn_kernel=0):
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import bf16_dev, f32_dev, i32_dev, weights_dev
     x = si.make_x(cfg, mb)
@@ -20,7 +20,7 @@ def run_layer(cfg, streaming=0, mb=0, W=None):
     for t in (buf.pool, buf.act, buf.ypool, buf.out):
         t.view(torch.int16).fill_(0x7FC0)                     # poisoned storage
     out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2,
-                      moe.moe_config(streaming, 0, 0, 0))
+                      moe.moe_config(streaming, 0, 0, 0, ffn_kernel))
     torch.cuda.synchronize()
     return buf, x, idx, w, W1, W2, out
 
@@ -44,14 +44,18 @@ SHAPES = [
 ]
 
 
+KERNELS = [1, 2]   # MOE_FFN_ONE_SM, MOE_FFN_SM_PAIR
+
+
+@pytest.mark.parametrize("ffn_kernel", KERNELS, ids=["one_sm", "sm_pair"])
 @pytest.mark.parametrize("streaming", [0, 1])
 @pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
-def test_layer_small_shapes(shape, streaming):
+def test_layer_small_shapes(shape, streaming, ffn_kernel):
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import assert_layer_close, to_f64, check_plan_exact
     name, T, H, I, E, k, tile = shape
     cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=1234 + T)
-    buf, x, idx, w, W1, W2, out = run_layer(cfg, streaming)
+    buf, x, idx, w, W1, W2, out = run_layer(cfg, streaming, ffn_kernel=ffn_kernel)
     code, aux = moe.moe_get_status(buf.plan)
     assert code == 0, (moe.moe_strerror(code), aux)
     check_plan_exact(buf, oracle.get().plan(idx, E, tile), T, k)
@@ -98,7 +102,7 @@ def test_back_to_back_layers_reuse_flags():
         ins.append((x, idx, w, bf16_dev(x), i32_dev(idx), f32_dev(w)))
     for mb in range(3):
         x, idx, w, dx, di, dw = ins[mb]
-        o = buf.forward(dx, di, dw, W1, W2, moe.moe_config(1, 0, 0, 0))
+        o = buf.forward(dx, di, dw, W1, W2, moe.moe_config(1, 0, 0, 0, 0))
         with torch.cuda.stream(buf.compute):
             outs.append(o.clone())
     torch.cuda.synchronize()

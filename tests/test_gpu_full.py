@@ -21,11 +21,12 @@ def _weights(cfg):
     return h1, h2, W1, W2
 
 
-@pytest.mark.parametrize("name,streaming,packed", [("qwen3_235b_a22b", 0, 0),
-                                                   ("qwen3_235b_a22b", 1, 1),
-                                                   ("deepseek_v3", 0, 1), ("deepseek_v3", 1, 0),
-                                                   ("decode_microbatch", 1, 1)])
-def test_full_layer(name, streaming, packed):
+# (workload, streaming, packed weights, grouped-GEMM kernel: 1 one SM, 2 SM pair)
+@pytest.mark.parametrize("name,streaming,packed,ffn_kernel", [
+    ("qwen3_235b_a22b", 0, 0, 1), ("qwen3_235b_a22b", 1, 1, 1), ("qwen3_235b_a22b", 0, 1, 2),
+    ("deepseek_v3", 0, 1, 1), ("deepseek_v3", 1, 0, 1), ("deepseek_v3", 0, 1, 2),
+    ("deepseek_v3", 1, 0, 2), ("decode_microbatch", 1, 1, 1), ("decode_microbatch", 0, 1, 2)])
+def test_full_layer(name, streaming, packed, ffn_kernel):
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import (assert_layer_close, bf16_dev, check_plan_exact, f32_dev, i32_dev,
                              sample_tokens, to_f64)
@@ -41,7 +42,7 @@ def test_full_layer(name, streaming, packed):
         x = si.make_x(cfg, mb)
         idx, w = si.make_routing(cfg, mb)
         out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2,
-                          moe.moe_config(streaming, 0, 0, packed, None))
+                          moe.moe_config(streaming, 0, 0, packed, ffn_kernel, None))
         torch.cuda.synchronize()
         code, aux = moe.moe_get_status(buf.plan)
         assert code == 0, (moe.moe_strerror(code), aux)

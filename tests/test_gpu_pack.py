@@ -60,7 +60,7 @@ def test_layer_with_packed_weights(shape):
     for st in (0, 1):
         buf.act.view(torch.int16).fill_(0x7FC0)
         out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1p, W2p,
-                          moe.moe_config(st, 0, 0, 1, None))
+                          moe.moe_config(st, 0, 0, 1, 0, None))
         torch.cuda.synchronize()
         assert moe.moe_get_status(buf.plan)[0] == 0
         ref = oracle.get().moe_forward(x, idx, w, list(W1), list(W2))
