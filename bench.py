@@ -496,15 +496,31 @@ def run_moe(args):
         kname = ("ffn_gemm_pair_kernel<0>"
                  if (ffn_kernel or moe.MOE_FFN_DEFAULT) == moe.MOE_FFN_SM_PAIR
                  else "ffn_gemm_kernel<0>")
-        line["roofline"] = {"kernel": f"{kname} (GEMM A + SwiGLU)", "bound": "tensor",
-                            "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-                            "unit": "TFLOP/s",
-                            "frac": achieved / peaks["bf16_tflops_sustained"],
-                            "traffic": committed_traffic(kname),
-                            "peak_source": f"{peak_src} bf16 sustained (timed inside a long "
-                                           "loop at the power cap)",
-                            "frac_of_burst": achieved / peaks["bf16_tflops"],
-                            "algorithmic": "useful flops pairs*4*H*I per launch"}
+        # GEMM A does 2*rows flops per weight element (2 bytes): with fewer live rows per
+        # expert than the ridge (sustained flop/s over HBM B/s) it streams weights from HBM.
+        ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        rows_per_expert = pairs_m / max(n_live_experts, 1.0)
+        if rows_per_expert >= ridge:
+            line["roofline"] = {"kernel": f"{kname} (GEMM A + SwiGLU)", "bound": "tensor",
+                                "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                                "unit": "TFLOP/s",
+                                "frac": achieved / peaks["bf16_tflops_sustained"],
+                                "traffic": committed_traffic(kname),
+                                "peak_source": f"{peak_src} bf16 sustained (timed inside a "
+                                               "long loop at the power cap)",
+                                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                                "algorithmic": "useful flops pairs*4*H*I per launch"}
+        else:
+            a_bytes = (n_live_experts * H * 2 * I * 2 + pairs_m * H * 2 + pairs_m * I * 2)
+            a_gbs = a_bytes / (ph["gemm_a"] / 1e3) / 1e9
+            line["roofline"] = {"kernel": f"{kname} (GEMM A + SwiGLU)", "bound": "hbm",
+                                "achieved": a_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": a_gbs / peaks["hbm_gbs"], "traffic": None,
+                                "peak_source": f"{peak_src} HBM copy",
+                                "algorithmic": "bytes per launch: W1 of the live experts "
+                                               "+ live pool rows read + act rows written",
+                                "rows_per_live_expert": rows_per_expert,
+                                "ridge_flop_per_byte": ridge}
     else:
         achieved = disp_bytes / (ph["dispatch"] / 1e3) / 1e9
         line["roofline"] = {"kernel": "dispatch_kernel", "bound": "hbm", "achieved": achieved,

@@ -61,6 +61,7 @@ constexpr int kBarrierBytes = 256;
 constexpr int kXposeBytes = 32 * 32 * 2;
 constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kEpiWarps * kXposeBytes + 1024;
 constexpr uint64_t kAbortGraceNs = 1000000;           // after an abort: loads in flight land
+constexpr uint32_t kParkNs = 20000;                   // epilogue waits: parked 20 us per try
 
 __device__ __forceinline__ void raise_abort_pair(volatile int *abort, uint32_t peer_abort,
                                                  int32_t *status, int32_t code, int32_t aux) {
@@ -315,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int32_t u = -1;
       int got = 1;
       if (lane == 0) {
-        got = mbar_wait_sleepy<true>(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort, 1024)
+        got = mbar_wait_parked<true>(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort,
+                                     kParkNs)
                   ? 1
                   : 0;
         if (got) {
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t rows = prm.mblk[3 * mb + 2];
       int ok = 1;
       if (lane == 0)
-        ok = mbar_wait_sleepy(acc_full, local & 1u, 3 * prm.timeout_ns, abort, 1024) ? 1 : 0;
+        ok = mbar_wait_parked(acc_full, local & 1u, 3 * prm.timeout_ns, abort, kParkNs) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);

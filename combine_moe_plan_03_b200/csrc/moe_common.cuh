@@ -143,6 +143,48 @@ __device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity,
   }
 }
 
+// try_wait with a suspend-time hint: the thread is parked by the hardware until the
+// phase completes or hint_ns pass, so a long wait neither polls nor wakes up late.
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar_addr, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  if (kCluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+        : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for waits that usually last long (a whole GEMM unit), built on
+// mbar_try_wait_hint: parked in slices of hint_ns, checking the abort flag and the
+// time budget between slices.
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait_parked(uint64_t *bar, uint32_t parity,
+                                                 uint64_t timeout_ns, const volatile int *abort,
+                                                 uint32_t hint_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_hint<kCluster>(a, parity, hint_ns)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_hint<kCluster>(a, parity, hint_ns)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
 // ---- clusters (an SM pair working on one tile) ------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

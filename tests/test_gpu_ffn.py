@@ -112,3 +112,43 @@ def test_back_to_back_layers_reuse_flags():
         ref = oracle_rows(cfg, x, idx, w, np.arange(cfg.T))
         assert_layer_close(to_f64(outs[mb]), ref, f"mb{mb}")
     buf.close()
+
+
+@pytest.mark.parametrize("ffn_kernel", KERNELS, ids=["one_sm", "sm_pair"])
+def test_act_every_live_row_within_one_bf16_ulp(ffn_kernel):
+    """GEMM A's SwiGLU output (act) on every live pool row against the oracle's
+    a = silu(g) * u in fp64, element by element: at most one bf16 ulp apart (the GPU's fp32
+    sums and its exponential / reciprocal move a by about 1e-5 relative before the final
+    rounding; near a = 0 the bound adds 1e-5 of the row's largest |a|). W1 is scaled by 4 (exact in bf16) so that g spans about [-16, 16]."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import bf16_dev, f32_dev, i32_dev, to_f64
+    cfg = si.custom("actulp", T=256, H=256, I=512, E=8, k=2, tile=64, seed=4242)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    # x4 only moves the exponent: the bf16 -> float32 -> bf16 round trip is exact
+    w1_bits = [torch.from_numpy(si.bf16_to_f64(si.make_w1_expert(cfg, e)).astype(np.float32) * 4)
+               .to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+               for e in range(cfg.E)]
+    w2_bits = [si.make_w2_expert(cfg, e) for e in range(cfg.E)]
+    W1 = bf16_dev(np.stack(w1_bits))
+    W2 = bf16_dev(np.stack(w2_bits))
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2,
+                moe.moe_config(0, 0, 0, 0, ffn_kernel))
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(buf.plan)[0] == 0
+    plan = oracle.get().plan(idx, cfg.E, cfg.tile)
+    act = to_f64(buf.act[: plan["P"]])
+    gmax = 0.0
+    for t in range(cfg.T):
+        for j in range(cfg.k):
+            e = idx[t, j]
+            g, u, a, _ = oracle.get().expert_ffn(x[t], w1_bits[e], w2_bits[e])
+            gmax = max(gmax, float(np.abs(g).max()))
+            got = act[plan["pool_row"][t, j]]
+            # one bf16 ulp of a, plus the fp32 summation error of g and u (~1e-7 of the
+            # row's scale) where a itself is near zero
+            bound = 2.0 ** -7 * np.abs(a) + 1e-5 * np.abs(a).max()
+            assert np.all(np.abs(got - a) <= bound), (t, j, float((np.abs(got - a) / bound).max()))
+    assert gmax > 10.0                      # the scaled weights reach the tails of silu
+    buf.close()
