@@ -10,14 +10,18 @@
 // Each block is one warp: lane j reads the token's j-th pool row id, lane 0 issues
 // the copies; two staging buffers let the load of the block's next token overlap
 // the stores of the current one.
-// Work items, grid-stride over E + T:
-//   item e < E    the padding rows of expert e (all in its last tile)
-//   item E + t    token t
+// Work items, grid-stride over kPadPieces*E + T, each about one token's worth of stores:
+//   item w < kPadPieces*E   padding rows 8q ... 8q + 7 (q = w % kPadPieces) of expert
+//                           w / kPadPieces (all padding rows are in the expert's last tile)
+//   item kPadPieces*E + t   token t
 // HBM traffic per call: T*H*2 read + (live pairs + padding rows)*H*2 written.
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
 namespace moe {
+
+constexpr int kPadRowsPerItem = 8;
+constexpr int kPadPieces = 128 / kPadRowsPerItem;  // covers the < tile <= 128 padding rows
 
 __device__ __forceinline__ void bulk_load_row(void *dst_smem, const void *src, uint32_t bytes,
                                               uint64_t *bar) {
@@ -72,7 +76,8 @@ __global__ void __launch_bounds__(32)
   fence_proxy_async_shared();  // the zeros and barriers, written by threads, are read by bulk copies
   __syncwarp();
 
-  const int64_t items = (int64_t)E + T;
+  const int64_t n_pad_items = (int64_t)kPadPieces * E;
+  const int64_t items = n_pad_items + T;
   const int64_t G = gridDim.x;
   // Lane 0 issues every copy. Token loads alternate between two staging buffers; the
   // load of the block's next token is issued before the current token's stores.
@@ -81,11 +86,11 @@ __global__ void __launch_bounds__(32)
   bool have = false;               // the current token's load was already issued
   bool failed = false;
   for (int64_t w = blockIdx.x; w < items && !failed; w += G) {
-    if (w < E) {
+    if (w < n_pad_items) {
       if (lane == 0) {
-        const int e = (int)w;
-        const int32_t start = offsets[e] + counts[e];
-        const int32_t end = offsets[e + 1];
+        const int e = (int)(w / kPadPieces);
+        const int32_t start = offsets[e] + counts[e] + (int32_t)(w % kPadPieces) * kPadRowsPerItem;
+        const int32_t end = min(offsets[e + 1], start + kPadRowsPerItem);
         if (end > start) {
           for (int32_t r = start; r < end; ++r)
             bulk_store_row(pool + (size_t)r * row_bytes, zeros, row_bytes);
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(32)
       }
       continue;
     }
-    const int64_t t = w - E;
+    const int64_t t = w - n_pad_items;
     const int32_t my_row = lane < k ? pool_row[t * k + lane] : -1;
     if (lane == 0) {
       if (!have) {
@@ -110,12 +115,12 @@ __global__ void __launch_bounds__(32)
       }
       const int64_t wn = w + G;
       const uint32_t nxt = cur ^ 1u;
-      const bool prefetch = wn < items && wn >= E;
+      const bool prefetch = wn < items && wn >= n_pad_items;
       if (prefetch) {
         bulk_wait_read<0>();  // the previous token's stores have read the other buffer
         mbar_arrive_expect_tx(bar + nxt, row_bytes);
-        bulk_load_row(sm + nxt * row_bytes, x + (size_t)(wn - E) * row_bytes, row_bytes,
-                      bar + nxt);
+        bulk_load_row(sm + nxt * row_bytes, x + (size_t)(wn - n_pad_items) * row_bytes,
+                      row_bytes, bar + nxt);
         ++uses[nxt];
       }
       if (!mbar_wait(bar + cur, (uses[cur] - 1u) & 1u, timeout_ns, never)) {
@@ -168,7 +173,7 @@ cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_bu
     attr_smem[dev] = smem;
   }
   const int per_sm = (int)(200 * 1024 / smem) > 0 ? (int)(200 * 1024 / smem) : 1;
-  const int64_t items = (int64_t)s.E + s.T;
+  const int64_t items = (int64_t)kPadPieces * s.E + s.T;
   int64_t grid = (int64_t)num_sms * (per_sm < 16 ? per_sm : 16);
   if (grid > items) grid = items;
   if (grid < 1) grid = 1;
