@@ -195,16 +195,18 @@ def kernel_source_hash(kernel: str = "ffn_gemm_kernel<0>") -> str:
     return h.hexdigest()[:16]
 
 
-def committed_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from a committed ncu summary, if it was taken on the
-    current kernel sources (else None: the counters are stale)."""
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu summary, if it
+    was taken on that workload and on the current kernel sources (else None: no capture,
+    or the counters are stale)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         d = json.load(open(path))
     except Exception:
         return None
     ent = d.get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
+    if (not ent or ent.get("source_hash") != kernel_source_hash(kernel)
+            or ent.get("workload") != workload):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -505,7 +507,7 @@ def run_moe(args):
                                 "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                                 "unit": "TFLOP/s",
                                 "frac": achieved / peaks["bf16_tflops_sustained"],
-                                "traffic": committed_traffic(kname),
+                                "traffic": committed_traffic(kname, cfg.name),
                                 "peak_source": f"{peak_src} bf16 sustained (timed inside a "
                                                "long loop at the power cap)",
                                 "frac_of_burst": achieved / peaks["bf16_tflops"],
@@ -526,7 +528,7 @@ def run_moe(args):
         line["roofline"] = {"kernel": "dispatch_kernel", "bound": "hbm", "achieved": achieved,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": achieved / peaks["hbm_gbs"],
-                            "traffic": committed_traffic("dispatch_kernel"),
+                            "traffic": committed_traffic("dispatch_kernel", cfg.name),
                             "peak_source": f"{peak_src} HBM copy"}
 
     # ---------------- router on the device (not part of the layer step: the layer takes
