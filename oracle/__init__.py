@@ -58,6 +58,9 @@ class Oracle:
         L.oracle_combine.restype = ctypes.c_int
         L.oracle_route.argtypes = [i64, i32, i32, vp, vp, vp, vp]
         L.oracle_route.restype = ctypes.c_int
+        L.oracle_moe_backward.argtypes = [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                          vp, ctypes.c_int]
+        L.oracle_moe_backward.restype = ctypes.c_int
         self.L = L
 
     # ---- plan -------------------------------------------------------------------------
@@ -134,6 +137,38 @@ class Oracle:
         if rc != 0:
             raise OracleError(rc)
         return y
+
+    def moe_backward(self, x_rows: np.ndarray, idx_rows: np.ndarray, w_rows: np.ndarray,
+                     W1: Sequence[Optional[np.ndarray]], W2: Sequence[Optional[np.ndarray]],
+                     dy_rows: np.ndarray, n_threads: int = 0):
+        """(dx [n, H], dw [n, k]) in float64: gradients of sum(dy * y) for the given tokens."""
+        x_rows = np.ascontiguousarray(x_rows, np.uint16)
+        idx_rows = np.ascontiguousarray(idx_rows, np.int32)
+        w_rows = np.ascontiguousarray(w_rows, np.float32)
+        dy_rows = np.ascontiguousarray(dy_rows, np.uint16)
+        n, H = x_rows.shape
+        k = idx_rows.shape[1]
+        E = len(W1)
+        I = next(w.shape[0] for w in W2 if w is not None)
+        keep = []
+        p1 = (ctypes.c_void_p * E)()
+        p2 = (ctypes.c_void_p * E)()
+        for e in range(E):
+            if W1[e] is not None:
+                a1 = np.ascontiguousarray(W1[e], np.uint16)
+                a2 = np.ascontiguousarray(W2[e], np.uint16)
+                keep += [a1, a2]
+                p1[e] = a1.ctypes.data
+                p2[e] = a2.ctypes.data
+        dx = np.empty((n, H), np.float64)
+        dw = np.empty((n, k), np.float64)
+        if n_threads <= 0:
+            n_threads = os.cpu_count() or 1
+        rc = self.L.oracle_moe_backward(n, H, I, E, k, _p(x_rows), _p(idx_rows), _p(w_rows),
+                                        p1, p2, _p(dy_rows), _p(dx), _p(dw), n_threads)
+        if rc != 0:
+            raise OracleError(rc)
+        return dx, dw
 
     def moe_forward_identity(self, x: np.ndarray, topk_idx: np.ndarray,
                              topk_w: np.ndarray) -> np.ndarray:

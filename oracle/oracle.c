@@ -20,6 +20,9 @@
  *     -> oracle_expert_ffn, oracle_moe_forward
  *   - "Per-tile streaming" / combine: each token's output is the routing-weighted
  *     sum of its k expert outputs. -> oracle_combine, oracle_moe_forward
+ *   - the backward grouped GEMMs A / Y and the backward pass mirroring dispatch and
+ *     combine: gradients of the layer with respect to x and the routing weights.
+ *     -> oracle_moe_backward
  * Readings where the README is silent (each one also listed in the design notes):
  *   - order inside an expert's pool segment: flat pair id f = t*k + j ascending;
  *   - W1[e] is [H, 2I]: columns [0, I) gate, [I, 2I) up (concatenated);
@@ -35,7 +38,9 @@
  * force of the plan, invariants, a dense all-experts brute force of the layer,
  * the E=1/k=1 textbook SwiGLU FFN against torch float64 matmuls, closed forms
  * (identity-like W1/W2, identity experts), linearity and permutation
- * equivariance, plus planted-mistake variants of this file that must fail them.
+ * equivariance; for the backward, central differences of oracle_moe_forward and
+ * torch float64 autograd on the dense E=1 layer; plus planted-mistake variants of
+ * this file that must fail them.
  */
 #include <math.h>
 #include <stddef.h>
@@ -216,6 +221,98 @@ int oracle_moe_forward(int64_t n, int32_t H, int32_t I, int32_t E, int32_t k,
     free(u);
     free(a);
     free(z);
+  }
+  return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/*
+ * Backward of the layer for a list of tokens (StreamEP README, How it works: the
+ * backward grouped GEMMs A and Y of "CuTeDSL compute kernels", and the backward pass
+ * that mirrors dispatch and combine, "Per-tile streaming"), in double. Given dy [n, H],
+ * the gradient of a loss with respect to the layer output y, and the forward values
+ * g, u, a, z of pair (t, j) with expert e (oracle_expert_ffn):
+ *   dw[t][j] = sum_m dy[t][m] * z[m]                            (routing weight)
+ *   dz[m]    = w[t][j] * dy[t][m]                               (combine, mirrored)
+ *   da[n]    = sum_m W2e[n][m] * dz[m]                          (backward Y)
+ *   dg[n]    = da[n] * u[n] * silu'(g[n]),   du[n] = da[n] * silu(g[n])
+ *   dx[t][h] = sum over the token's pairs of
+ *              sum_n W1e[h][n] * dg[n] + W1e[h][I + n] * du[n]  (backward A; dispatch,
+ *                                                                mirrored, sums the pairs)
+ * with silu'(v) = s (1 + v (1 - s)), s = 1 / (1 + exp(-v)). Sums run over their index in
+ * ascending order, pairs in j order. Dropped pairs (index -1) contribute nothing and get
+ * dw = 0. dx [n, H] and dw [n, k] are double.
+ */
+static double silu_grad(double v) {
+  double s = 1.0 / (1.0 + exp(-v));
+  return s * (1.0 + v * (1.0 - s));
+}
+
+int oracle_moe_backward(int64_t n, int32_t H, int32_t I, int32_t E, int32_t k,
+                        const uint16_t *x_rows, const int32_t *idx_rows, const float *w_rows,
+                        const uint16_t *const *W1, const uint16_t *const *W2,
+                        const uint16_t *dy_rows, double *dx, double *dw, int n_threads) {
+  if (n < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return ORACLE_ERR_ARG;
+  for (int64_t f = 0; f < n * k; ++f) {
+    int32_t e = idx_rows[f];
+    if (e < -1 || e >= E) return ORACLE_ERR_BAD_INDEX;
+    if (e >= 0 && (!W1[e] || !W2[e])) return ORACLE_ERR_MISSING_EXPERT;
+  }
+  int err = 0;
+  const int64_t two_i = 2 * (int64_t)I;
+#pragma omp parallel num_threads(n_threads > 0 ? n_threads : 1)
+  {
+    double *g = (double *)malloc(sizeof(double) * (size_t)I);
+    double *u = (double *)malloc(sizeof(double) * (size_t)I);
+    double *a = (double *)malloc(sizeof(double) * (size_t)I);
+    double *z = (double *)malloc(sizeof(double) * (size_t)H);
+    double *dz = (double *)malloc(sizeof(double) * (size_t)H);
+    double *dg = (double *)malloc(sizeof(double) * (size_t)I);
+    double *du = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!g || !u || !a || !z || !dz || !dg || !du) {
+#pragma omp atomic write
+      err = 1;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < n; ++t) {
+      if (!g || !u || !a || !z || !dz || !dg || !du) continue;
+      double *dxt = dx + t * H;
+      for (int32_t h = 0; h < H; ++h) dxt[h] = 0.0;
+      for (int32_t j = 0; j < k; ++j) {
+        int32_t e = idx_rows[t * k + j];
+        dw[t * k + j] = 0.0;
+        if (e < 0) continue;
+        oracle_expert_ffn(H, I, x_rows + t * H, W1[e], W2[e], g, u, a, z);
+        const double w = (double)w_rows[t * k + j];
+        double s = 0.0;
+        for (int32_t m = 0; m < H; ++m) {
+          const double dym = bf16_to_double(dy_rows[t * H + m]);
+          s += dym * z[m];
+          dz[m] = w * dym;
+        }
+        dw[t * k + j] = s;
+        for (int32_t q = 0; q < I; ++q) {
+          const uint16_t *w2 = W2[e] + (int64_t)q * H;
+          double da = 0.0;
+          for (int32_t m = 0; m < H; ++m) da += bf16_to_double(w2[m]) * dz[m];
+          dg[q] = da * u[q] * silu_grad(g[q]);
+          du[q] = da * silu(g[q]);
+        }
+        for (int32_t h = 0; h < H; ++h) {
+          const uint16_t *w1 = W1[e] + (int64_t)h * two_i;
+          double acc = 0.0;
+          for (int32_t q = 0; q < I; ++q)
+            acc += bf16_to_double(w1[q]) * dg[q] + bf16_to_double(w1[I + q]) * du[q];
+          dxt[h] += acc;
+        }
+      }
+    }
+    free(g);
+    free(u);
+    free(a);
+    free(z);
+    free(dz);
+    free(dg);
+    free(du);
   }
   return err ? ORACLE_ERR_ARG : ORACLE_OK;
 }

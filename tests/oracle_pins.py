@@ -351,9 +351,90 @@ def pin_route_special_cases(orc):
     np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-15)
 
 
+def _bf16_neighbours(b: int):
+    """The bf16 values just below and just above the bf16 pattern b (b not +-0)."""
+    if b & 0x8000:          # negative: a larger pattern is more negative
+        return b + 1, b - 1
+    return b - 1, b + 1
+
+
+def pin_backward_finite_differences(orc):
+    """dx and dw against central differences of the forward oracle's L = sum(dy * y).
+    x moves to its neighbouring bf16 values (the inputs stay exact bf16); y is linear in
+    w, so the difference quotient in w is exact up to rounding."""
+    rng = _rng(11)
+    T, H, I, E, k = 3, 16, 8, 3, 2
+    x, W1, W2, idx, w = _rand_layer(rng, T, H, I, E, k)
+    idx[1, 1] = -1                                   # one dropped pair
+    dy = bf16(rng.standard_normal((T, H)))
+    W1l, W2l = list(W1), list(W2)
+    dx, dw = orc.moe_backward(x, idx, w, W1l, W2l, dy, n_threads=1)
+    dyf = f64(dy)
+
+    def loss(xx, ww):
+        return float((orc.moe_forward(xx, idx, ww, W1l, W2l, n_threads=1) * dyf).sum())
+
+    fd = np.zeros_like(dx)
+    for t in range(T):
+        for h in range(H):
+            lo, hi = _bf16_neighbours(int(x[t, h]))
+            xl, xh = x.copy(), x.copy()
+            xl[t, h], xh[t, h] = lo, hi
+            step = float(f64(np.array([hi], np.uint16))[0] - f64(np.array([lo], np.uint16))[0])
+            fd[t, h] = (loss(xh, w) - loss(xl, w)) / step
+    np.testing.assert_allclose(dx, fd, rtol=0, atol=2e-3 * np.abs(fd).max())
+    for t in range(T):
+        for j in range(k):
+            d = np.float32(2.0 ** -8) * max(abs(w[t, j]), np.float32(1e-3))
+            wl, wh = w.copy(), w.copy()
+            wl[t, j] -= d
+            wh[t, j] += d
+            q = (loss(x, wh) - loss(x, wl)) / (float(wh[t, j]) - float(wl[t, j]))
+            assert abs(dw[t, j] - q) <= 1e-9 * max(1.0, abs(q)), (t, j, dw[t, j], q)
+    assert dw[1, 1] == 0.0                           # the dropped pair
+
+
+def pin_backward_textbook_torch(orc):
+    """E=1, k=1, w=1: the gradient of sum(dy * FFN(x)) for a dense SwiGLU FFN by torch
+    float64 autograd; dw is sum(dy * FFN(x)) per token."""
+    import torch
+    rng = _rng(12)
+    T, H, I = 6, 24, 16
+    x, W1, W2, _, _ = _rand_layer(rng, T, H, I, 1, 1)
+    dy = bf16(rng.standard_normal((T, H)))
+    idx = np.zeros((T, 1), np.int32)
+    w = np.ones((T, 1), np.float32)
+    dx, dw = orc.moe_backward(x, idx, w, [W1[0]], [W2[0]], dy, n_threads=1)
+    X = torch.from_numpy(f64(x)).requires_grad_(True)
+    Wg = torch.from_numpy(f64(W1[0][:, :I]))
+    Wu = torch.from_numpy(f64(W1[0][:, I:]))
+    Wd = torch.from_numpy(f64(W2[0]))
+    Y = (torch.nn.functional.silu(X @ Wg) * (X @ Wu)) @ Wd
+    D = torch.from_numpy(f64(dy))
+    (Y * D).sum().backward()
+    np.testing.assert_allclose(dx, X.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dw[:, 0], (Y * D).sum(1).detach().numpy(), rtol=1e-10,
+                               atol=1e-12)
+
+
+def pin_backward_linear_in_dy(orc):
+    """Doubling dy doubles dx and dw exactly (every operation is linear in dy and scaling
+    by 2 is exact in double); dy = 0 gives zeros."""
+    rng = _rng(13)
+    x, W1, W2, idx, w = _rand_layer(rng, 4, 16, 8, 3, 2, drop=0.25)
+    dy = bf16(rng.standard_normal((4, 16)))
+    dy2 = bf16(2.0 * f64(dy))
+    a = orc.moe_backward(x, idx, w, list(W1), list(W2), dy, n_threads=1)
+    b = orc.moe_backward(x, idx, w, list(W1), list(W2), dy2, n_threads=1)
+    assert np.array_equal(2.0 * a[0], b[0]) and np.array_equal(2.0 * a[1], b[1])
+    z = orc.moe_backward(x, idx, w, list(W1), list(W2), np.zeros_like(dy), n_threads=1)
+    assert not z[0].any() and not z[1].any()
+
+
 ALL_PINS = [
     pin_plan_worked, pin_plan_bruteforce, pin_plan_invariants, pin_plan_bad_index,
     pin_pool_gather, pin_ffn_worked, pin_ffn_dense_bruteforce, pin_ffn_textbook_torch,
     pin_ffn_closed_form, pin_ffn_linearity, pin_ffn_permutation, pin_identity_closed_form,
     pin_combine_gather, pin_route_bruteforce, pin_route_special_cases,
+    pin_backward_finite_differences, pin_backward_textbook_torch, pin_backward_linear_in_dy,
 ]

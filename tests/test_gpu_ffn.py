@@ -152,3 +152,29 @@ def test_act_every_live_row_within_one_bf16_ulp(ffn_kernel):
             assert np.all(np.abs(got - a) <= bound), (t, j, float((np.abs(got - a) / bound).max()))
     assert gmax > 10.0                      # the scaled weights reach the tails of silu
     buf.close()
+
+
+@pytest.mark.parametrize("ffn_ctas", [2, 3, 6], ids=["1cluster", "odd3", "3clusters"])
+def test_pair_kernel_few_clusters_many_units(ffn_ctas):
+    """The SM-pair kernel with 1 or 3 clusters (an odd CTA count rounds down to whole pairs):
+    every cluster runs many units in a row through the ticket ring, and the ticket
+    counters reset themselves for the next launch (two layer calls on the same plan)."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import assert_layer_close, bf16_dev, f32_dev, i32_dev, to_f64, weights_dev
+    cfg = si.custom("fewcl", T=700, H=256, I=384, E=5, k=2, tile=128, seed=777)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    c = moe.moe_config(0, ffn_ctas, 0, 0, moe.MOE_FFN_SM_PAIR)
+    ref = oracle_rows(cfg, x, idx, w, np.arange(cfg.T))
+    for call in range(2):
+        out = buf.forward(bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2, c)
+        torch.cuda.synchronize()
+        code, aux = moe.moe_get_status(buf.plan)
+        assert code == 0, (moe.moe_strerror(code), aux)
+        assert_layer_close(to_f64(out), ref, f"fewcl call{call}")
+        # both GEMMs' ticket / done counters are back to zero after each launch
+        meta = buf.plan_view("meta").cpu().numpy()
+        assert (meta[4:8] == 0).all(), meta
+    buf.close()

@@ -45,6 +45,15 @@ MUTANTS = {
                              "if (!taken[e] && (best < 0 || v[e] < v[best])) best = e;"),
     "route_bias_ignored": ("v[e] = bias ? logits[t * E + e] + bias[e] : logits[t * E + e];",
                            "v[e] = logits[t * E + e];"),
+    "bwd_silu_grad_is_sigmoid": ("return s * (1.0 + v * (1.0 - s));", "return s;"),
+    "bwd_dg_du_swapped": (
+        "acc += bf16_to_double(w1[q]) * dg[q] + bf16_to_double(w1[I + q]) * du[q];",
+        "acc += bf16_to_double(w1[q]) * du[q] + bf16_to_double(w1[I + q]) * dg[q];"),
+    "bwd_routing_weight_not_applied": ("dz[m] = w * dym;", "dz[m] = dym;"),
+    "bwd_dw_weighted": ("s += dym * z[m];", "s += w * dym * z[m];"),
+    "bwd_w2_transposed": ("da += bf16_to_double(w2[m]) * dz[m];",
+                          "da += bf16_to_double(W2[e][(int64_t)m * I + q]) * dz[m];"),
+    "bwd_du_uses_gate_only": ("du[q] = da * silu(g[q]);", "du[q] = da * g[q];"),
 }
 
 
