@@ -80,6 +80,8 @@ def _load():
         "moe_combine": [P(moe_shape), vp, vp, P(moe_plan_buffers), vp, vp],
         "moe_forward": [P(moe_shape), vp, vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp,
                         P(moe_config), vp, vp, vp, vp],
+        "moe_backward": [P(moe_shape), vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp, vp,
+                         vp, vp, P(moe_config), vp],
         "moe_events_create": [P(vp), i32],
         "moe_timing_events_create": [P(vp), i32],
         "moe_event_elapsed_ms": [vp, vp, P(ctypes.c_float)],
@@ -107,7 +109,8 @@ _lib = _load()
 
 # Names exported by include/moe.h, in declaration order.
 EXPORTS = ["moe_route", "moe_route_plan", "moe_packed_weight_bytes", "moe_pack_weights", "moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
-           "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_events_create",
+           "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_backward",
+           "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
            "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
            "moe_version"]
@@ -230,6 +233,18 @@ def moe_forward(shape, x_ptr: int, topk_idx_ptr: int, topk_w_ptr: int, w1_ptr: i
         ctypes.byref(_shape(shape)), x_ptr, topk_idx_ptr, topk_w_ptr, w1_ptr or None,
         w2_ptr or None, ctypes.byref(plan), pool_ptr, act_ptr or None, ypool_ptr or None, out_ptr,
         ctypes.byref(cfg), comm_stream or None, compute_stream or None, ev_plan, ev_dispatch))
+
+
+def moe_backward(shape, dy_ptr: int, topk_w_ptr: int, w1_ptr: int, w2_ptr: int,
+                 plan: moe_plan_buffers, pool_ptr: int, ypool_ptr: int, gu_ptr: int, dgu_ptr: int,
+                 dpool_ptr: int, dx_ptr: int, dw_ptr: int, cfg: moe_config | None,
+                 stream: int) -> None:
+    cfg = cfg or moe_config()
+    _check("moe_backward", _lib.moe_backward(
+        ctypes.byref(_shape(shape)), dy_ptr or None, topk_w_ptr or None, w1_ptr or None,
+        w2_ptr or None, ctypes.byref(plan), pool_ptr or None, ypool_ptr or None, gu_ptr or None,
+        dgu_ptr or None, dpool_ptr or None, dx_ptr or None, dw_ptr or None, ctypes.byref(cfg),
+        stream or None))
 
 
 def moe_events_create(n: int) -> list[int]:

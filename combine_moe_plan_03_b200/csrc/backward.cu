@@ -1,0 +1,92 @@
+// Backward of the layer's activation path (StreamEP README, How it works: "The backward
+// pass mirrors both overlaps" and the backward grouped GEMMs A and Y of "CuTeDSL compute
+// kernels"). Given dy = d loss / d out [T, H] and the forward call's plan, pool and ypool:
+//   combine, mirrored:   dypool[p] = bf16(w[t,j] * dy[t])  for p = pool_row[t,j]
+//                        dw[t,j]   = sum_h dy[t,h] * ypool[p,h]       (fp32)
+//   gate / up recompute: gu[p]     = bf16(pool[p] . W1[e])            (GEMM A without SwiGLU)
+//   backward Y:          da[p]     = dypool[p] . W2[e]^T, and in its epilogue
+//                        dgu[p]    = bf16(da * u * silu'(g), da * silu(g))
+//   backward A:          dpool[p]  = bf16(dgu[p] . W1[e]^T)
+//   dispatch, mirrored:  dx[t]     = bf16(sum_j dpool[pool_row[t,j]])  (fp32 sum, j order)
+// This file holds the combine backward; the GEMMs are the SM-pair kernel (ffn_gemm_pair.cu)
+// with the weights read K-major, and the dispatch backward is the combine kernel with unit
+// weights (combine.cu).
+#include "ffn_gemm.cuh"
+
+namespace moe {
+
+constexpr int kCbThreads = 128;
+
+__device__ __forceinline__ float dot_bf16x8(const uint4 &a, const uint4 &b) {
+  const uint32_t x[4] = {a.x, a.y, a.z, a.w};
+  const uint32_t y[4] = {b.x, b.y, b.z, b.w};
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s = fmaf(__uint_as_float(x[i] << 16), __uint_as_float(y[i] << 16), s);
+    s = fmaf(__uint_as_float(x[i] & 0xFFFF0000u), __uint_as_float(y[i] & 0xFFFF0000u), s);
+  }
+  return s;
+}
+
+__device__ __forceinline__ uint4 scale_bf16x8(const uint4 &a, float w) {
+  const uint32_t x[4] = {a.x, a.y, a.z, a.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    o[i] = pack_bf16x2(w * __uint_as_float(x[i] << 16), w * __uint_as_float(x[i] & 0xFFFF0000u));
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One block of 128 threads per token (grid-stride): for each live pair, thread v handles
+// 16-byte vectors v, v + 128, ... of the row: dypool = bf16(w * dy), and a partial dot
+// product of dy with ypool, reduced over the block for dw. Dropped pairs get dw = 0.
+// HBM traffic per call: T*H*2 (dy) + 2 * live pairs * H*2 (ypool read, dypool written).
+__global__ void __launch_bounds__(kCbThreads)
+    combine_backward_kernel(const uint4 *__restrict__ dy, const uint4 *__restrict__ ypool,
+                            const float *__restrict__ topk_w, const int32_t *__restrict__ pool_row,
+                            uint4 *__restrict__ dypool, float *__restrict__ dw, int32_t T,
+                            int32_t k, int32_t hv) {
+  __shared__ float s_red[kCbThreads / 32];
+  const int tid = threadIdx.x;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    for (int j = 0; j < k; ++j) {
+      const int32_t p = pool_row[t * k + j];  // uniform across the block
+      if (p < 0) {
+        if (tid == 0) dw[t * k + j] = 0.0f;
+        continue;
+      }
+      const float w = topk_w[t * k + j];
+      float part = 0.0f;
+      for (int v = tid; v < hv; v += kCbThreads) {
+        const uint4 d = dy[(size_t)t * hv + v];
+        part += dot_bf16x8(d, ypool[(size_t)p * hv + v]);
+        dypool[(size_t)p * hv + v] = scale_bf16x8(d, w);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if ((tid & 31) == 0) s_red[tid >> 5] = part;
+      __syncthreads();
+      if (tid == 0) {
+        float s = 0.0f;
+        for (int i = 0; i < kCbThreads / 32; ++i) s += s_red[i];
+        dw[t * k + j] = s;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+cudaError_t launch_combine_backward(const moe_shape &s, const void *dy, const void *ypool,
+                                    const float *topk_w, const moe_plan_buffers &p,
+                                    void *dypool, float *dw, int num_sms, cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  int64_t grid = (int64_t)num_sms * 16;
+  if (grid > s.T) grid = s.T;
+  combine_backward_kernel<<<(int)grid, kCbThreads, 0, st>>>(
+      static_cast<const uint4 *>(dy), static_cast<const uint4 *>(ypool), topk_w, p.pool_row,
+      static_cast<uint4 *>(dypool), dw, s.T, s.k, s.H / 8);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -2,6 +2,8 @@
 // a token once its expert outputs exist): out[t] = bf16(sum_j w[t,j] * ypool[row]),
 // the routing weight fused here as an fp32 fused multiply-add chain over j
 // ascending, rounded once to bf16 (nearest-even). Dropped pairs add nothing.
+// With topk_w == nullptr every weight is 1: the backward of dispatch, which sums
+// the gradients of a token's k pool rows.
 //
 // One block of 128 threads per token (grid-stride): the k row ids and weights go
 // to shared memory, then each thread gathers 16-byte vectors of the k rows (all
@@ -44,7 +46,7 @@ __global__ void __launch_bounds__(kCombThreads)
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     if (tid < k) {
       s_p[tid] = pool_row[t * k + tid];
-      s_w[tid] = topk_w[t * k + tid];
+      s_w[tid] = topk_w != nullptr ? topk_w[t * k + tid] : 1.0f;
     }
     __syncthreads();
     for (int v = tid; v < hv; v += kCombThreads) {

@@ -477,6 +477,7 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   a.col1_off = s.I;
   a.n_blocks = (s.I + kBM - 1) / kBM;
   a.n_out = s.I;
+  a.n_out1 = s.I;
   a.k_rows = s.H;
   a.tile = s.tile;
   a.streaming = cfg.streaming;
@@ -495,7 +496,7 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   a.timeout_ns = timeout_ns;
   cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(cfg.timing_events);
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t e = pair ? launch_ffn_pair(0, tw1, tx_pool, a, grid, st)
+  cudaError_t e = pair ? launch_ffn_pair(0, false, tw1, tx_pool, a, grid, st)
                        : launch_one<0>(tw1, tx_pool, a, grid, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -508,6 +509,7 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   y.col1_off = kBM;
   y.n_blocks = (s.H + 2 * kBM - 1) / (2 * kBM);
   y.n_out = s.H;
+  y.n_out1 = s.H;
   y.k_rows = s.I;
   y.streaming = 0;
   y.sched = p.meta + 6;
@@ -522,10 +524,98 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
     y.pk_nb = 4 * pg.kb2;
     y.pk_v = pg.kb2;
   }
-  e = pair ? launch_ffn_pair(1, tw2, tx_act, y, grid_y, st)
+  e = pair ? launch_ffn_pair(1, false, tw2, tx_act, y, grid_y, st)
            : launch_one<1>(tw2, tx_act, y, grid_y, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+// The backward's three grouped GEMMs on SM pairs (backward.cu has the order and the
+// formulas): gate / up recompute (W1 read MN-major, as in GEMM A), backward Y (W2 read
+// K-major, SwiGLU backward in the epilogue), backward A (W1 read K-major). dypool_dpool
+// holds dypool on entry and dpool on return.
+int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
+                        const moe_plan_buffers &p, const void *pool, void *dypool_dpool, void *gu,
+                        void *dgu, const moe_config &cfg, int num_sms, cudaStream_t st,
+                        cudaEvent_t const *tev) {
+  const PlanGeom g = plan_geom(s);
+  if (g.pmax == 0) return MOE_OK;
+  CUtensorMap tw1_mn, tw2_k, tw1_k, tx_pool, tx_dy, tx_dgu;
+  if (!make_tmap(&tw1_mn, W1, 2ull * s.I, (uint64_t)s.E * s.H, kBK) ||
+      !make_tmap(&tw2_k, W2, (uint64_t)s.H, (uint64_t)s.E * s.I, 128) ||
+      !make_tmap(&tw1_k, W1, 2ull * s.I, (uint64_t)s.E * s.H, 128) ||
+      !make_tmap(&tx_pool, pool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
+      !make_tmap(&tx_dy, dypool_dpool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
+      !make_tmap(&tx_dgu, dgu, 2ull * s.I, (uint64_t)g.pmax, kRowBox))
+    return MOE_ERR_CUDA;
+  const int fit = ffn_pair_max_clusters(0);
+  if (fit < 1) return MOE_ERR_CUDA;
+  int clusters = (cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms) / 2;
+  if (clusters < 1) clusters = 1;
+  if (clusters > fit) clusters = fit;
+  const uint64_t timeout_ns =
+      (uint64_t)(cfg.wait_timeout_us > 0 ? cfg.wait_timeout_us : 2000000) * 1000ull;
+
+  FfnParams b{};
+  b.mblk = p.mblk;
+  b.meta = p.meta;
+  b.flags = p.tile_flags;
+  b.status = p.status;
+  b.tile = s.tile;
+  b.streaming = 0;
+  b.packed = 0;
+  b.timeout_ns = timeout_ns;
+  b.col_step = 2 * kBM;
+
+  // gate / up recompute: gu[p] = [pool[p] . W1g | pool[p] . W1u]
+  FfnParams r = b;
+  r.out = static_cast<uint16_t *>(gu);
+  r.out_ld = 2 * s.I;
+  r.K = s.H;
+  r.col1_off = s.I;
+  r.n_blocks = (s.I + 2 * kBM - 1) / (2 * kBM);
+  r.n_out = s.I;
+  r.n_out1 = 2 * s.I;
+  r.k_rows = s.H;
+  r.sched = p.meta + 4;
+  if (launch_ffn_pair(1, false, tw1_mn, tx_pool, r, clusters, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[2], st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // backward Y: da = dypool . W2^T (two 256-column blocks of da), SwiGLU backward -> dgu
+  FfnParams y = b;
+  y.out = static_cast<uint16_t *>(dgu);
+  y.out_ld = 2 * s.I;
+  y.K = s.H;
+  y.col_step = 4 * kBM;
+  y.col1_off = 2 * kBM;
+  y.n_blocks = (s.I + 4 * kBM - 1) / (4 * kBM);
+  y.n_out = s.I;
+  y.n_out1 = s.I;
+  y.k_rows = s.I;
+  y.sched = p.meta + 6;
+  y.aux = static_cast<const uint16_t *>(gu);
+  y.aux_ld = 2 * s.I;
+  y.aux_off = s.I;
+  if (launch_ffn_pair(2, true, tw2_k, tx_dy, y, clusters, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // backward A: dpool = dgu . W1^T (two 256-column blocks of dpool)
+  FfnParams a = b;
+  a.out = static_cast<uint16_t *>(dypool_dpool);
+  a.out_ld = s.H;
+  a.K = 2 * s.I;
+  a.col_step = 4 * kBM;
+  a.col1_off = 2 * kBM;
+  a.n_blocks = (s.H + 4 * kBM - 1) / (4 * kBM);
+  a.n_out = s.H;
+  a.n_out1 = s.H;
+  a.k_rows = s.H;
+  a.sched = p.meta + 4;
+  if (launch_ffn_pair(1, true, tw1_k, tx_dgu, a, clusters, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -19,7 +19,9 @@ struct FfnParams {
   int32_t col_step;        // weight columns per block
   int32_t col1_off;        // first column of accumulator 1 inside the block's weights
   int32_t n_out;           // output columns (I or H): masks a ragged last block
-  int32_t k_rows;          // rows per expert in the weight tensor map (H for W1, I for W2)
+  int32_t n_out1;          // the same limit for accumulator 1's columns (SM-pair kernel)
+  int32_t k_rows;          // rows per expert in the weight tensor map ([E*H, 2I] W1: H,
+                           // [E*I, H] W2: I), whichever way the MMA reads them
   int32_t tile;            // pool tile rows
   int32_t streaming;
   int32_t *sched;          // {next unit ticket, CTAs done}: zero at launch, zeroed again at exit
@@ -28,6 +30,11 @@ struct FfnParams {
   // (rank = CTA of an SM pair, j = accumulator)
   int32_t pk_e, pk_j, pk_nb, pk_v;
   uint64_t timeout_ns;
+  // SwiGLU backward epilogue (mode 2): g at aux[p*aux_ld + n], u at aux[p*aux_ld + aux_off + n];
+  // dg and du written to out at the same offsets
+  const uint16_t *aux;
+  int64_t aux_ld;
+  int32_t aux_off;
 };
 
 // 2^x on the MUFU (ex2.approx.ftz.f32).
@@ -70,8 +77,12 @@ bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
                uint32_t box_outer);
 
 // Pair-kernel launch (ffn_gemm_pair.cu): grid = 2 * clusters CTAs, clusters of two.
-cudaError_t launch_ffn_pair(int mode, const CUtensorMap &tw, const CUtensorMap &tx,
-                            const FfnParams &prm, int clusters, cudaStream_t st);
+// mode 0: SwiGLU epilogue (GEMM A); 1: plain bf16 (GEMM Y, backward A, gate / up
+// recompute); 2: SwiGLU backward (backward Y). a_kmajor: the weights are read K-major
+// (rows of the tensor map are output columns: W2 for backward Y, W1 for backward A).
+cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
+                            const CUtensorMap &tx, const FfnParams &prm, int clusters,
+                            cudaStream_t st);
 // Clusters of two of the pair kernel that fit on the device at once (0 on error).
 int ffn_pair_max_clusters(int mode);
 

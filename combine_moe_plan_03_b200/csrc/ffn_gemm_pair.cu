@@ -70,7 +70,15 @@ __device__ __forceinline__ void raise_abort_pair(volatile int *abort, uint32_t p
   st_cluster_u32(peer_abort, 1u);
 }
 
-template <int kMode>
+// SiLU and its derivative from one sigmoid: s = 1 / (1 + e^-g) as in silu_mul.
+__device__ __forceinline__ void swiglu_backward(float da, float g, float u, float &dg, float &du) {
+  const float s = recip_newton2(1.0f + ex2_approx(fminf(g * -1.4426950408889634f, 100.0f)));
+  const float silu = g * s;
+  du = da * silu;
+  dg = da * u * (s * fmaf(g, 1.0f - s, 1.0f));
+}
+
+template <int kMode, bool kAK>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                          const __grid_constant__ CUtensorMap tm_x, const FfnParams prm) {
@@ -205,7 +213,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             issued |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           }
-          if (prm.packed) {
+          if (kAK) {
+            // K-major weights: rows of the map are output columns, 64 k per 128-byte row
+            const int32_t wrow = e * prm.k_rows + wcol0;
+            tma_load_2d_pair(sw0, &tm_w, fb, kb * kBK, wrow);
+            tma_load_2d_pair(sw1, &tm_w, fb, kb * kBK, wrow + prm.col1_off);
+          } else if (prm.packed) {
             const int32_t t0 =
                 e * prm.pk_e + nb * prm.pk_nb + (int32_t)rank * prm.pk_v + kb;
             tma_load_2d_pair(sw0, &tm_w, fb, 0, t0 * 128);
@@ -261,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int mb = u / prm.n_blocks;
         const int32_t rows = prm.mblk[3 * mb + 2];
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_f32_ab(2 * kBM, n_mma, /*a_mn=*/true, /*b_mn=*/false);
+        const uint32_t idesc = idesc_bf16_f32_ab(2 * kBM, n_mma, /*a_mn=*/!kAK, /*b_mn=*/false);
         // Both CTAs' epilogues have read the previous unit's accumulators.
         if (!mbar_wait<true>(acc_empty, (local + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
           raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
@@ -282,9 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kBK / 16; ++kk) {
             // weights: MN-major, 64-column chunks kChunkBytes apart, +2048 B per 16 k;
             // pool rows: K-major 128-byte rows, 8-row groups 1024 B apart, +32 B per 16 k
+            // (K-major weights: the same form as the pool rows)
             const uint64_t xdesc = smem_desc_sw128(sx + kk * 32, 16, 1024);
-            const uint64_t w0 = smem_desc_sw128(sw0 + kk * 2048, kChunkBytes, 1024);
-            const uint64_t w1 = smem_desc_sw128(sw1 + kk * 2048, kChunkBytes, 1024);
+            const uint64_t w0 = kAK ? smem_desc_sw128(sw0 + kk * 32, 16, 1024)
+                                    : smem_desc_sw128(sw0 + kk * 2048, kChunkBytes, 1024);
+            const uint64_t w1 = kAK ? smem_desc_sw128(sw1 + kk * 32, 16, 1024)
+                                    : smem_desc_sw128(sw1 + kk * 2048, kChunkBytes, 1024);
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
             tc_mma_bf16_pair(tmem_base, w0, xdesc, idesc, acc);
             tc_mma_bf16_pair(tmem_base + kAccStride, w1, xdesc, idesc, acc);
@@ -355,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t cb0 = nb * prm.col_step + (int32_t)rank * kBM + quad * 32;
       const int32_t cb1 = cb0 + prm.col1_off;
       const bool ok0 = cb0 < prm.n_out;
-      const bool ok1 = kMode == 1 && cb1 < prm.n_out;
+      const bool ok1 = kMode != 0 && cb1 < prm.n_out1;
       // First the warp's whole share of both accumulators (at most four 32-row groups)
       // into registers as bf16 pairs (rows 2i, 2i+1 of a group in pk[.][i]), and the TMEM
       // back to the MMA thread; then the slower turn through shared memory and the
@@ -424,8 +440,36 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int part = v & 3;
               if (r < lim) {
                 const uint4 val = *reinterpret_cast<const uint4 *>(xp + r * 32 + part * 8);
-                *reinterpret_cast<uint4 *>(prm.out + (size_t)(row0 + c + r) * prm.out_ld + cb +
-                                           part * 8) = val;
+                if (kMode != 2) {
+                  *reinterpret_cast<uint4 *>(prm.out + (size_t)(row0 + c + r) * prm.out_ld +
+                                             cb + part * 8) = val;
+                } else {
+                  const size_t o = (size_t)(row0 + c + r) * prm.out_ld + cb + part * 8;
+                  // 8 columns of one row: da from the turned block, g and u from the
+                  // saved pre-activations, dg and du to the same columns of out
+                  const size_t a = (size_t)(row0 + c + r) * prm.aux_ld + cb + part * 8;
+                  const uint4 g8 = *reinterpret_cast<const uint4 *>(prm.aux + a);
+                  const uint4 u8 = *reinterpret_cast<const uint4 *>(prm.aux + a + prm.aux_off);
+                  const uint32_t dv[4] = {val.x, val.y, val.z, val.w};
+                  const uint32_t gv[4] = {g8.x, g8.y, g8.z, g8.w};
+                  const uint32_t uv[4] = {u8.x, u8.y, u8.z, u8.w};
+                  uint32_t dgo[4], duo[4];
+#pragma unroll
+                  for (int h = 0; h < 4; ++h) {
+                    float dg0, du0, dg1, du1;
+                    swiglu_backward(__uint_as_float(dv[h] << 16), __uint_as_float(gv[h] << 16),
+                                    __uint_as_float(uv[h] << 16), dg0, du0);
+                    swiglu_backward(__uint_as_float(dv[h] & 0xFFFF0000u),
+                                    __uint_as_float(gv[h] & 0xFFFF0000u),
+                                    __uint_as_float(uv[h] & 0xFFFF0000u), dg1, du1);
+                    dgo[h] = pack_bf16x2(dg0, dg1);
+                    duo[h] = pack_bf16x2(du0, du1);
+                  }
+                  *reinterpret_cast<uint4 *>(prm.out + o) =
+                      make_uint4(dgo[0], dgo[1], dgo[2], dgo[3]);
+                  *reinterpret_cast<uint4 *>(prm.out + o + prm.aux_off) =
+                      make_uint4(duo[0], duo[1], duo[2], duo[3]);
+                }
               }
             }
           }
@@ -450,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kMode>
+template <int kMode, bool kAK>
 cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnParams &prm,
                         int clusters, cudaStream_t st) {
   static bool attr_set[64] = {false};
@@ -458,7 +502,7 @@ cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnP
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode>,
+    cudaError_t e = cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -475,18 +519,18 @@ cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnP
   lc.stream = st;
   lc.attrs = at;
   lc.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&lc, ffn_gemm_pair_kernel<kMode>, tw, tx, prm);
+  cudaError_t e = cudaLaunchKernelEx(&lc, ffn_gemm_pair_kernel<kMode, kAK>, tw, tx, prm);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <int kMode>
+template <int kMode, bool kAK>
 int max_clusters_mode() {
   static int cached[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev] == 0) {
-    if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode>,
+    if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBytes) != cudaSuccess)
       return 0;
@@ -502,7 +546,7 @@ int max_clusters_mode() {
     lc.attrs = at;
     lc.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, ffn_gemm_pair_kernel<kMode>, &lc) != cudaSuccess)
+    if (cudaOccupancyMaxActiveClusters(&n, ffn_gemm_pair_kernel<kMode, kAK>, &lc) != cudaSuccess)
       return 0;
     cached[dev] = n;
   }
@@ -511,14 +555,17 @@ int max_clusters_mode() {
 
 }  // namespace
 
-cudaError_t launch_ffn_pair(int mode, const CUtensorMap &tw, const CUtensorMap &tx,
-                            const FfnParams &prm, int clusters, cudaStream_t st) {
-  return mode == 0 ? launch_mode<0>(tw, tx, prm, clusters, st)
-                   : launch_mode<1>(tw, tx, prm, clusters, st);
+cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
+                            const CUtensorMap &tx, const FfnParams &prm, int clusters,
+                            cudaStream_t st) {
+  if (!a_kmajor)
+    return mode == 0 ? launch_mode<0, false>(tw, tx, prm, clusters, st)
+                     : launch_mode<1, false>(tw, tx, prm, clusters, st);
+  return mode == 2 ? launch_mode<2, true>(tw, tx, prm, clusters, st)
+                   : launch_mode<1, true>(tw, tx, prm, clusters, st);
 }
 
-int ffn_pair_max_clusters(int mode) {
-  return mode == 0 ? max_clusters_mode<0>() : max_clusters_mode<1>();
-}
+// All instantiations have the same block size and shared memory, hence the same count.
+int ffn_pair_max_clusters(int) { return max_clusters_mode<0, false>(); }
 
 }  // namespace moe

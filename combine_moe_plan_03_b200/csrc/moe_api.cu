@@ -251,6 +251,39 @@ int moe_combine(const moe_shape *s, const void *ypool, const float *topk_w,
   return MOE_OK;
 }
 
+int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
+                 const void *W2, const moe_plan_buffers *p, const void *pool, const void *ypool,
+                 void *gu, void *dgu, void *dpool, void *dx, float *dw, const moe_config *cfg,
+                 void *stream) {
+  int rc = check_shape(s, true);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (!W1 || !W2 || !pool || !ypool || !gu || !dgu || !dpool) return MOE_ERR_INVALID_ARG;
+  if (s->T > 0 && (!dy || !topk_w || !dx || !dw)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(W1) || !aligned16(W2) || !aligned16(pool) ||
+      !aligned16(ypool) || !aligned16(gu) || !aligned16(dgu) || !aligned16(dpool) ||
+      !aligned16(dx))
+    return MOE_ERR_MISALIGNED;
+  moe_config c{};
+  if (cfg != nullptr) c = *cfg;
+  if ((rc = check_config(c)) != MOE_OK) return rc;
+  if (c.packed_weights || c.streaming || c.ffn_kernel == MOE_FFN_ONE_SM)
+    return MOE_ERR_INVALID_ARG;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(c.timing_events);
+  if (tev != nullptr && cudaEventRecord(tev[0], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_combine_backward(*s, dy, ypool, topk_w, *p, dpool, dw, nsm, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[1], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((rc = launch_ffn_backward(*s, W1, W2, *p, pool, dpool, gu, dgu, c, nsm, st, tev)) != MOE_OK)
+    return rc;
+  if (launch_combine(*s, dpool, nullptr, *p, dx, nsm, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, const float *topk_w,
                 const void *W1, const void *W2, const moe_plan_buffers *p, void *pool, void *act,
                 void *ypool, void *out, const moe_config *cfg, void *comm_stream,

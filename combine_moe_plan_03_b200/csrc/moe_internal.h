@@ -57,6 +57,14 @@ cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_bu
                             void *pool, int signal, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const moe_shape &s, const void *ypool, const float *topk_w,
                            const moe_plan_buffers &p, void *out, int num_sms, cudaStream_t st);
+cudaError_t launch_combine_backward(const moe_shape &s, const void *dy, const void *ypool,
+                                    const float *topk_w, const moe_plan_buffers &p,
+                                    void *dypool, float *dw, int num_sms, cudaStream_t st);
+// Returns MOE_OK or a MOE_ERR_* code.
+int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
+                        const moe_plan_buffers &p, const void *pool, void *dypool_dpool, void *gu,
+                        void *dgu, const moe_config &cfg, int num_sms, cudaStream_t st,
+                        cudaEvent_t const *tev);
 // Returns MOE_OK or a MOE_ERR_* code.
 int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void *W2,
                const moe_plan_buffers &p, void *act, void *ypool, const moe_config &cfg,

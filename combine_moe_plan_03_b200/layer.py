@@ -8,9 +8,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (moe_config, moe_events_create, moe_events_destroy, moe_forward, moe_pack_weights,
-               moe_packed_weight_bytes, moe_plan_arena_bytes, moe_plan_bind, moe_pool_rows_max,
-               moe_shape)
+from . import (moe_backward, moe_config, moe_events_create, moe_events_destroy, moe_forward,
+               moe_pack_weights, moe_packed_weight_bytes, moe_plan_arena_bytes, moe_plan_bind,
+               moe_pool_rows_max, moe_shape)
 
 _PLAN_FIELDS = ("counts", "offsets", "pool_row", "row_src", "tile_expert", "mblk", "meta",
                 "tile_flags", "workspace", "status")
@@ -43,6 +43,7 @@ class MoELayerBuffers:
             streams = (torch.cuda.Stream(self.device), torch.cuda.Stream(self.device))
         self.comm, self.compute = streams
         self.events = moe_events_create(2)
+        self.gu = self.dgu = self.dpool = None      # backward work buffers, on first use
 
     def close(self):
         if self.events:
@@ -108,3 +109,30 @@ class MoELayerBuffers:
                     self.comm.cuda_stream, self.compute.cuda_stream, self.events[0],
                     self.events[1])
         return out
+
+    def backward(self, dy: torch.Tensor, topk_w: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
+                 cfg: moe_config | None = None, dx: torch.Tensor | None = None,
+                 dw: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+        """Backward of the last ``forward`` call on these buffers (its plan, pool and ypool),
+        on the compute stream: returns (dx [T, H] bf16, dw [T, k] fp32) for the upstream
+        gradient dy [T, H] bf16 (moe_backward). W1 / W2 in their given layout."""
+        s = self.shape
+        assert not self.identity
+        assert dy.dtype == torch.bfloat16 and tuple(dy.shape) == (s.T, s.H) and dy.is_contiguous()
+        assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (s.T, s.k)
+        assert tuple(W1.shape) == (s.E, s.H, 2 * s.I) and tuple(W2.shape) == (s.E, s.I, s.H)
+        bf = torch.bfloat16
+        rows = max(self.P_max, 1)
+        if self.gu is None:
+            self.gu = torch.empty((rows, 2 * s.I), dtype=bf, device=self.device)
+            self.dgu = torch.empty((rows, 2 * s.I), dtype=bf, device=self.device)
+            self.dpool = torch.empty((rows, s.H), dtype=bf, device=self.device)
+        if dx is None:
+            dx = torch.empty((max(s.T, 1), s.H), dtype=bf, device=self.device)[: s.T]
+        if dw is None:
+            dw = torch.empty((max(s.T, 1), s.k), dtype=torch.float32, device=self.device)[: s.T]
+        moe_backward(s, dy.data_ptr(), topk_w.data_ptr(), W1.data_ptr(), W2.data_ptr(), self.plan,
+                     self.pool.data_ptr(), self.ypool.data_ptr(), self.gu.data_ptr(),
+                     self.dgu.data_ptr(), self.dpool.data_ptr(), dx.data_ptr(), dw.data_ptr(), cfg,
+                     self.compute.cuda_stream)
+        return dx, dw

@@ -220,6 +220,35 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
                 void *ypool, void *out, const moe_config *cfg, void *comm_stream,
                 void *compute_stream, void *ev_plan, void *ev_dispatch);
 
+/*
+ * Backward of the layer's activation path (StreamEP README, How it works: the backward
+ * grouped GEMMs A and Y of "CuTeDSL compute kernels", and the backward pass that mirrors
+ * dispatch and combine, "Per-tile streaming"), on one stream. Given
+ *   dy [T, H] bf16        the gradient of the loss with respect to moe_forward's out,
+ *   topk_w [T, k] fp32    the routing weights of that forward call,
+ *   W1, W2                the weights in their given layout [E,H,2I] / [E,I,H] (read
+ *                         K-major here; prepacked tiles are not accepted),
+ *   p, pool, ypool        the plan buffers, pool and ypool of that forward call (it must
+ *                         have run with weights, not identity experts),
+ * it computes, with e the expert of pool row p = pool_row[t,j]:
+ *   dw[t,j]  = sum_h dy[t,h] * ypool[p,h]                       (fp32; 0 for a dropped pair)
+ *   dypool[p] = bf16(topk_w[t,j] * dy[t])                        (into dpool)
+ *   gu[p]    = bf16([pool[p] W1[e]_gate | pool[p] W1[e]_up])    (gate / up recompute)
+ *   dgu[p]   = bf16([da * u * silu'(g) | da * silu(g)]),  da = dypool[p] W2[e]^T (fp32)
+ *   dpool[p] = bf16(dgu[p] W1[e]^T)                              (overwrites dypool)
+ *   dx[t]    = bf16(sum_j dpool[pool_row[t,j]])                  (fp32 sum in j order)
+ * Work buffers (device, caller-owned, 16-byte aligned): gu and dgu [P_max, 2I] bf16,
+ * dpool [P_max, H] bf16. Outputs: dx [T, H] bf16, dw [T, k] fp32. The grouped GEMMs run on
+ * SM pairs (cfg->ffn_kernel must be 0 or MOE_FFN_SM_PAIR; cfg->packed_weights and
+ * cfg->streaming must be 0). cfg->timing_events, if set, receives on `stream`: [0] before,
+ * [1] after the combine backward, [2] after the recompute, [3] after backward Y, [4] after
+ * backward A, [5] after the dispatch backward.
+ */
+int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
+                 const void *W2, const moe_plan_buffers *p, const void *pool, const void *ypool,
+                 void *gu, void *dgu, void *dpool, void *dx, float *dw, const moe_config *cfg,
+                 void *stream);
+
 /* Create / destroy n cudaEvent_t (timing disabled) for moe_forward's ordering. */
 int moe_events_create(void **events, int32_t n);
 int moe_events_destroy(void **events, int32_t n);

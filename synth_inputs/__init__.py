@@ -39,6 +39,7 @@ STREAM_BIAS = 5
 STREAM_PERM = 6
 STREAM_DRAW = 7
 STREAM_ZLOGITS = 8
+STREAM_DY = 9        # upstream gradient of the layer output (backward)
 
 SEED_BASE = 0x5EED0000
 
@@ -235,6 +236,13 @@ def make_x(cfg: MoEConfig, micro_batch: int = 0) -> np.ndarray:
     t0 = micro_batch * cfg.T
     return normal_bf16(cfg.seed, STREAM_X, t0 * cfg.H, cfg.T * cfg.H).reshape(cfg.T, cfg.H)
 
+
+
+def make_dy(cfg: MoEConfig, mb: int = 0) -> np.ndarray:
+    """dy [T, H] bf16 ~ N(0, 1): the gradient of a loss with respect to the layer output,
+    for the backward (micro-batch mb)."""
+    n = cfg.T * cfg.H
+    return normal_bf16(cfg.seed, STREAM_DY, mb * n, n, 1.0).reshape(cfg.T, cfg.H)
 
 def make_x_rows(cfg: MoEConfig, tokens: np.ndarray, micro_batch: int = 0) -> np.ndarray:
     """Selected rows of x (global regeneration of single rows)."""

@@ -87,3 +87,26 @@ def test_ffn_kernel_constants_and_config_layout():
             moe.moe_grouped_ffn(s, 1 << 20, 1 << 21, 1 << 21, p, 1 << 22, 1 << 23,
                                 moe.moe_config(0, 0, 0, 0, bad))
         assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+
+
+def test_backward_rejects_unsupported_configs_on_the_host():
+    """moe_backward needs the weights in their given layout, no streaming, the SM-pair
+    kernels and every buffer; each violation is refused before any device work."""
+    import combine_moe_plan_03_b200 as moe
+    s = moe.moe_shape(16, 128, 128, 8, 2, 64)
+    p = moe.moe_plan_bind(s, 1 << 20)
+    ptrs = [(1 << 21) + i * (1 << 16) for i in range(11)]
+    for cfg in (moe.moe_config(0, 0, 0, 1, 0), moe.moe_config(1, 0, 0, 0, 0),
+                moe.moe_config(0, 0, 0, 0, moe.MOE_FFN_ONE_SM), moe.moe_config(0, 0, 0, 0, 9)):
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_backward(s, ptrs[0], ptrs[1], ptrs[2], ptrs[3], p, ptrs[4], ptrs[5],
+                             ptrs[6], ptrs[7], ptrs[8], ptrs[9], ptrs[10], cfg, 0)
+        assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoEError) as ei:         # a missing work buffer
+        moe.moe_backward(s, ptrs[0], ptrs[1], ptrs[2], ptrs[3], p, ptrs[4], ptrs[5], 0,
+                         ptrs[7], ptrs[8], ptrs[9], ptrs[10], None, 0)
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoEError) as ei:         # a misaligned dx
+        moe.moe_backward(s, ptrs[0], ptrs[1], ptrs[2], ptrs[3], p, ptrs[4], ptrs[5], ptrs[6],
+                         ptrs[7], ptrs[8], ptrs[9] + 4, ptrs[10], None, 0)
+    assert ei.value.code == moe.MOE_ERR_MISALIGNED

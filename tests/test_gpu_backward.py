@@ -1,0 +1,82 @@
+"""Backward of the layer's activation path (moe_backward: combine backward, gate / up
+recompute, backward Y with the SwiGLU backward, backward A, dispatch backward) against the
+oracle's fp64 gradients: dx on every token of small shapes that span several tiles and
+ragged chunks, and on sampled tokens of the full DeepSeek-V3-shaped layer; dw likewise."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2   # max |err| <= TOL * max |ref|, as for the forward
+
+
+def _close(got, ref, what):
+    scale = np.abs(ref).max()
+    err = np.abs(got - ref).max()
+    assert err <= TOL * scale, f"{what}: max err {err:.3e} vs {TOL} * {scale:.3e}"
+
+
+def _run(cfg, W1, W2, x, idx, w, dy):
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import bf16_dev, f32_dev, i32_dev
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    dw_dev = f32_dev(w)
+    buf.forward(bf16_dev(x), i32_dev(idx), dw_dev, W1, W2)
+    dx, dwg = buf.backward(bf16_dev(dy), dw_dev, W1, W2)
+    torch.cuda.synchronize()
+    code, aux = moe.moe_get_status(buf.plan)
+    assert code == 0, (moe.moe_strerror(code), aux)
+    return buf, dx, dwg
+
+
+SHAPES = [
+    # name, T, H, I, E, k, tile
+    ("tiny-like", 256, 256, 512, 8, 2, 64),
+    ("tile128-ragged", 300, 256, 256, 4, 2, 128),
+    ("I64-H192", 200, 192, 64, 3, 2, 64),
+    ("H640-I384", 150, 640, 384, 5, 3, 128),
+    ("pairs-tile64", 500, 128, 128, 3, 2, 64),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
+def test_backward_small_shapes_all_tokens(shape):
+    from gpu_helpers import to_f64, weights_dev
+    name, T, H, I, E, k, tile = shape
+    cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=4321 + T)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    idx[3, 0] = -1                                   # a dropped pair
+    dy = si.make_dy(cfg)
+    buf, dx, dw = _run(cfg, W1, W2, x, idx, w, dy)
+    W1l = [si.make_w1_expert(cfg, e) for e in range(E)]
+    W2l = [si.make_w2_expert(cfg, e) for e in range(E)]
+    rdx, rdw = oracle.get().moe_backward(x, idx, w, W1l, W2l, dy)
+    _close(to_f64(dx), rdx, f"{name} dx")
+    _close(dw.cpu().numpy().astype(np.float64), rdw, f"{name} dw")
+    assert float(dw[3, 0]) == 0.0
+    buf.close()
+
+
+def test_backward_full_deepseek_sampled_tokens():
+    """The DeepSeek-V3-shaped layer at full size: dx and dw on 24 sampled tokens."""
+    from gpu_helpers import sample_tokens, to_f64
+    from test_gpu_full import _weights
+    cfg = si.CONFIGS["deepseek_v3"]
+    h1, h2, W1, W2 = _weights(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    dy = si.make_dy(cfg)
+    buf, dx, dw = _run(cfg, W1, W2, x, idx, w, dy)
+    tok = sample_tokens(cfg.T, 24, seed=5)
+    rdx, rdw = oracle.get().moe_backward(x[tok], idx[tok], w[tok], [h1[e] for e in range(cfg.E)],
+                                         [h2[e] for e in range(cfg.E)], dy[tok])
+    sel = torch.from_numpy(tok).to(dx.device)
+    _close(to_f64(dx[sel]), rdx, "deepseek dx")
+    _close(dw[sel].cpu().numpy().astype(np.float64), rdw, "deepseek dw")
+    buf.close()
