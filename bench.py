@@ -49,6 +49,8 @@ def parse_args(argv=None):
                     help="1: prepack the weights once before timing (moe_pack_weights)")
     ap.add_argument("--ffn-kernel", type=int, default=0,
                     help="grouped-GEMM kernel: 1 one CTA per unit, 2 SM pairs; 0: default")
+    ap.add_argument("--backward", type=int, default=1,
+                    help="1: also time moe_backward (after one forward), reported under 'backward'")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=16, help="oracle tokens per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -346,6 +348,64 @@ def config_block(cfg, world):
 
 # ------------------------------------------------------------------ the CUDA path
 
+def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed, ffn_kernel,
+                  pairs, peaks, peak_src, steps):
+    """moe_backward after one forward of micro-batch 0: `steps` calls back to back with
+    per-phase CUDA events on the compute stream (max over ranks)."""
+    import ctypes
+    import torch
+    H, I, T = cfg.H, cfg.I, cfg.T
+    buf.forward(x, idx, w, W1, W2, moe.moe_config(0, 0, 0, packed, ffn_kernel, None))
+    dy = torch.from_numpy(si.make_dy(cfg).view(np.int16)).to(dev).view(torch.bfloat16)
+    gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    gw = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    plain = moe.moe_config(0, 0, 0, 0, 0, None)
+    for _ in range(3):
+        buf.backward(dy, w, W1u, W2u, plain, dx=gx, dw=gw)
+    torch.cuda.synchronize()
+    tev = moe.moe_timing_events_create(7 * steps)
+    arrs = [(ctypes.c_void_p * 7)(*tev[7 * c: 7 * c + 7]) for c in range(steps)]
+    cfgs = [moe.moe_config(0, 0, 0, 0, 0, ctypes.cast(a, ctypes.c_void_p)) for a in arrs]
+    barrier(world)
+    torch.cuda.synchronize()
+    for c in range(steps):
+        buf.backward(dy, w, W1u, W2u, cfgs[c], dx=gx, dw=gw)
+    torch.cuda.synchronize()
+    code, aux = moe.moe_get_status(buf.plan)
+    if code != 0:
+        raise RuntimeError(f"device status after the backward: {moe.moe_strerror(code)} ({aux})")
+    el = moe.moe_event_elapsed_ms
+    names = ("combine_bwd", "recompute_gu", "gemm_y_bwd", "gemm_a_bwd", "dispatch_bwd")
+    ph = {k: 0.0 for k in names}
+    for c in range(steps):
+        e = tev[7 * c: 7 * c + 7]
+        for i, k in enumerate(names):
+            ph[k] += el(e[i], e[i + 1]) / steps
+    total = el(tev[0], tev[7 * (steps - 1) + 5]) / steps
+    red = reduce_max([total] + [ph[k] for k in names], dev, world)
+    total, ph = red[0], dict(zip(names, red[1:]))
+    moe.moe_events_destroy(tev)
+    flops_gemm = pairs * 10.0 * H * I           # recompute 4HI + backward Y 2HI + backward A 4HI
+    gemm_ms = ph["recompute_gu"] + ph["gemm_y_bwd"] + ph["gemm_a_bwd"]
+    a_tf = pairs * 4.0 * H * I / (ph["gemm_a_bwd"] / 1e3) / 1e12
+    cb_bytes = T * H * 2 + 2 * pairs * H * 2 + T * cfg.k * 8
+    db_bytes = pairs * H * 2 + T * H * 2
+    return {"ms_per_call": total, "tokens_per_s": world * T / (total / 1e3),
+            "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
+            "grouped_gemms_useful_tflops": flops_gemm / (gemm_ms / 1e3) / 1e12,
+            "combine_bwd_gbs": cb_bytes / (ph["combine_bwd"] / 1e3) / 1e9,
+            "dispatch_bwd_gbs": db_bytes / (ph["dispatch_bwd"] / 1e3) / 1e9,
+            "roofline": {"kernel": "ffn_gemm_pair_kernel<1, K-major W1> (backward A)",
+                         "bound": "tensor", "achieved": a_tf,
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": a_tf / peaks["bf16_tflops_sustained"],
+                         "peak_source": f"{peak_src} bf16 sustained",
+                         "algorithmic": "useful flops pairs*4*H*I per launch"},
+            "weights": "as given (read K-major by the backward GEMMs)",
+            "calls": steps, "gpu_launches": 5 * steps,
+            "note": "after one forward; each call recomputes the same gradients"}
+
+
 def run_moe(args):
     import torch
     rank, world, local = dist_env()
@@ -386,6 +446,8 @@ def run_moe(args):
                               identity=cfg.identity)
     packed = 1 if (args.packed and not cfg.identity) else 0
     ffn_kernel = args.ffn_kernel
+    do_bwd = bool(args.backward) and not cfg.identity
+    W1u, W2u = (W1, W2) if do_bwd else (None, None)   # the backward reads the given layout
     if packed:
         # one-time layout copy (as at model load), outside every timed region
         W1, W2 = buf.pack_weights(W1, W2)
@@ -565,6 +627,13 @@ def run_moe(args):
                                                       if rank == 0 and mbs == 1 else True)}
         rb.close()
 
+    # ---------------- backward of the layer (moe_backward), timed on its own after one forward:
+    # every call recomputes the same gradients from the forward's plan, pool and ypool
+    if do_bwd:
+        line["backward"] = time_backward(moe, buf, cfg, dev, world, dx[0], didx[0], dw[0], W1,
+                                         W2, W1u, W2u, packed, ffn_kernel, pairs[0], peaks,
+                                         peak_src, args.steps)
+
     # ---------------- e2e: pinned host inputs in, result out, copies inside the timed region
     hx = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in xs]
     hidx = [torch.from_numpy(a).pin_memory() for a in idxs]
@@ -617,7 +686,7 @@ def run_moe(args):
     line["e2e"] = {"value": world * tokens_step * args.steps / (e2e_ms / 1000.0),
                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     kernels_per_call = 5 if cfg.identity else 7
-    line["gpu_launches"] = kernels_per_call * calls
+    line["gpu_launches"] = kernels_per_call * calls   # the forward's timed region
     line["clocks"] = clocks
     if want_cpu and not cfg.identity:
         line["cpu_baseline"] = cpu_baseline(cfg, xs[0], idxs[0], ws[0], host,
