@@ -350,12 +350,28 @@ def config_block(cfg, world):
 
 def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed, ffn_kernel,
                   pairs, peaks, peak_src, steps):
-    """moe_backward after one forward of micro-batch 0: `steps` calls back to back with
-    per-phase CUDA events on the compute stream (max over ranks)."""
+    """A training step of the layer on micro-batch 0: the forward that also keeps the gate /
+    up values (moe_config.gate_up) and the backward that reads them, each timed over
+    `steps` calls back to back with per-phase CUDA events (max over ranks)."""
     import ctypes
     import torch
     H, I, T = cfg.H, cfg.I, cfg.T
-    buf.forward(x, idx, w, W1, W2, moe.moe_config(0, 0, 0, packed, ffn_kernel, None))
+    fwd_ev = moe.moe_timing_events_create(7 * steps)
+    farr = [(ctypes.c_void_p * 7)(*fwd_ev[7 * c: 7 * c + 7]) for c in range(steps)]
+    fcfg = [moe.moe_config(0, 0, 0, packed, ffn_kernel, ctypes.cast(a, ctypes.c_void_p))
+            for a in farr]
+    for _ in range(3):
+        buf.forward(x, idx, w, W1, W2, moe.moe_config(0, 0, 0, packed, ffn_kernel, None),
+                    save_for_backward=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    for c in range(steps):
+        buf.forward(x, idx, w, W1, W2, fcfg[c], save_for_backward=True)
+    torch.cuda.synchronize()
+    el = moe.moe_event_elapsed_ms
+    fwd_ms = el(fwd_ev[0], fwd_ev[7 * (steps - 1) + 6]) / steps
+    fwd_gemm_a = sum(el(fwd_ev[7 * c + 3], fwd_ev[7 * c + 4]) for c in range(steps)) / steps
+    moe.moe_events_destroy(fwd_ev)
     dy = torch.from_numpy(si.make_dy(cfg).view(np.int16)).to(dev).view(torch.bfloat16)
     gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     gw = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
@@ -374,7 +390,6 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
     code, aux = moe.moe_get_status(buf.plan)
     if code != 0:
         raise RuntimeError(f"device status after the backward: {moe.moe_strerror(code)} ({aux})")
-    el = moe.moe_event_elapsed_ms
     names = ("combine_bwd", "recompute_gu", "gemm_y_bwd", "gemm_a_bwd", "dispatch_bwd")
     ph = {k: 0.0 for k in names}
     for c in range(steps):
@@ -382,15 +397,19 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
         for i, k in enumerate(names):
             ph[k] += el(e[i], e[i + 1]) / steps
     total = el(tev[0], tev[7 * (steps - 1) + 5]) / steps
-    red = reduce_max([total] + [ph[k] for k in names], dev, world)
-    total, ph = red[0], dict(zip(names, red[1:]))
+    red = reduce_max([total, fwd_ms, fwd_gemm_a] + [ph[k] for k in names], dev, world)
+    total, fwd_ms, fwd_gemm_a, ph = red[0], red[1], red[2], dict(zip(names, red[3:]))
     moe.moe_events_destroy(tev)
-    flops_gemm = pairs * 10.0 * H * I           # recompute 4HI + backward Y 2HI + backward A 4HI
-    gemm_ms = ph["recompute_gu"] + ph["gemm_y_bwd"] + ph["gemm_a_bwd"]
+    flops_gemm = pairs * 6.0 * H * I            # backward Y 2HI + backward A 4HI (g, u kept)
+    gemm_ms = ph["gemm_y_bwd"] + ph["gemm_a_bwd"]
     a_tf = pairs * 4.0 * H * I / (ph["gemm_a_bwd"] / 1e3) / 1e12
     cb_bytes = T * H * 2 + 2 * pairs * H * 2 + T * cfg.k * 8
     db_bytes = pairs * H * 2 + T * H * 2
     return {"ms_per_call": total, "tokens_per_s": world * T / (total / 1e3),
+            "train_step": {"forward_saving_gate_up_ms": fwd_ms,
+                           "forward_gemm_a_ms": fwd_gemm_a, "backward_ms": total,
+                           "ms": fwd_ms + total,
+                           "tokens_per_s": world * T / ((fwd_ms + total) / 1e3)},
             "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
             "grouped_gemms_useful_tflops": flops_gemm / (gemm_ms / 1e3) / 1e12,
             "combine_bwd_gbs": cb_bytes / (ph["combine_bwd"] / 1e3) / 1e9,
@@ -402,8 +421,9 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
                          "peak_source": f"{peak_src} bf16 sustained",
                          "algorithmic": "useful flops pairs*4*H*I per launch"},
             "weights": "as given (read K-major by the backward GEMMs)",
-            "calls": steps, "gpu_launches": 5 * steps,
-            "note": "after one forward; each call recomputes the same gradients"}
+            "calls": steps, "gpu_launches": 4 * steps,
+            "note": "after a forward that kept g | u (no recompute); every call computes the "
+                    "same gradients"}
 
 
 def run_moe(args):

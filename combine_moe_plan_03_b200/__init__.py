@@ -47,7 +47,8 @@ class moe_plan_buffers(ctypes.Structure):
 class moe_config(ctypes.Structure):
     _fields_ = [("streaming", ctypes.c_int32), ("ffn_ctas", ctypes.c_int32),
                 ("wait_timeout_us", ctypes.c_int32), ("packed_weights", ctypes.c_int32),
-                ("ffn_kernel", ctypes.c_int32), ("timing_events", ctypes.c_void_p)]
+                ("ffn_kernel", ctypes.c_int32), ("timing_events", ctypes.c_void_p),
+                ("gate_up", ctypes.c_void_p)]
 
 
 MOE_FFN_ONE_SM = 1

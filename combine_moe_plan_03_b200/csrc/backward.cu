@@ -38,42 +38,67 @@ __device__ __forceinline__ uint4 scale_bf16x8(const uint4 &a, float w) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// One block of 128 threads per token (grid-stride): for each live pair, thread v handles
-// 16-byte vectors v, v + 128, ... of the row: dypool = bf16(w * dy), and a partial dot
-// product of dy with ypool, reduced over the block for dw. Dropped pairs get dw = 0.
-// HBM traffic per call: T*H*2 (dy) + 2 * live pairs * H*2 (ypool read, dypool written).
+// One block of 128 threads per token (grid-stride); thread v owns the 16-byte vectors v,
+// v + 128, ... of the row. Per vector, dy is loaded once and the ypool vectors of up to 8
+// pairs are all loaded before they are used; each pair's dypool vector is stored and its
+// partial dot product kept in a register. One block reduction per token gives dw (0 for a
+// dropped pair). HBM traffic per call: T*H*2 (dy) + 2 * live pairs * H*2 (ypool read,
+// dypool written).
+constexpr int kCbGroup = 8;
+
 __global__ void __launch_bounds__(kCbThreads)
     combine_backward_kernel(const uint4 *__restrict__ dy, const uint4 *__restrict__ ypool,
                             const float *__restrict__ topk_w, const int32_t *__restrict__ pool_row,
                             uint4 *__restrict__ dypool, float *__restrict__ dw, int32_t T,
                             int32_t k, int32_t hv) {
-  __shared__ float s_red[kCbThreads / 32];
+  __shared__ int32_t s_p[kMaxTopK];
+  __shared__ float s_w[kMaxTopK];
+  __shared__ float s_red[kCbThreads / 32][kMaxTopK];
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    for (int j = 0; j < k; ++j) {
-      const int32_t p = pool_row[t * k + j];  // uniform across the block
-      if (p < 0) {
-        if (tid == 0) dw[t * k + j] = 0.0f;
-        continue;
-      }
-      const float w = topk_w[t * k + j];
-      float part = 0.0f;
+    if (tid < k) {
+      s_p[tid] = pool_row[t * k + tid];
+      s_w[tid] = topk_w[t * k + tid];
+    }
+    __syncthreads();
+    for (int j0 = 0; j0 < k; j0 += kCbGroup) {
+      float part[kCbGroup];
+#pragma unroll
+      for (int jj = 0; jj < kCbGroup; ++jj) part[jj] = 0.0f;
       for (int v = tid; v < hv; v += kCbThreads) {
         const uint4 d = dy[(size_t)t * hv + v];
-        part += dot_bf16x8(d, ypool[(size_t)p * hv + v]);
-        dypool[(size_t)p * hv + v] = scale_bf16x8(d, w);
+        uint4 y[kCbGroup];
+#pragma unroll
+        for (int jj = 0; jj < kCbGroup; ++jj) {
+          const int j = j0 + jj;
+          if (j < k && s_p[j] >= 0) y[jj] = ypool[(size_t)s_p[j] * hv + v];
+        }
+#pragma unroll
+        for (int jj = 0; jj < kCbGroup; ++jj) {
+          const int j = j0 + jj;
+          if (j < k && s_p[j] >= 0) {
+            part[jj] += dot_bf16x8(d, y[jj]);
+            dypool[(size_t)s_p[j] * hv + v] = scale_bf16x8(d, s_w[j]);
+          }
+        }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if ((tid & 31) == 0) s_red[tid >> 5] = part;
-      __syncthreads();
-      if (tid == 0) {
-        float s = 0.0f;
-        for (int i = 0; i < kCbThreads / 32; ++i) s += s_red[i];
-        dw[t * k + j] = s;
+      for (int jj = 0; jj < kCbGroup; ++jj) {
+        float x = part[jj];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0 && j0 + jj < k) s_red[warp][j0 + jj] = x;
       }
-      __syncthreads();
     }
+    __syncthreads();
+    if (tid < k) {
+      float sum = 0.0f;
+#pragma unroll
+      for (int i = 0; i < kCbThreads / 32; ++i) sum += s_red[i][tid];
+      dw[t * k + tid] = s_p[tid] >= 0 ? sum : 0.0f;
+    }
+    __syncthreads();
   }
 }
 

@@ -496,7 +496,16 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
   a.timeout_ns = timeout_ns;
   cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(cfg.timing_events);
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t e = pair ? launch_ffn_pair(0, false, tw1, tx_pool, a, grid, st)
+  int a_mode = 0;
+  if (cfg.gate_up != nullptr) {           // training step: also keep g | u for the backward
+    a_mode = 3;
+    a.out = static_cast<uint16_t *>(cfg.gate_up);
+    a.out_ld = 2 * s.I;
+    a.n_out1 = 2 * s.I;
+    a.out2 = static_cast<uint16_t *>(act);
+    a.out2_ld = s.I;
+  }
+  cudaError_t e = pair ? launch_ffn_pair(a_mode, false, tw1, tx_pool, a, grid, st)
                        : launch_one<0>(tw1, tx_pool, a, grid, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -568,7 +577,8 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   b.timeout_ns = timeout_ns;
   b.col_step = 2 * kBM;
 
-  // gate / up recompute: gu[p] = [pool[p] . W1g | pool[p] . W1u]
+  // gate / up recompute: gu[p] = [pool[p] . W1g | pool[p] . W1u], unless the forward kept them
+  if (cfg.gate_up != nullptr) gu = cfg.gate_up;
   FfnParams r = b;
   r.out = static_cast<uint16_t *>(gu);
   r.out_ld = 2 * s.I;
@@ -579,7 +589,8 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   r.n_out1 = 2 * s.I;
   r.k_rows = s.H;
   r.sched = p.meta + 4;
-  if (launch_ffn_pair(1, false, tw1_mn, tx_pool, r, clusters, st) != cudaSuccess)
+  if (cfg.gate_up == nullptr && launch_ffn_pair(1, false, tw1_mn, tx_pool, r, clusters, st) !=
+                                    cudaSuccess)
     return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[2], st) != cudaSuccess) return MOE_ERR_CUDA;
 

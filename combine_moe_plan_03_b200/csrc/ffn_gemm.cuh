@@ -35,6 +35,9 @@ struct FfnParams {
   const uint16_t *aux;
   int64_t aux_ld;
   int32_t aux_off;
+  // mode 3 (GEMM A saving gate / up): out = [g | u], act = bf16(silu(g) u) to out2
+  uint16_t *out2;
+  int64_t out2_ld;
 };
 
 // 2^x on the MUFU (ex2.approx.ftz.f32).
@@ -78,7 +81,7 @@ bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
 
 // Pair-kernel launch (ffn_gemm_pair.cu): grid = 2 * clusters CTAs, clusters of two.
 // mode 0: SwiGLU epilogue (GEMM A); 1: plain bf16 (GEMM Y, backward A, gate / up
-// recompute); 2: SwiGLU backward (backward Y). a_kmajor: the weights are read K-major
+// recompute); 2: SwiGLU backward (backward Y); 3: GEMM A that also stores g | u. a_kmajor: the weights are read K-major
 // (rows of the tensor map are output columns: W2 for backward Y, W1 for backward A).
 cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
                             const CUtensorMap &tx, const FfnParams &prm, int clusters,

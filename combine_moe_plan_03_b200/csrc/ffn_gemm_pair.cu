@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t half_rows = ((rows + 15) & ~15) >> 1;   // N / 2
         const int nbox = (half_rows + kRowBox - 1) / kRowBox;  // same in both CTAs
         const int32_t xrow0 = row0 + (int32_t)rank * half_rows;
-        if (kMode == 0 && prm.streaming) {
+        if ((kMode == 0 || kMode == 3) && prm.streaming) {
           const int32_t t_end = (row0 + rows - 1) / prm.tile;
           for (int32_t t = row0 / prm.tile; t <= t_end && !*abort; ++t) {
             const uint64_t t0 = globaltimer_ns();
@@ -473,6 +473,31 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
+          if (kMode == 3 && ok0) {
+            // act = bf16(silu(g) * u) from the bf16 g and u just stored, into out2; the
+            // pairs of g are overwritten by the pairs of act
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint32_t gp = pk[kOuts * g][i], up = pk[kOuts * g + 1][i];
+              pk[kOuts * g][i] = pack_bf16x2(
+                  silu_mul(__uint_as_float(gp << 16), __uint_as_float(up << 16)),
+                  silu_mul(__uint_as_float(gp & 0xFFFF0000u), __uint_as_float(up & 0xFFFF0000u)));
+              xp[(2 * i) * 32 + lane] = (uint16_t)(pk[kOuts * g][i] & 0xFFFFu);
+              xp[(2 * i + 1) * 32 + lane] = (uint16_t)(pk[kOuts * g][i] >> 16);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int v = lane + 32 * q;
+              const int r = v >> 2;
+              const int part = v & 3;
+              if (r < lim)
+                *reinterpret_cast<uint4 *>(prm.out2 + (size_t)(row0 + c + r) * prm.out2_ld +
+                                           cb0 + part * 8) =
+                    *reinterpret_cast<const uint4 *>(xp + r * 32 + part * 8);
+            }
+          }
         }
       }
     }
@@ -559,8 +584,9 @@ cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
                             const CUtensorMap &tx, const FfnParams &prm, int clusters,
                             cudaStream_t st) {
   if (!a_kmajor)
-    return mode == 0 ? launch_mode<0, false>(tw, tx, prm, clusters, st)
-                     : launch_mode<1, false>(tw, tx, prm, clusters, st);
+    return mode == 0   ? launch_mode<0, false>(tw, tx, prm, clusters, st)
+           : mode == 3 ? launch_mode<3, false>(tw, tx, prm, clusters, st)
+                       : launch_mode<1, false>(tw, tx, prm, clusters, st);
   return mode == 2 ? launch_mode<2, true>(tw, tx, prm, clusters, st)
                    : launch_mode<1, true>(tw, tx, prm, clusters, st);
 }

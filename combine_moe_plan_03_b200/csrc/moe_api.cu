@@ -56,6 +56,10 @@ int check_config(const moe_config &c) {
   if (c.ffn_kernel != 0 && c.ffn_kernel != MOE_FFN_ONE_SM && c.ffn_kernel != MOE_FFN_SM_PAIR)
     return MOE_ERR_INVALID_ARG;
   if (c.ffn_ctas < 0 || c.wait_timeout_us < 0) return MOE_ERR_INVALID_ARG;
+  if (c.gate_up != nullptr && (c.ffn_kernel == MOE_FFN_ONE_SM ||
+                               (MOE_FFN_DEFAULT == MOE_FFN_ONE_SM && c.ffn_kernel == 0)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(c.gate_up)) return MOE_ERR_MISALIGNED;
   return MOE_OK;
 }
 
@@ -258,7 +262,8 @@ int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const 
   int rc = check_shape(s, true);
   if (rc != MOE_OK) return rc;
   if ((rc = check_plan(p)) != MOE_OK) return rc;
-  if (!W1 || !W2 || !pool || !ypool || !gu || !dgu || !dpool) return MOE_ERR_INVALID_ARG;
+  if (!W1 || !W2 || !pool || !ypool || !dgu || !dpool) return MOE_ERR_INVALID_ARG;
+  if (!gu && !(cfg != nullptr && cfg->gate_up != nullptr)) return MOE_ERR_INVALID_ARG;
   if (s->T > 0 && (!dy || !topk_w || !dx || !dw)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(dy) || !aligned16(W1) || !aligned16(W2) || !aligned16(pool) ||
       !aligned16(ypool) || !aligned16(gu) || !aligned16(dgu) || !aligned16(dpool) ||

@@ -6,11 +6,17 @@ call shape (x, topk_idx, topk_weights, w1, w2, streams) on one GPU.
 """
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from . import (moe_backward, moe_config, moe_events_create, moe_events_destroy, moe_forward,
                moe_pack_weights, moe_packed_weight_bytes, moe_plan_arena_bytes, moe_plan_bind,
                moe_pool_rows_max, moe_shape)
+
+def ctypes_copy(dst: ctypes.Structure, src: ctypes.Structure) -> None:
+    ctypes.memmove(ctypes.addressof(dst), ctypes.addressof(src), ctypes.sizeof(dst))
+
 
 _PLAN_FIELDS = ("counts", "offsets", "pool_row", "row_src", "tile_expert", "mblk", "meta",
                 "tile_flags", "workspace", "status")
@@ -79,13 +85,32 @@ class MoELayerBuffers:
         self.compute.synchronize()
         return W1p, W2p
 
+    def _backward_buffers(self):
+        s = self.shape
+        if self.gu is None:
+            rows, bf = max(self.P_max, 1), torch.bfloat16
+            self.gu = torch.empty((rows, 2 * s.I), dtype=bf, device=self.device)
+            self.dgu = torch.empty((rows, 2 * s.I), dtype=bf, device=self.device)
+            self.dpool = torch.empty((rows, s.H), dtype=bf, device=self.device)
+
     def forward(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
                 W1: torch.Tensor | None, W2: torch.Tensor | None,
-                cfg: moe_config | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+                cfg: moe_config | None = None, out: torch.Tensor | None = None,
+                save_for_backward: bool = False) -> torch.Tensor:
         """Enqueue the layer (plan + dispatch on comm, FFN + combine on compute).
         Writes ``out`` [T, H] bf16 (default: this object's own buffer) and returns it; it is
-        ready once the compute stream reaches this point."""
+        ready once the compute stream reaches this point. With ``save_for_backward`` GEMM A
+        also keeps the gate / up values (``moe_config.gate_up``), so that ``backward`` need
+        not recompute them."""
         s = self.shape
+        if save_for_backward and not self.identity:
+            self._backward_buffers()
+            c = moe_config()
+            if cfg is not None:
+                ctypes_copy(c, cfg)
+            c.gate_up = self.gu.data_ptr()
+            cfg = c
+        self._gu_saved = bool(save_for_backward and not self.identity)
         if out is None:
             out = self.out[: s.T]
         assert out.dtype == torch.bfloat16 and tuple(out.shape) == (s.T, s.H) and out.is_contiguous()
@@ -122,11 +147,13 @@ class MoELayerBuffers:
         assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (s.T, s.k)
         assert tuple(W1.shape) == (s.E, s.H, 2 * s.I) and tuple(W2.shape) == (s.E, s.I, s.H)
         bf = torch.bfloat16
-        rows = max(self.P_max, 1)
-        if self.gu is None:
-            self.gu = torch.empty((rows, 2 * s.I), dtype=bf, device=self.device)
-            self.dgu = torch.empty((rows, 2 * s.I), dtype=bf, device=self.device)
-            self.dpool = torch.empty((rows, s.H), dtype=bf, device=self.device)
+        self._backward_buffers()
+        c = moe_config()
+        if cfg is not None:
+            ctypes_copy(c, cfg)
+        # the gate / up values kept by a forward(save_for_backward=True) replace the recompute
+        c.gate_up = self.gu.data_ptr() if getattr(self, "_gu_saved", False) else None
+        cfg = c
         if dx is None:
             dx = torch.empty((max(s.T, 1), s.H), dtype=bf, device=self.device)[: s.T]
         if dw is None:

@@ -113,6 +113,12 @@ typedef struct moe_config {
      [5] compute after GEMM Y, [6] compute after combine. moe_grouped_ffn records
      [3], [4], [5]. For per-kernel timing with cudaEventElapsedTime. */
   void *const *timing_events;
+  /* NULL, or a device buffer [P_max, 2I] bf16 (16-byte aligned) for the gate / up values of
+     a training step, SM-pair kernels only. moe_forward / moe_grouped_ffn: GEMM A also stores
+     [g | u] = bf16([pool W1_gate | pool W1_up]) of every live row there, and computes
+     act = bf16(silu(g) * u) from those bf16 values. moe_backward: g and u are read from
+     there (from the forward call made with the same buffer) instead of being recomputed. */
+  void *gate_up;
 } moe_config;
 
 /*

@@ -77,9 +77,10 @@ def test_ffn_kernel_constants_and_config_layout():
     assert int(defs["MOE_FFN_SM_PAIR"]) == moe.MOE_FFN_SM_PAIR
     assert getattr(moe, defs["MOE_FFN_DEFAULT"]) == moe.MOE_FFN_DEFAULT
     body = re.search(r"typedef struct moe_config \{(.*?)\} moe_config;", src, re.S).group(1)
-    fields = re.findall(r"^\s*(?:int32_t|void \*const \*)\s*(\w+);", body, re.M)
+    fields = re.findall(r"^\s*(?:int32_t|void \*const \*|void \*)\s*(\w+);", body, re.M)
     assert fields == [f for f, _ in moe.moe_config._fields_]
-    assert moe.moe_config.timing_events.offset == 24 and ctypes.sizeof(moe.moe_config) == 32
+    assert moe.moe_config.timing_events.offset == 24 and moe.moe_config.gate_up.offset == 32
+    assert ctypes.sizeof(moe.moe_config) == 40
     s = moe.moe_shape(16, 128, 128, 8, 2, 64)
     p = moe.moe_plan_bind(s, 1 << 20)
     for bad in (3, -1):

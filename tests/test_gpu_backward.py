@@ -80,3 +80,43 @@ def test_backward_full_deepseek_sampled_tokens():
     _close(to_f64(dx[sel]), rdx, "deepseek dx")
     _close(dw[sel].cpu().numpy().astype(np.float64), rdw, "deepseek dw")
     buf.close()
+
+
+@pytest.mark.parametrize("shape", SHAPES[:3], ids=[s[0] for s in SHAPES[:3]])
+def test_forward_saving_gate_up_then_backward(shape):
+    """A training step: forward with save_for_backward (GEMM A also stores g | u and makes
+    act from them), then the backward without the recompute. The forward output, the saved
+    g and u, dx and dw all against the oracle."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import assert_layer_close, bf16_dev, f32_dev, i32_dev, to_f64, weights_dev
+    name, T, H, I, E, k, tile = shape
+    cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=999 + T)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    dy = si.make_dy(cfg)
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    wd = f32_dev(w)
+    out = buf.forward(bf16_dev(x), i32_dev(idx), wd, W1, W2, save_for_backward=True)
+    dx, dw = buf.backward(bf16_dev(dy), wd, W1, W2)
+    torch.cuda.synchronize()
+    code, aux = moe.moe_get_status(buf.plan)
+    assert code == 0, (moe.moe_strerror(code), aux)
+    W1l = [si.make_w1_expert(cfg, e) for e in range(E)]
+    W2l = [si.make_w2_expert(cfg, e) for e in range(E)]
+    ref = oracle.get().moe_forward(x, idx, w, W1l, W2l)
+    assert_layer_close(to_f64(out), ref, f"{name} forward")
+    plan = oracle.get().plan(idx, E, tile)
+    gu = to_f64(buf.gu[: plan["P"]])
+    for f in (0, 7, T * k - 1):
+        t, j = divmod(f, k)
+        if idx[t, j] < 0:
+            continue
+        g, u, _, _ = oracle.get().expert_ffn(x[t], W1l[idx[t, j]], W2l[idx[t, j]])
+        row = gu[plan["pool_row"][t, j]]
+        for got, want in ((row[:I], g), (row[I:], u)):
+            assert np.all(np.abs(got - want) <= 2.0 ** -7 * np.abs(want) + 1e-5 * np.abs(want).max())
+    rdx, rdw = oracle.get().moe_backward(x, idx, w, W1l, W2l, dy)
+    _close(to_f64(dx), rdx, f"{name} dx")
+    _close(dw.cpu().numpy().astype(np.float64), rdw, f"{name} dw")
+    buf.close()
