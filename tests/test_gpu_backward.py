@@ -120,3 +120,57 @@ def test_forward_saving_gate_up_then_backward(shape):
     _close(to_f64(dx), rdx, f"{name} dx")
     _close(dw.cpu().numpy().astype(np.float64), rdw, f"{name} dw")
     buf.close()
+
+
+EDGE = [
+    # name, T, H, I, E, k, tile, drop (fraction of pairs set to -1)
+    ("k16", 64, 128, 128, 32, 16, 64, 0.0),         # two groups of 8 pairs per token
+    ("E1-k1", 100, 128, 192, 1, 1, 128, 0.0),       # one expert: a dense SwiGLU FFN
+    ("half-dropped", 90, 128, 128, 4, 2, 64, 0.5),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_backward_edge_cases(case):
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import to_f64, weights_dev
+    name, T, H, I, E, k, tile, drop = case
+    cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=2024 + T)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    if drop:
+        rng = np.random.default_rng(7)
+        idx[rng.random(idx.shape) < drop] = -1
+    dy = si.make_dy(cfg)
+    buf, dx, dw = _run(cfg, W1, W2, x, idx, w, dy)
+    W1l = [si.make_w1_expert(cfg, e) for e in range(E)]
+    W2l = [si.make_w2_expert(cfg, e) for e in range(E)]
+    rdx, rdw = oracle.get().moe_backward(x, idx, w, W1l, W2l, dy)
+    _close(to_f64(dx), rdx, f"{name} dx")
+    _close(dw.cpu().numpy().astype(np.float64), rdw, f"{name} dw")
+    assert np.all(dw.cpu().numpy()[idx < 0] == 0.0)
+    buf.close()
+
+
+def test_backward_no_live_pairs_and_no_tokens():
+    """Every pair dropped: dx = 0 and dw = 0 with no device error. T = 0: nothing to do."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import bf16_dev, f32_dev, i32_dev, weights_dev
+    cfg = si.custom("alldrop", T=40, H=128, I=128, E=4, k=2, tile=64, seed=5)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    idx[:] = -1
+    buf, dx, dw = _run(cfg, W1, W2, x, idx, w, si.make_dy(cfg))
+    assert not dx.float().abs().sum().item() and not dw.abs().sum().item()
+    buf.close()
+    buf = moe.MoELayerBuffers(0, 128, 128, 4, 2, 64)
+    e = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    ei = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+    ew = torch.empty((0, 2), dtype=torch.float32, device="cuda")
+    buf.forward(e, ei, ew, W1, W2)
+    dx, dw = buf.backward(e, ew, W1, W2)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(buf.plan)[0] == 0 and dx.numel() == 0 and dw.numel() == 0
+    buf.close()
