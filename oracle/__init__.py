@@ -61,6 +61,9 @@ class Oracle:
         L.oracle_moe_backward.argtypes = [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp,
                                           vp, ctypes.c_int]
         L.oracle_moe_backward.restype = ctypes.c_int
+        L.oracle_expert_weight_grads.argtypes = [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp,
+                                                 i32, vp, vp, vp]
+        L.oracle_expert_weight_grads.restype = ctypes.c_int
         self.L = L
 
     # ---- plan -------------------------------------------------------------------------
@@ -169,6 +172,27 @@ class Oracle:
         if rc != 0:
             raise OracleError(rc)
         return dx, dw
+
+    def expert_weight_grads(self, x: np.ndarray, topk_idx: np.ndarray, topk_w: np.ndarray,
+                            W1e: np.ndarray, W2e: np.ndarray, e: int, dy: np.ndarray):
+        """(dW1 [H, 2I], dW2 [I, H]) in float64 for expert e, over all tokens of the call."""
+        x = np.ascontiguousarray(x, np.uint16)
+        idx = np.ascontiguousarray(topk_idx, np.int32)
+        w = np.ascontiguousarray(topk_w, np.float32)
+        W1e = np.ascontiguousarray(W1e, np.uint16)
+        W2e = np.ascontiguousarray(W2e, np.uint16)
+        dy = np.ascontiguousarray(dy, np.uint16)
+        T, H = x.shape
+        k = idx.shape[1]
+        I = W2e.shape[0]
+        dW1 = np.empty((H, 2 * I), np.float64)
+        dW2 = np.empty((I, H), np.float64)
+        E = int(max(idx.max(initial=0), e)) + 1
+        rc = self.L.oracle_expert_weight_grads(T, H, I, E, k, _p(x), _p(idx), _p(w), _p(W1e),
+                                               _p(W2e), e, _p(dy), _p(dW1), _p(dW2))
+        if rc != 0:
+            raise OracleError(rc)
+        return dW1, dW2
 
     def moe_forward_identity(self, x: np.ndarray, topk_idx: np.ndarray,
                              topk_w: np.ndarray) -> np.ndarray:

@@ -22,7 +22,8 @@
  *     sum of its k expert outputs. -> oracle_combine, oracle_moe_forward
  *   - the backward grouped GEMMs A / Y and the backward pass mirroring dispatch and
  *     combine: gradients of the layer with respect to x and the routing weights.
- *     -> oracle_moe_backward
+ *     -> oracle_moe_backward; the weight gradients of one expert.
+ *     -> oracle_expert_weight_grads
  * Readings where the README is silent (each one also listed in the design notes):
  *   - order inside an expert's pool segment: flat pair id f = t*k + j ascending;
  *   - W1[e] is [H, 2I]: columns [0, I) gate, [I, 2I) up (concatenated);
@@ -315,6 +316,71 @@ int oracle_moe_backward(int64_t n, int32_t H, int32_t I, int32_t E, int32_t k,
     free(du);
   }
   return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/*
+ * Weight gradients of one expert e (the backward's weight GEMMs), in double, from the same
+ * per-pair values as oracle_moe_backward:
+ *   dW1[h][n]     = sum over the pairs (t, j) with topk_idx[t][j] == e of x[t][h] * dg[n]
+ *   dW1[h][I + n] = the same sum of x[t][h] * du[n]
+ *   dW2[n][m]     = the same sum of a[n] * dz[m],   dz = w[t][j] * dy[t]
+ * pairs in flat-pair order t*k + j ascending. dW1 [H, 2I] and dW2 [I, H] are double.
+ */
+int oracle_expert_weight_grads(int64_t T, int32_t H, int32_t I, int32_t E, int32_t k,
+                               const uint16_t *x, const int32_t *topk_idx, const float *topk_w,
+                               const uint16_t *W1e, const uint16_t *W2e, int32_t e,
+                               const uint16_t *dy, double *dW1, double *dW2) {
+  if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || e < 0 || e >= E) return ORACLE_ERR_ARG;
+  const int64_t two_i = 2 * (int64_t)I;
+  double *g = (double *)malloc(sizeof(double) * (size_t)I);
+  double *u = (double *)malloc(sizeof(double) * (size_t)I);
+  double *a = (double *)malloc(sizeof(double) * (size_t)I);
+  double *z = (double *)malloc(sizeof(double) * (size_t)H);
+  double *dz = (double *)malloc(sizeof(double) * (size_t)H);
+  double *dg = (double *)malloc(sizeof(double) * (size_t)I);
+  double *du = (double *)malloc(sizeof(double) * (size_t)I);
+  int rc = ORACLE_OK;
+  if (!g || !u || !a || !z || !dz || !dg || !du) rc = ORACLE_ERR_ARG;
+  for (int64_t i = 0; rc == ORACLE_OK && i < (int64_t)H * two_i; ++i) dW1[i] = 0.0;
+  for (int64_t i = 0; rc == ORACLE_OK && i < (int64_t)I * H; ++i) dW2[i] = 0.0;
+  for (int64_t f = 0; rc == ORACLE_OK && f < T * k; ++f) {
+    if (topk_idx[f] < -1 || topk_idx[f] >= E) {
+      rc = ORACLE_ERR_BAD_INDEX;
+      break;
+    }
+    if (topk_idx[f] != e) continue;
+    const int64_t t = f / k;
+    oracle_expert_ffn(H, I, x + t * H, W1e, W2e, g, u, a, z);
+    const double w = (double)topk_w[f];
+    for (int32_t m = 0; m < H; ++m) dz[m] = w * bf16_to_double(dy[t * H + m]);
+    for (int32_t q = 0; q < I; ++q) {
+      const uint16_t *w2 = W2e + (int64_t)q * H;
+      double da = 0.0;
+      for (int32_t m = 0; m < H; ++m) da += bf16_to_double(w2[m]) * dz[m];
+      dg[q] = da * u[q] * silu_grad(g[q]);
+      du[q] = da * silu(g[q]);
+    }
+    for (int32_t h = 0; h < H; ++h) {
+      const double xh = bf16_to_double(x[t * H + h]);
+      double *row = dW1 + (int64_t)h * two_i;
+      for (int32_t q = 0; q < I; ++q) {
+        row[q] += xh * dg[q];
+        row[I + q] += xh * du[q];
+      }
+    }
+    for (int32_t q = 0; q < I; ++q) {
+      double *row = dW2 + (int64_t)q * H;
+      for (int32_t m = 0; m < H; ++m) row[m] += a[q] * dz[m];
+    }
+  }
+  free(g);
+  free(u);
+  free(a);
+  free(z);
+  free(dz);
+  free(dg);
+  free(du);
+  return rc;
 }
 
 /*

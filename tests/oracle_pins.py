@@ -431,10 +431,59 @@ def pin_backward_linear_in_dy(orc):
     assert not z[0].any() and not z[1].any()
 
 
+def pin_weight_grads_finite_differences(orc):
+    """dW1 and dW2 of one expert against central differences of the forward oracle's
+    L = sum(dy * y), each weight moved to its neighbouring bf16 values."""
+    rng = _rng(14)
+    T, H, I, E, k = 5, 8, 4, 3, 2
+    x, W1, W2, idx, w = _rand_layer(rng, T, H, I, E, k)
+    idx[2, 1] = -1
+    e = int(idx[0, 0])
+    dy = bf16(rng.standard_normal((T, H)))
+    dW1, dW2 = orc.expert_weight_grads(x, idx, w, W1[e], W2[e], e, dy)
+    dyf = f64(dy)
+
+    def loss(W1m, W2m):
+        return float((orc.moe_forward(x, idx, w, list(W1m), list(W2m), n_threads=1) * dyf).sum())
+
+    for name, W, dW in (("W1", W1, dW1), ("W2", W2, dW2)):
+        fd = np.zeros_like(dW)
+        for pos in np.ndindex(*dW.shape):
+            lo, hi = _bf16_neighbours(int(W[e][pos]))
+            Wl, Wh = W.copy(), W.copy()
+            Wl[e][pos], Wh[e][pos] = lo, hi
+            step = float(f64(np.array([hi], np.uint16))[0] - f64(np.array([lo], np.uint16))[0])
+            if name == "W1":
+                fd[pos] = (loss(Wh, W2) - loss(Wl, W2)) / step
+            else:
+                fd[pos] = (loss(W1, Wh) - loss(W1, Wl)) / step
+        np.testing.assert_allclose(dW, fd, rtol=0, atol=2e-3 * np.abs(fd).max(), err_msg=name)
+
+
+def pin_weight_grads_textbook_torch(orc):
+    """E=1, k=1, w=1: dW1 and dW2 of a dense SwiGLU FFN by torch float64 autograd."""
+    import torch
+    rng = _rng(15)
+    T, H, I = 7, 16, 12
+    x, W1, W2, _, _ = _rand_layer(rng, T, H, I, 1, 1)
+    dy = bf16(rng.standard_normal((T, H)))
+    idx = np.zeros((T, 1), np.int32)
+    w = np.ones((T, 1), np.float32)
+    dW1, dW2 = orc.expert_weight_grads(x, idx, w, W1[0], W2[0], 0, dy)
+    X = torch.from_numpy(f64(x))
+    A = torch.from_numpy(f64(W1[0])).requires_grad_(True)
+    B = torch.from_numpy(f64(W2[0])).requires_grad_(True)
+    Y = (torch.nn.functional.silu(X @ A[:, :I]) * (X @ A[:, I:])) @ B
+    (Y * torch.from_numpy(f64(dy))).sum().backward()
+    np.testing.assert_allclose(dW1, A.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dW2, B.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
 ALL_PINS = [
     pin_plan_worked, pin_plan_bruteforce, pin_plan_invariants, pin_plan_bad_index,
     pin_pool_gather, pin_ffn_worked, pin_ffn_dense_bruteforce, pin_ffn_textbook_torch,
     pin_ffn_closed_form, pin_ffn_linearity, pin_ffn_permutation, pin_identity_closed_form,
     pin_combine_gather, pin_route_bruteforce, pin_route_special_cases,
     pin_backward_finite_differences, pin_backward_textbook_torch, pin_backward_linear_in_dy,
+    pin_weight_grads_finite_differences, pin_weight_grads_textbook_torch,
 ]

@@ -51,9 +51,19 @@ MUTANTS = {
         "acc += bf16_to_double(w1[q]) * du[q] + bf16_to_double(w1[I + q]) * dg[q];"),
     "bwd_routing_weight_not_applied": ("dz[m] = w * dym;", "dz[m] = dym;"),
     "bwd_dw_weighted": ("s += dym * z[m];", "s += w * dym * z[m];"),
-    "bwd_w2_transposed": ("da += bf16_to_double(w2[m]) * dz[m];",
-                          "da += bf16_to_double(W2[e][(int64_t)m * I + q]) * dz[m];"),
-    "bwd_du_uses_gate_only": ("du[q] = da * silu(g[q]);", "du[q] = da * g[q];"),
+    "bwd_w2_transposed": ("          for (int32_t m = 0; m < H; ++m) da += bf16_to_double(w2[m]) * dz[m];",
+                          "          for (int32_t m = 0; m < H; ++m) da += bf16_to_double(W2[e][(int64_t)m * I + q]) * dz[m];"),
+    "bwd_du_uses_gate_only": ("          du[q] = da * silu(g[q]);", "          du[q] = da * g[q];"),
+    "wgrad_w2_transposed": ("\n      for (int32_t m = 0; m < H; ++m) da += bf16_to_double(w2[m]) * dz[m];",
+                            "\n      for (int32_t m = 0; m < H; ++m) da += bf16_to_double(W2e[(int64_t)m * I + q]) * dz[m];"),
+    "wgrad_du_uses_gate_only": ("\n      du[q] = da * silu(g[q]);", "\n      du[q] = da * g[q];"),
+    "wgrad_gate_up_swapped": ("row[q] += xh * dg[q];\n        row[I + q] += xh * du[q];",
+                              "row[q] += xh * du[q];\n        row[I + q] += xh * dg[q];"),
+    "wgrad_w2_no_routing_weight": (
+        "for (int32_t m = 0; m < H; ++m) dz[m] = w * bf16_to_double(dy[t * H + m]);",
+        "for (int32_t m = 0; m < H; ++m) dz[m] = bf16_to_double(dy[t * H + m]);"),
+    "wgrad_w2_uses_preactivation": ("for (int32_t m = 0; m < H; ++m) row[m] += a[q] * dz[m];",
+                                    "for (int32_t m = 0; m < H; ++m) row[m] += g[q] * dz[m];"),
 }
 
 
