@@ -375,33 +375,38 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
     dy = torch.from_numpy(si.make_dy(cfg).view(np.int16)).to(dev).view(torch.bfloat16)
     gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     gw = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    gW1 = torch.empty((cfg.E, H, 2 * I), dtype=torch.bfloat16, device=dev)
+    gW2 = torch.empty((cfg.E, I, H), dtype=torch.bfloat16, device=dev)
     plain = moe.moe_config(0, 0, 0, 0, 0, None)
     for _ in range(3):
-        buf.backward(dy, w, W1u, W2u, plain, dx=gx, dw=gw)
+        buf.backward(dy, w, W1u, W2u, plain, dx=gx, dw=gw, dW1=gW1, dW2=gW2)
     torch.cuda.synchronize()
-    tev = moe.moe_timing_events_create(7 * steps)
-    arrs = [(ctypes.c_void_p * 7)(*tev[7 * c: 7 * c + 7]) for c in range(steps)]
+    tev = moe.moe_timing_events_create(8 * steps)
+    arrs = [(ctypes.c_void_p * 8)(*tev[8 * c: 8 * c + 8]) for c in range(steps)]
     cfgs = [moe.moe_config(0, 0, 0, 0, 0, ctypes.cast(a, ctypes.c_void_p)) for a in arrs]
     barrier(world)
     torch.cuda.synchronize()
     for c in range(steps):
-        buf.backward(dy, w, W1u, W2u, cfgs[c], dx=gx, dw=gw)
+        buf.backward(dy, w, W1u, W2u, cfgs[c], dx=gx, dw=gw, dW1=gW1, dW2=gW2)
     torch.cuda.synchronize()
     code, aux = moe.moe_get_status(buf.plan)
     if code != 0:
         raise RuntimeError(f"device status after the backward: {moe.moe_strerror(code)} ({aux})")
-    names = ("combine_bwd", "recompute_gu", "gemm_y_bwd", "gemm_a_bwd", "dispatch_bwd")
+    names = ("combine_bwd", "recompute_gu", "gemm_y_bwd", "wgrad_w2", "gemm_a_bwd", "wgrad_w1",
+             "dispatch_bwd")
     ph = {k: 0.0 for k in names}
     for c in range(steps):
-        e = tev[7 * c: 7 * c + 7]
+        e = tev[8 * c: 8 * c + 8]
         for i, k in enumerate(names):
             ph[k] += el(e[i], e[i + 1]) / steps
-    total = el(tev[0], tev[7 * (steps - 1) + 5]) / steps
+    total = el(tev[0], tev[8 * (steps - 1) + 7]) / steps
     red = reduce_max([total, fwd_ms, fwd_gemm_a] + [ph[k] for k in names], dev, world)
     total, fwd_ms, fwd_gemm_a, ph = red[0], red[1], red[2], dict(zip(names, red[3:]))
     moe.moe_events_destroy(tev)
     flops_gemm = pairs * 6.0 * H * I            # backward Y 2HI + backward A 4HI (g, u kept)
     gemm_ms = ph["gemm_y_bwd"] + ph["gemm_a_bwd"]
+    wg_bytes = cfg.E * 3.0 * H * I * 2          # dW1 + dW2 written (bf16)
+    wg_ms = ph["wgrad_w1"] + ph["wgrad_w2"]
     a_tf = pairs * 4.0 * H * I / (ph["gemm_a_bwd"] / 1e3) / 1e12
     cb_bytes = T * H * 2 + 2 * pairs * H * 2 + T * cfg.k * 8
     db_bytes = pairs * H * 2 + T * H * 2
@@ -412,6 +417,9 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
                            "tokens_per_s": world * T / ((fwd_ms + total) / 1e3)},
             "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
             "grouped_gemms_useful_tflops": flops_gemm / (gemm_ms / 1e3) / 1e12,
+            "weight_grads": {"ms": wg_ms, "useful_tflops": flops_gemm / (wg_ms / 1e3) / 1e12,
+                             "written_gbs": wg_bytes / (wg_ms / 1e3) / 1e9,
+                             "note": "dW1 [E,H,2I] + dW2 [E,I,H] in bf16; the writes bound it"},
             "combine_bwd_gbs": cb_bytes / (ph["combine_bwd"] / 1e3) / 1e9,
             "dispatch_bwd_gbs": db_bytes / (ph["dispatch_bwd"] / 1e3) / 1e9,
             "roofline": {"kernel": "ffn_gemm_pair_kernel<1, K-major W1> (backward A)",
@@ -421,7 +429,7 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
                          "peak_source": f"{peak_src} bf16 sustained",
                          "algorithmic": "useful flops pairs*4*H*I per launch"},
             "weights": "as given (read K-major by the backward GEMMs)",
-            "calls": steps, "gpu_launches": 4 * steps,
+            "calls": steps, "gpu_launches": 9 * steps,
             "note": "after a forward that kept g | u (no recompute); every call computes the "
                     "same gradients"}
 

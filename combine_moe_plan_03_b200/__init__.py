@@ -82,7 +82,7 @@ def _load():
         "moe_forward": [P(moe_shape), vp, vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp,
                         P(moe_config), vp, vp, vp, vp],
         "moe_backward": [P(moe_shape), vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp, vp,
-                         vp, vp, P(moe_config), vp],
+                         vp, vp, vp, vp, vp, P(moe_config), vp],
         "moe_events_create": [P(vp), i32],
         "moe_timing_events_create": [P(vp), i32],
         "moe_event_elapsed_ms": [vp, vp, P(ctypes.c_float)],
@@ -237,15 +237,15 @@ def moe_forward(shape, x_ptr: int, topk_idx_ptr: int, topk_w_ptr: int, w1_ptr: i
 
 
 def moe_backward(shape, dy_ptr: int, topk_w_ptr: int, w1_ptr: int, w2_ptr: int,
-                 plan: moe_plan_buffers, pool_ptr: int, ypool_ptr: int, gu_ptr: int, dgu_ptr: int,
-                 dpool_ptr: int, dx_ptr: int, dw_ptr: int, cfg: moe_config | None,
-                 stream: int) -> None:
+                 plan: moe_plan_buffers, pool_ptr: int, act_ptr: int, ypool_ptr: int, gu_ptr: int,
+                 dgu_ptr: int, dpool_ptr: int, dx_ptr: int, dw_ptr: int, dw1_ptr: int,
+                 dw2_ptr: int, cfg: moe_config | None, stream: int) -> None:
     cfg = cfg or moe_config()
     _check("moe_backward", _lib.moe_backward(
         ctypes.byref(_shape(shape)), dy_ptr or None, topk_w_ptr or None, w1_ptr or None,
-        w2_ptr or None, ctypes.byref(plan), pool_ptr or None, ypool_ptr or None, gu_ptr or None,
-        dgu_ptr or None, dpool_ptr or None, dx_ptr or None, dw_ptr or None, ctypes.byref(cfg),
-        stream or None))
+        w2_ptr or None, ctypes.byref(plan), pool_ptr or None, act_ptr or None, ypool_ptr or None,
+        gu_ptr or None, dgu_ptr or None, dpool_ptr or None, dx_ptr or None, dw_ptr or None,
+        dw1_ptr or None, dw2_ptr or None, ctypes.byref(cfg), stream or None))
 
 
 def moe_events_create(n: int) -> list[int]:

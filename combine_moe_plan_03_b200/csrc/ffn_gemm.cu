@@ -545,8 +545,9 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
 // K-major, SwiGLU backward in the epilogue), backward A (W1 read K-major). dypool_dpool
 // holds dypool on entry and dpool on return.
 int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
-                        const moe_plan_buffers &p, const void *pool, void *dypool_dpool, void *gu,
-                        void *dgu, const moe_config &cfg, int num_sms, cudaStream_t st,
+                        const moe_plan_buffers &p, const void *pool, void *act,
+                        void *dypool_dpool, void *gu, void *dgu, void *dW1, void *dW2,
+                        const moe_config &cfg, int num_sms, cudaStream_t st,
                         cudaEvent_t const *tev) {
   const PlanGeom g = plan_geom(s);
   if (g.pmax == 0) return MOE_OK;
@@ -612,6 +613,16 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   if (launch_ffn_pair(2, true, tw2_k, tx_dy, y, clusters, st) != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
 
+  // dW2 = act^T . dypool per expert (before backward A overwrites dypool)
+  if (dW2 != nullptr) {
+    if (launch_zero_pad_rows(s, act, s.I, p, num_sms, st) != cudaSuccess ||
+        launch_zero_pad_rows(s, dypool_dpool, s.H, p, num_sms, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const int rc = launch_wgrad(s, act, s.I, dypool_dpool, s.H, dW2, p, p.meta + 6, cfg, num_sms, st);
+    if (rc != MOE_OK) return rc;
+  }
+  if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
+
   // backward A: dpool = dgu . W1^T (two 256-column blocks of dpool)
   FfnParams a = b;
   a.out = static_cast<uint16_t *>(dypool_dpool);
@@ -626,7 +637,15 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   a.sched = p.meta + 4;
   if (launch_ffn_pair(1, true, tw1_k, tx_dgu, a, clusters, st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // dW1 = pool^T . dgu per expert (the pool's padding rows are zero already)
+  if (dW1 != nullptr) {
+    if (launch_zero_pad_rows(s, dgu, 2 * s.I, p, num_sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+    const int rc = launch_wgrad(s, pool, s.H, dgu, 2 * s.I, dW1, p, p.meta + 4, cfg, num_sms, st);
+    if (rc != MOE_OK) return rc;
+  }
+  if (tev != nullptr && cudaEventRecord(tev[6], st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

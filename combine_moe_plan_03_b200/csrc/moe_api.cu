@@ -256,9 +256,9 @@ int moe_combine(const moe_shape *s, const void *ypool, const float *topk_w,
 }
 
 int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
-                 const void *W2, const moe_plan_buffers *p, const void *pool, const void *ypool,
-                 void *gu, void *dgu, void *dpool, void *dx, float *dw, const moe_config *cfg,
-                 void *stream) {
+                 const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
+                 const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
+                 void *dW1, void *dW2, const moe_config *cfg, void *stream) {
   int rc = check_shape(s, true);
   if (rc != MOE_OK) return rc;
   if ((rc = check_plan(p)) != MOE_OK) return rc;
@@ -267,8 +267,9 @@ int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const 
   if (s->T > 0 && (!dy || !topk_w || !dx || !dw)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(dy) || !aligned16(W1) || !aligned16(W2) || !aligned16(pool) ||
       !aligned16(ypool) || !aligned16(gu) || !aligned16(dgu) || !aligned16(dpool) ||
-      !aligned16(dx))
+      !aligned16(dx) || !aligned16(act) || !aligned16(dW1) || !aligned16(dW2))
     return MOE_ERR_MISALIGNED;
+  if (dW2 != nullptr && act == nullptr) return MOE_ERR_INVALID_ARG;
   moe_config c{};
   if (cfg != nullptr) c = *cfg;
   if ((rc = check_config(c)) != MOE_OK) return rc;
@@ -282,10 +283,11 @@ int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const 
   if (launch_combine_backward(*s, dy, ypool, topk_w, *p, dpool, dw, nsm, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[1], st) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((rc = launch_ffn_backward(*s, W1, W2, *p, pool, dpool, gu, dgu, c, nsm, st, tev)) != MOE_OK)
+  if ((rc = launch_ffn_backward(*s, W1, W2, *p, pool, act, dpool, gu, dgu, dW1, dW2, c, nsm, st,
+                                tev)) != MOE_OK)
     return rc;
   if (launch_combine(*s, dpool, nullptr, *p, dx, nsm, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[7], st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -1,0 +1,442 @@
+// Weight gradients of the grouped FFN (the backward's weight GEMMs): for every expert e,
+//   dW1[e] = pool_e^T . dgu_e      [H, 2I]      dgu = [dg | du] of the backward Y epilogue
+//   dW2[e] = act_e^T  . dypool_e   [I, H]
+// where X_e are the rows of expert e's pool segment. As one grouped GEMM:
+//   D[e] [M, N] = sum over the segment's rows p of A[p, 0:M]^T (x) B[p, 0:N]
+// with A, B row-major [P_max, M] / [P_max, N] activations and D [E, M, N] bf16.
+//
+// Design (tcgen05, SM pairs as in ffn_gemm_pair.cu): a work unit is (expert, 256 rows of D,
+// 256 columns of D); one cta_group::2 MMA has M = 256 (128 rows of D per CTA) and N = 256
+// (each CTA holds 128 of B's columns), K = 16; the K loop runs over the expert's rows in
+// steps of 64 (its live rows rounded up to 64: rows past the live ones must be zero, which
+// zero_pad_rows_kernel ensures for the operands that are not zero there already). Both
+// operands are read MN-major straight from the activations (for A the rows of D are
+// contiguous in memory, for B its columns), two TMA boxes of 64 columns x 64 rows each per
+// operand and CTA: 32 KB per stage, 6 stages. One accumulator of 256 TMEM columns per unit
+// in two buffers, so the epilogue of one unit overlaps the MMAs of the next. In the epilogue
+// each thread holds one row of D (its TMEM lane) and 32 consecutive columns per load and
+// stores them as 64 contiguous bytes: no turn through shared memory. An expert with no rows
+// gets a zero gradient. Waits are bounded as in the forward kernels; a wait that runs out
+// reports MOE_ERR_PIPE_TIMEOUT and raises both CTAs' abort flags.
+#include "ffn_gemm.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBK = 64;
+constexpr int kBoxBytes = 64 * kBK * 2;       // 8 KB: 64 columns x 64 rows
+constexpr int kOpBytes = 2 * kBoxBytes;       // 16 KB: 128 columns of one operand
+constexpr int kStageBytes = 2 * kOpBytes;     // A and B
+constexpr int kStages = 6;
+constexpr int kRingBytes = kStages * kStageBytes;  // 192 KB
+constexpr int kTmemCols = 512;
+constexpr int kBufCols = 256;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr int kSchedSlots = 4;
+constexpr int kSchedReaders = 1 + kEpiWarps + 1 + kEpiWarps;
+constexpr int kBarrierBytes = 256;
+constexpr int kSmemBytes = kRingBytes + kBarrierBytes + 1024;
+constexpr uint64_t kAbortGraceNs = 1000000;
+constexpr uint32_t kParkNs = 20000;
+
+struct WgradParams {
+  const int32_t *offsets;   // [E + 1] expert segment starts (rows)
+  const int32_t *counts;    // [E] live rows per expert
+  int32_t *status;
+  uint16_t *out;            // D [E, M, N]
+  int32_t E, M, N;
+  int32_t mb_count, nb_count;  // blocks of 256 rows / columns of D
+  int32_t *sched;           // {ticket, clusters done}
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ void raise_abort_w(volatile int *abort, uint32_t peer_abort,
+                                              int32_t *status, int32_t code, int32_t aux) {
+  if (!*abort) report(status, code, aux);
+  *abort = 1;
+  st_cluster_u32(peer_abort, 1u);
+}
+
+__device__ __forceinline__ int32_t k_steps(const WgradParams &prm, int32_t e) {
+  return (prm.counts[e] + kBK - 1) / kBK;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    wgrad_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                      const __grid_constant__ CUtensorMap tm_b, const WgradParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+  uint64_t *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages;    // [2]
+  uint64_t *acc_empty = acc_full + 2;      // [2]
+  uint64_t *drain = acc_empty + 2;
+  uint64_t *sched_full = drain + 1;
+  uint64_t *sched_empty = sched_full + kSchedSlots;
+  int32_t *sched = reinterpret_cast<int32_t *>(sched_empty + kSchedSlots);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched + kSchedSlots);
+  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+  int *never = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const bool lead = rank == 0;
+  const uint32_t peer_abort = cluster_map(smem_u32(abort_flag), peer);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, 2 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    for (int i = 0; i < kSchedSlots; ++i) {
+      mbar_init(sched_full + i, 1);
+      mbar_init(sched_empty + i, kSchedReaders);
+    }
+    *abort_flag = 0;
+    *never = 0;
+    fence_mbarrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  volatile int *abort = abort_flag;
+  const int32_t units_per_e = prm.mb_count * prm.nb_count;
+  const int32_t n_units = prm.E * units_per_e;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      uint32_t stage = 0, phase = 0, issued = 0, last_parity = 0;
+      uint32_t sslot = 0, sphase = 0;
+      for (;;) {
+        int32_t u;
+        if (lead) {
+          if (!mbar_wait<true>(sched_empty + sslot, sphase ^ 1u, 2 * prm.timeout_ns, abort)) {
+            raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+            break;
+          }
+          const int32_t ticket = atomicAdd(prm.sched + 0, 1);
+          u = (ticket < n_units && !*abort) ? ticket : -1;
+          sched[sslot] = u;
+          st_cluster_u32(cluster_map(smem_u32(sched + sslot), peer), (uint32_t)u);
+          mbar_arrive(sched_full + sslot);
+          mbar_arrive_cluster(cluster_map(smem_u32(sched_full + sslot), peer));
+        } else {
+          if (!mbar_wait<true>(sched_full + sslot, sphase, 2 * prm.timeout_ns, abort)) {
+            raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+            break;
+          }
+          u = sched[sslot];
+          mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
+        }
+        if (++sslot == kSchedSlots) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (u < 0) break;
+        const int32_t e = u / units_per_e;
+        const int32_t rest = u % units_per_e;
+        const int32_t mb = rest / prm.nb_count;
+        const int32_t nb = rest % prm.nb_count;
+        const int32_t kcount = k_steps(prm, e);
+        const int32_t row0 = prm.offsets[e];
+        const int32_t acol = mb * 256 + (int32_t)rank * 128;
+        const int32_t bcol = nb * 256 + (int32_t)rank * 128;
+        for (int32_t kb = 0; kb < kcount; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1u, 2 * prm.timeout_ns, abort)) {
+            raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+            break;
+          }
+          uint8_t *sa = smem + stage * kStageBytes;
+          uint8_t *sb = sa + kOpBytes;
+          const uint32_t fb = cluster_map(smem_u32(full + stage), 0);
+          if (lead) {
+            mbar_arrive_expect_tx(full + stage, 2u * kStageBytes);
+            issued |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          const int32_t r = row0 + kb * kBK;
+          tma_load_2d_pair(sa, &tm_a, fb, acol, r);
+          tma_load_2d_pair(sa + kBoxBytes, &tm_a, fb, acol + 64, r);
+          tma_load_2d_pair(sb, &tm_b, fb, bcol, r);
+          tma_load_2d_pair(sb + kBoxBytes, &tm_b, fb, bcol + 64, r);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort) {
+        if (lead)
+          for (int s = 0; s < kStages; ++s)
+            if (issued & (1u << s))
+              mbar_wait(full + s, (last_parity >> s) & 1u, prm.timeout_ns, never);
+      } else if (lead) {
+        __threadfence();
+        if (atomicAdd(prm.sched + 1, 1) == (int)(gridDim.x >> 1) - 1) {
+          atomicExch(prm.sched + 0, 0);
+          atomicExch(prm.sched + 1, 0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && lead) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t stage = 0, phase = 0, local = 0, sslot = 0, sphase = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_bf16_f32_ab(256, 256, /*a_mn=*/true, /*b_mn=*/true);
+      for (;; ++local) {
+        if (!mbar_wait(sched_full + sslot, sphase, 2 * prm.timeout_ns, abort)) {
+          raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+          break;
+        }
+        const int32_t u = sched[sslot];
+        mbar_arrive(sched_empty + sslot);
+        if (++sslot == kSchedSlots) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (u < 0) break;
+        const int32_t kcount = k_steps(prm, u / units_per_e);
+        const uint32_t buf = local & 1u, use = local >> 1;
+        if (!mbar_wait<true>(acc_empty + buf, (use + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
+          raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * kBufCols;
+        for (int32_t kb = 0; kb < kcount; ++kb) {
+          if (!mbar_wait(full + stage, phase, 2 * prm.timeout_ns, abort)) {
+            raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sb = sa + kOpBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            // both MN-major: 64-column chunks kBoxBytes apart, 8 rows per 1024 B, +2048 B
+            // per 16 rows of K
+            const uint64_t ad = smem_desc_sw128(sa + kk * 2048, kBoxBytes, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + kk * 2048, kBoxBytes, 1024);
+            tc_mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair_mc(empty + stage, 0x3);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(acc_full + buf, 0x3);
+      }
+      tc_commit_pair_mc(drain, 0x1);
+      mbar_wait(drain, 0, prm.timeout_ns, never);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    // warp w reads TMEM lanes 32 (w % 4) ... (rows of D) and columns 128 h ... 128 h + 127,
+    // h = (w - 2) / 4, of the unit's 256 columns
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
+    uint32_t local = 0, sslot = 0, sphase = 0;
+    for (;; ++local) {
+      int32_t u = -1;
+      int got = 1;
+      if (lane == 0) {
+        got = mbar_wait_parked<true>(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort,
+                                     kParkNs)
+                  ? 1
+                  : 0;
+        if (got) {
+          u = sched[sslot];
+          if (lead)
+            mbar_arrive(sched_empty + sslot);
+          else
+            mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (++sslot == kSchedSlots) {
+        sslot = 0;
+        sphase ^= 1u;
+      }
+      if (!got) {
+        if (lane == 0) raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+        break;
+      }
+      if (u < 0) break;
+      const int32_t e = u / units_per_e;
+      const int32_t rest = u % units_per_e;
+      const int32_t mb = rest / prm.nb_count;
+      const int32_t nb = rest % prm.nb_count;
+      const bool live = k_steps(prm, e) > 0;
+      const uint32_t buf = local & 1u, use = local >> 1;
+      int ok = 1;
+      if (lane == 0)
+        ok = mbar_wait_parked(acc_full + buf, use & 1u, 3 * prm.timeout_ns, abort, kParkNs) ? 1
+                                                                                          : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+        break;
+      }
+      tc_fence_after();
+      const int32_t m = mb * 256 + (int32_t)rank * 128 + quad * 32 + lane;  // row of D
+      uint16_t *orow = prm.out + ((size_t)e * prm.M + m) * prm.N;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int32_t col = half * 128 + q * 32;         // inside the unit's 256 columns
+        const int32_t ncol = nb * 256 + col;             // column of D
+        uint32_t a[32];
+        __syncwarp();
+        if (live) {
+          tmem_ld_32x32b_x32(tq + buf * kBufCols + col, a);
+          tmem_ld_wait();
+        }
+        if (m < prm.M && ncol < prm.N) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + ncol);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 o = make_uint4(0u, 0u, 0u, 0u);
+            if (live)
+              o = make_uint4(pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
+                             pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
+                             pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5])),
+                             pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7])));
+            dst[v] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (lead)
+          mbar_arrive(acc_empty + buf);
+        else
+          mbar_arrive_cluster(cluster_map(smem_u32(acc_empty + buf), 0));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  if (threadIdx.x == 0 && (*abort || ld_cluster_u32(peer_abort) != 0u)) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kAbortGraceNs) __nanosleep(1000);
+  }
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+// Rows [offsets[e] + counts[e], offsets[e] + roundup(counts[e], 64)) of a [P, width] bf16
+// buffer set to zero: the rows the weight-gradient GEMMs read past an expert's live rows.
+// One block per expert, 16-byte stores.
+__global__ void __launch_bounds__(256)
+    zero_pad_rows_kernel(uint16_t *__restrict__ buf, int32_t width, const int32_t *__restrict__ offsets,
+                         const int32_t *__restrict__ counts, int32_t E) {
+  for (int e = blockIdx.x; e < E; e += gridDim.x) {
+    const int32_t c = counts[e];
+    const int32_t r0 = offsets[e] + c;
+    const int32_t r1 = offsets[e] + ((c + kBK - 1) / kBK) * kBK;
+    const int32_t vpr = width / 8;
+    const int64_t n = (int64_t)(r1 - r0) * vpr;
+    uint4 *base = reinterpret_cast<uint4 *>(buf + (size_t)r0 * width);
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_zero_pad_rows(const moe_shape &s, void *buf, int32_t width,
+                                 const moe_plan_buffers &p, int num_sms, cudaStream_t st) {
+  const int grid = s.E < num_sms * 4 ? s.E : num_sms * 4;
+  zero_pad_rows_kernel<<<grid, 256, 0, st>>>(static_cast<uint16_t *>(buf), width, p.offsets,
+                                            p.counts, s.E);
+  return cudaGetLastError();
+}
+
+// D [E, M, N] = per expert A_e^T B_e over the expert's segment; A [P_max, M], B [P_max, N].
+int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, int32_t N,
+                 void *D, const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg,
+                 int num_sms, cudaStream_t st) {
+  const PlanGeom g = plan_geom(s);
+  CUtensorMap ta, tb;
+  const uint64_t rows = g.pmax > 0 ? (uint64_t)g.pmax : 1;
+  if (!make_tmap(&ta, A, (uint64_t)M, rows, kBK) || !make_tmap(&tb, B, (uint64_t)N, rows, kBK))
+    return MOE_ERR_CUDA;
+  static bool attr_set[64] = {false};
+  static int fit_cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.dynamicSmemBytes = kSmemBytes;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    lc.gridDim = dim3(2, 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, wgrad_pair_kernel, &lc) != cudaSuccess || n < 1)
+      return MOE_ERR_CUDA;
+    fit_cache[dev] = n;
+    attr_set[dev] = true;
+  }
+  int clusters = (cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms) / 2;
+  if (clusters < 1) clusters = 1;
+  if (clusters > fit_cache[dev]) clusters = fit_cache[dev];
+  WgradParams prm{};
+  prm.offsets = p.offsets;
+  prm.counts = p.counts;
+  prm.status = p.status;
+  prm.out = static_cast<uint16_t *>(D);
+  prm.E = s.E;
+  prm.M = M;
+  prm.N = N;
+  prm.mb_count = (M + 255) / 256;
+  prm.nb_count = (N + 255) / 256;
+  prm.sched = sched;
+  prm.timeout_ns = (uint64_t)(cfg.wait_timeout_us > 0 ? cfg.wait_timeout_us : 2000000) * 1000ull;
+  lc.gridDim = dim3(2 * clusters, 1, 1);
+  lc.stream = st;
+  if (cudaLaunchKernelEx(&lc, wgrad_pair_kernel, ta, tb, prm) != cudaSuccess) return MOE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

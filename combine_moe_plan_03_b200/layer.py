@@ -137,10 +137,13 @@ class MoELayerBuffers:
 
     def backward(self, dy: torch.Tensor, topk_w: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
                  cfg: moe_config | None = None, dx: torch.Tensor | None = None,
-                 dw: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
-        """Backward of the last ``forward`` call on these buffers (its plan, pool and ypool),
-        on the compute stream: returns (dx [T, H] bf16, dw [T, k] fp32) for the upstream
-        gradient dy [T, H] bf16 (moe_backward). W1 / W2 in their given layout."""
+                 dw: torch.Tensor | None = None, dW1: torch.Tensor | None = None,
+                 dW2: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+        """Backward of the last ``forward`` call on these buffers (its plan, pool, act and
+        ypool), on the compute stream: returns (dx [T, H] bf16, dw [T, k] fp32) for the
+        upstream gradient dy [T, H] bf16 (moe_backward), and fills the weight gradients
+        dW1 [E, H, 2I] / dW2 [E, I, H] (bf16) when they are given. W1 / W2 in their given
+        layout."""
         s = self.shape
         assert not self.identity
         assert dy.dtype == torch.bfloat16 and tuple(dy.shape) == (s.T, s.H) and dy.is_contiguous()
@@ -158,8 +161,11 @@ class MoELayerBuffers:
             dx = torch.empty((max(s.T, 1), s.H), dtype=bf, device=self.device)[: s.T]
         if dw is None:
             dw = torch.empty((max(s.T, 1), s.k), dtype=torch.float32, device=self.device)[: s.T]
+        for t, shp in ((dW1, (s.E, s.H, 2 * s.I)), (dW2, (s.E, s.I, s.H))):
+            assert t is None or (t.dtype == bf and tuple(t.shape) == shp and t.is_contiguous())
         moe_backward(s, dy.data_ptr(), topk_w.data_ptr(), W1.data_ptr(), W2.data_ptr(), self.plan,
-                     self.pool.data_ptr(), self.ypool.data_ptr(), self.gu.data_ptr(),
-                     self.dgu.data_ptr(), self.dpool.data_ptr(), dx.data_ptr(), dw.data_ptr(), cfg,
-                     self.compute.cuda_stream)
+                     self.pool.data_ptr(), self.act.data_ptr(), self.ypool.data_ptr(),
+                     self.gu.data_ptr(), self.dgu.data_ptr(), self.dpool.data_ptr(),
+                     dx.data_ptr(), dw.data_ptr(), dW1.data_ptr() if dW1 is not None else 0,
+                     dW2.data_ptr() if dW2 is not None else 0, cfg, self.compute.cuda_stream)
         return dx, dw

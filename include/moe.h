@@ -107,7 +107,8 @@ typedef struct moe_config {
   int32_t ffn_kernel;      /* grouped-GEMM kernel: MOE_FFN_ONE_SM (one CTA per work unit,
                               MMA M = 128) or MOE_FFN_SM_PAIR (a cluster of two CTAs on two
                               SMs per unit, cta_group::2 MMA with M = 256); 0 = default */
-  /* NULL, or 7 cudaEvent_t that moe_forward records at the phase boundaries, each on
+  /* NULL, or 7 cudaEvent_t (8 for moe_backward) that moe_forward records at the phase
+     boundaries, each on
      the stream of the kernels around it: [0] comm before plan, [1] comm after plan,
      [2] comm after dispatch, [3] compute before the FFN, [4] compute after GEMM A,
      [5] compute after GEMM Y, [6] compute after combine. moe_grouped_ffn records
@@ -243,17 +244,23 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
  *   dgu[p]   = bf16([da * u * silu'(g) | da * silu(g)]),  da = dypool[p] W2[e]^T (fp32)
  *   dpool[p] = bf16(dgu[p] W1[e]^T)                              (overwrites dypool)
  *   dx[t]    = bf16(sum_j dpool[pool_row[t,j]])                  (fp32 sum in j order)
+ * and, when dW2 / dW1 are not NULL, the weight gradients (fp32 sums, bf16 results; an expert
+ * with no rows gets zeros):
+ *   dW2[e] = sum over e's rows p of act[p]^T dypool[p]           [E, I, H]
+ *   dW1[e] = sum over e's rows p of pool[p]^T dgu[p]             [E, H, 2I]
+ * act is the forward call's act buffer (needed for dW2; its padding rows are set to zero).
  * Work buffers (device, caller-owned, 16-byte aligned): gu and dgu [P_max, 2I] bf16,
- * dpool [P_max, H] bf16. Outputs: dx [T, H] bf16, dw [T, k] fp32. The grouped GEMMs run on
- * SM pairs (cfg->ffn_kernel must be 0 or MOE_FFN_SM_PAIR; cfg->packed_weights and
- * cfg->streaming must be 0). cfg->timing_events, if set, receives on `stream`: [0] before,
- * [1] after the combine backward, [2] after the recompute, [3] after backward Y, [4] after
- * backward A, [5] after the dispatch backward.
+ * dpool [P_max, H] bf16. Outputs: dx [T, H] bf16, dw [T, k] fp32, dW1, dW2 bf16. The grouped
+ * GEMMs run on SM pairs (cfg->ffn_kernel must be 0 or MOE_FFN_SM_PAIR; cfg->packed_weights
+ * and cfg->streaming must be 0). cfg->timing_events, if set, holds 8 events recorded on
+ * `stream`: [0] before, [1] after the combine backward, [2] after the recompute, [3] after
+ * backward Y, [4] after dW2, [5] after backward A, [6] after dW1, [7] after the dispatch
+ * backward.
  */
 int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
-                 const void *W2, const moe_plan_buffers *p, const void *pool, const void *ypool,
-                 void *gu, void *dgu, void *dpool, void *dx, float *dw, const moe_config *cfg,
-                 void *stream);
+                 const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
+                 const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
+                 void *dW1, void *dW2, const moe_config *cfg, void *stream);
 
 /* Create / destroy n cudaEvent_t (timing disabled) for moe_forward's ordering. */
 int moe_events_create(void **events, int32_t n);

@@ -96,18 +96,25 @@ def test_backward_rejects_unsupported_configs_on_the_host():
     import combine_moe_plan_03_b200 as moe
     s = moe.moe_shape(16, 128, 128, 8, 2, 64)
     p = moe.moe_plan_bind(s, 1 << 20)
-    ptrs = [(1 << 21) + i * (1 << 16) for i in range(11)]
+    q = [(1 << 21) + i * (1 << 16) for i in range(14)]
+
+    def call(cfg, **over):
+        a = dict(dy=q[0], tw=q[1], w1=q[2], w2=q[3], pool=q[4], act=q[5], ypool=q[6], gu=q[7],
+                 dgu=q[8], dpool=q[9], dx=q[10], dw=q[11], dW1=q[12], dW2=q[13])
+        a.update(over)
+        moe.moe_backward(s, a["dy"], a["tw"], a["w1"], a["w2"], p, a["pool"], a["act"],
+                         a["ypool"], a["gu"], a["dgu"], a["dpool"], a["dx"], a["dw"], a["dW1"],
+                         a["dW2"], cfg, 0)
+
     for cfg in (moe.moe_config(0, 0, 0, 1, 0), moe.moe_config(1, 0, 0, 0, 0),
                 moe.moe_config(0, 0, 0, 0, moe.MOE_FFN_ONE_SM), moe.moe_config(0, 0, 0, 0, 9)):
         with pytest.raises(moe.MoEError) as ei:
-            moe.moe_backward(s, ptrs[0], ptrs[1], ptrs[2], ptrs[3], p, ptrs[4], ptrs[5],
-                             ptrs[6], ptrs[7], ptrs[8], ptrs[9], ptrs[10], cfg, 0)
+            call(cfg)
         assert ei.value.code == moe.MOE_ERR_INVALID_ARG
-    with pytest.raises(moe.MoEError) as ei:         # a missing work buffer
-        moe.moe_backward(s, ptrs[0], ptrs[1], ptrs[2], ptrs[3], p, ptrs[4], ptrs[5], 0,
-                         ptrs[7], ptrs[8], ptrs[9], ptrs[10], None, 0)
-    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
-    with pytest.raises(moe.MoEError) as ei:         # a misaligned dx
-        moe.moe_backward(s, ptrs[0], ptrs[1], ptrs[2], ptrs[3], p, ptrs[4], ptrs[5], ptrs[6],
-                         ptrs[7], ptrs[8], ptrs[9] + 4, ptrs[10], None, 0)
-    assert ei.value.code == moe.MOE_ERR_MISALIGNED
+    for over, code in (({"gu": 0}, moe.MOE_ERR_INVALID_ARG),          # a missing work buffer
+                       ({"act": 0}, moe.MOE_ERR_INVALID_ARG),         # dW2 needs act
+                       ({"dx": q[10] + 4}, moe.MOE_ERR_MISALIGNED),
+                       ({"dW1": q[12] + 8}, moe.MOE_ERR_MISALIGNED)):
+        with pytest.raises(moe.MoEError) as ei:
+            call(None, **over)
+        assert ei.value.code == code, over

@@ -20,16 +20,25 @@ def _close(got, ref, what):
     assert err <= TOL * scale, f"{what}: max err {err:.3e} vs {TOL} * {scale:.3e}"
 
 
-def _run(cfg, W1, W2, x, idx, w, dy):
+def _run(cfg, W1, W2, x, idx, w, dy, weight_grads=False):
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import bf16_dev, f32_dev, i32_dev
     buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
     dw_dev = f32_dev(w)
     buf.forward(bf16_dev(x), i32_dev(idx), dw_dev, W1, W2)
-    dx, dwg = buf.backward(bf16_dev(dy), dw_dev, W1, W2)
+    gW = None
+    if weight_grads:
+        gW = (torch.full((cfg.E, cfg.H, 2 * cfg.I), float("nan"), dtype=torch.bfloat16,
+                         device=W1.device),
+              torch.full((cfg.E, cfg.I, cfg.H), float("nan"), dtype=torch.bfloat16,
+                         device=W1.device))
+    dx, dwg = buf.backward(bf16_dev(dy), dw_dev, W1, W2, dW1=gW[0] if gW else None,
+                           dW2=gW[1] if gW else None)
     torch.cuda.synchronize()
     code, aux = moe.moe_get_status(buf.plan)
     assert code == 0, (moe.moe_strerror(code), aux)
+    if weight_grads:
+        return buf, dx, dwg, gW
     return buf, dx, dwg
 
 
@@ -173,4 +182,54 @@ def test_backward_no_live_pairs_and_no_tokens():
     dx, dw = buf.backward(e, ew, W1, W2)
     torch.cuda.synchronize()
     assert moe.moe_get_status(buf.plan)[0] == 0 and dx.numel() == 0 and dw.numel() == 0
+    buf.close()
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
+def test_weight_gradients_small_shapes_every_expert(shape):
+    """dW1 and dW2 of every expert against the oracle (expert 0 is left without rows, so its
+    gradients must be exactly zero); dx and dw of the same call too."""
+    from gpu_helpers import to_f64, weights_dev
+    name, T, H, I, E, k, tile = shape
+    cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=777 + T)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    if E > k:
+        idx[idx == 0] = -1                           # expert 0 gets no rows
+    dy = si.make_dy(cfg)
+    buf, dx, dw, (gW1, gW2) = _run(cfg, W1, W2, x, idx, w, dy, weight_grads=True)
+    W1l = [si.make_w1_expert(cfg, e) for e in range(E)]
+    W2l = [si.make_w2_expert(cfg, e) for e in range(E)]
+    for e in range(E):
+        r1, r2 = oracle.get().expert_weight_grads(x, idx, w, W1l[e], W2l[e], e, dy)
+        g1, g2 = to_f64(gW1[e]), to_f64(gW2[e])
+        if not (idx == e).any():
+            assert not np.any(g1) and not np.any(g2), f"{name} expert {e} without rows"
+            continue
+        _close(g1, r1, f"{name} dW1[{e}]")
+        _close(g2, r2, f"{name} dW2[{e}]")
+    rdx, rdw = oracle.get().moe_backward(x, idx, w, W1l, W2l, dy)
+    _close(to_f64(dx), rdx, f"{name} dx")
+    _close(dw.cpu().numpy().astype(np.float64), rdw, f"{name} dw")
+    buf.close()
+
+
+def test_weight_gradients_full_deepseek_two_experts():
+    """The DeepSeek-V3-shaped layer at full size: dW1 and dW2 of the two experts with the
+    fewest (non-zero) rows, element by element against the oracle."""
+    from gpu_helpers import to_f64
+    from test_gpu_full import _weights
+    cfg = si.CONFIGS["deepseek_v3"]
+    h1, h2, W1, W2 = _weights(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    dy = si.make_dy(cfg)
+    buf, dx, dw, (gW1, gW2) = _run(cfg, W1, W2, x, idx, w, dy, weight_grads=True)
+    cnt = np.bincount(idx[idx >= 0].reshape(-1), minlength=cfg.E)
+    order = [int(e) for e in np.argsort(cnt, kind="stable") if cnt[e] > 0][:2]
+    for e in order:
+        r1, r2 = oracle.get().expert_weight_grads(x, idx, w, h1[e], h2[e], e, dy)
+        _close(to_f64(gW1[e]), r1, f"deepseek dW1[{e}] ({cnt[e]} rows)")
+        _close(to_f64(gW2[e]), r2, f"deepseek dW2[{e}] ({cnt[e]} rows)")
     buf.close()
