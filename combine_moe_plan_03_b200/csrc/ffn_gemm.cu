@@ -400,18 +400,24 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-               uint32_t box_outer) {
+bool make_tmap_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+               uint32_t box_outer) {
+  return make_tmap_box(m, base, inner, outer, 64, box_outer, true);
 }
 
 template <int kMode>

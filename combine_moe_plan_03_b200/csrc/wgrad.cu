@@ -12,12 +12,14 @@
 // zero_pad_rows_kernel ensures for the operands that are not zero there already). Both
 // operands are read MN-major straight from the activations (for A the rows of D are
 // contiguous in memory, for B its columns), two TMA boxes of 64 columns x 64 rows each per
-// operand and CTA: 32 KB per stage, 6 stages. One accumulator of 256 TMEM columns per unit
+// operand and CTA: 32 KB per stage, 4 stages. One accumulator of 256 TMEM columns per unit
 // in two buffers, so the epilogue of one unit overlaps the MMAs of the next. In the epilogue
-// each thread holds one row of D (its TMEM lane) and 32 consecutive columns per load and
-// stores them as 64 contiguous bytes: no turn through shared memory. An expert with no rows
-// gets a zero gradient. Waits are bounded as in the forward kernels; a wait that runs out
-// reports MOE_ERR_PIPE_TIMEOUT and raises both CTAs' abort flags.
+// each thread holds one row of D (its TMEM lane) and 32 consecutive columns per load; a
+// warp's 32 x 128 share of a unit goes through shared memory (128-byte swizzled) to two
+// TMA stores, which write whole 128-byte row segments (the gradients are 3·E·H·I bf16
+// values per call and their writes bound the kernel). An expert with no rows gets a zero
+// gradient. Waits are bounded as in the forward kernels; a wait that runs out reports
+// MOE_ERR_PIPE_TIMEOUT and raises both CTAs' abort flags.
 #include "ffn_gemm.cuh"
 
 namespace moe {
@@ -28,8 +30,8 @@ constexpr int kBK = 64;
 constexpr int kBoxBytes = 64 * kBK * 2;       // 8 KB: 64 columns x 64 rows
 constexpr int kOpBytes = 2 * kBoxBytes;       // 16 KB: 128 columns of one operand
 constexpr int kStageBytes = 2 * kOpBytes;     // A and B
-constexpr int kStages = 6;
-constexpr int kRingBytes = kStages * kStageBytes;  // 192 KB
+constexpr int kStages = 4;
+constexpr int kRingBytes = kStages * kStageBytes;  // 128 KB
 constexpr int kTmemCols = 512;
 constexpr int kBufCols = 256;
 constexpr int kEpiWarps = 8;
@@ -37,7 +39,11 @@ constexpr int kThreads = 64 + kEpiWarps * 32;
 constexpr int kSchedSlots = 4;
 constexpr int kSchedReaders = 1 + kEpiWarps + 1 + kEpiWarps;
 constexpr int kBarrierBytes = 256;
-constexpr int kSmemBytes = kRingBytes + kBarrierBytes + 1024;
+constexpr int kStageOutBytes = 32 * 128 * 2;   // a warp's 32 rows x 128 columns of D
+constexpr int kOutBytes = kEpiWarps * kStageOutBytes;
+// shared memory: stage ring, then the epilogue's blocks (1024-byte aligned, as the 128-byte
+// swizzle of their TMA stores wants), then the barriers
+constexpr int kSmemBytes = kRingBytes + kOutBytes + kBarrierBytes + 1024;
 constexpr uint64_t kAbortGraceNs = 1000000;
 constexpr uint32_t kParkNs = 20000;
 
@@ -65,11 +71,12 @@ __device__ __forceinline__ int32_t k_steps(const WgradParams &prm, int32_t e) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
-                      const __grid_constant__ CUtensorMap tm_b, const WgradParams prm) {
+                      const __grid_constant__ CUtensorMap tm_b,
+                      const __grid_constant__ CUtensorMap tm_d, const WgradParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRingBytes + kOutBytes);
   uint64_t *empty = full + kStages;
   uint64_t *acc_full = empty + kStages;    // [2]
   uint64_t *acc_empty = acc_full + 2;      // [2]
@@ -111,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
   }
+  if (warp == 2 && lane == 0) tma_prefetch_desc(&tm_d);
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
     tmem_relinquish_pair();
@@ -256,11 +264,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    // warp w reads TMEM lanes 32 (w % 4) ... (rows of D) and columns 128 h ... 128 h + 127,
-    // h = (w - 2) / 4, of the unit's 256 columns
+    // warp w reads TMEM lanes 32 (w % 4) ... (32 rows of D) and columns 128 h ... 128 h + 127,
+    // h = (w - 2) / 4, of the unit's 256 columns, 32 at a time: each thread puts its row's
+    // 128 columns into the warp's two 32 x 64 blocks in shared memory, in the 128-byte
+    // swizzled order (16-byte chunk c of row r at c ^ (r % 8), so a warp's stores hit every
+    // bank once), and one thread writes the blocks to D with two TMA stores.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
+    uint8_t *stg = smem + kRingBytes + (warp - 2) * kStageOutBytes;
     uint32_t local = 0, sslot = 0, sphase = 0;
     for (;; ++local) {
       int32_t u = -1;
@@ -305,30 +317,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int32_t m = mb * 256 + (int32_t)rank * 128 + quad * 32 + lane;  // row of D
-      uint16_t *orow = prm.out + ((size_t)e * prm.M + m) * prm.N;
+      const int32_t m0 = mb * 256 + (int32_t)rank * 128 + quad * 32;  // first row of D here
+      const int32_t ncol0 = nb * 256 + half * 128;                     // first column of D here
+      const bool store = m0 < prm.M && ncol0 < prm.N;                  // uniform across the warp
+      // the previous unit's store has read the block
+      if (lane == 0) bulk_wait_group_read<0>();
+      __syncwarp();
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int32_t col = half * 128 + q * 32;         // inside the unit's 256 columns
-        const int32_t ncol = nb * 256 + col;             // column of D
         uint32_t a[32];
         __syncwarp();
         if (live) {
-          tmem_ld_32x32b_x32(tq + buf * kBufCols + col, a);
+          tmem_ld_32x32b_x32(tq + buf * kBufCols + half * 128 + q * 32, a);
           tmem_ld_wait();
         }
-        if (m < prm.M && ncol < prm.N) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + ncol);
+        // block q / 2, 16-byte chunks 4 (q % 2) ... 4 (q % 2) + 3 of this thread's row
+        uint4 *row = reinterpret_cast<uint4 *>(stg + (q >> 1) * (kStageOutBytes / 2) + lane * 128);
+        if (store) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 o = make_uint4(0u, 0u, 0u, 0u);
-            if (live)
-              o = make_uint4(pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
-                             pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
-                             pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5])),
-                             pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7])));
-            dst[v] = o;
-          }
+          for (int v = 0; v < 4; ++v)
+            row[(4 * (q & 1) + v) ^ (lane & 7)] =
+                live ? make_uint4(
+                           pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
+                           pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
+                           pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5])),
+                           pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7])))
+                     : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      if (store) {
+        fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
+        __syncwarp();
+        // a ragged last block (N a multiple of 64, not of 128) has no second half
+        if (lane == 0) {
+          tma_store_2d(&tm_d, stg, ncol0, e * prm.M + m0);
+          if (ncol0 + 64 < prm.N)
+            tma_store_2d(&tm_d, stg + kStageOutBytes / 2, ncol0 + 64, e * prm.M + m0);
+          bulk_commit_group();
         }
       }
       tc_fence_before();
@@ -340,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_cluster(cluster_map(smem_u32(acc_empty + buf), 0));
       }
     }
+    if (lane == 0) bulk_wait_group_all();   // every block written before the CTA exits
   }
 
   tc_fence_before();
@@ -388,9 +414,10 @@ int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, in
                  void *D, const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg,
                  int num_sms, cudaStream_t st) {
   const PlanGeom g = plan_geom(s);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, td;
   const uint64_t rows = g.pmax > 0 ? (uint64_t)g.pmax : 1;
-  if (!make_tmap(&ta, A, (uint64_t)M, rows, kBK) || !make_tmap(&tb, B, (uint64_t)N, rows, kBK))
+  if (!make_tmap(&ta, A, (uint64_t)M, rows, kBK) || !make_tmap(&tb, B, (uint64_t)N, rows, kBK) ||
+      !make_tmap_box(&td, D, (uint64_t)N, (uint64_t)s.E * M, 64, 32, true))
     return MOE_ERR_CUDA;
   static bool attr_set[64] = {false};
   static int fit_cache[64] = {0};
@@ -435,7 +462,8 @@ int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, in
   prm.timeout_ns = (uint64_t)(cfg.wait_timeout_us > 0 ? cfg.wait_timeout_us : 2000000) * 1000ull;
   lc.gridDim = dim3(2 * clusters, 1, 1);
   lc.stream = st;
-  if (cudaLaunchKernelEx(&lc, wgrad_pair_kernel, ta, tb, prm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaLaunchKernelEx(&lc, wgrad_pair_kernel, ta, tb, td, prm) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
