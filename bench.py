@@ -408,6 +408,26 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
     wg_bytes = cfg.E * 3.0 * H * I * 2          # dW1 + dW2 written (bf16)
     wg_ms = ph["wgrad_w1"] + ph["wgrad_w2"]
     a_tf = pairs * 4.0 * H * I / (ph["gemm_a_bwd"] / 1e3) / 1e12
+    # backward A reads W1 K-major: 2*rows flops per weight element, as GEMM A; with fewer
+    # live rows per expert than the ridge it streams W1 from HBM
+    n_live = float(len(np.unique(idx.cpu().numpy()[idx.cpu().numpy() >= 0])))
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if pairs / max(n_live, 1.0) >= ridge:
+        bwd_roofline = {"kernel": "ffn_gemm_pair_kernel<1, K-major W1> (backward A)",
+                        "bound": "tensor", "achieved": a_tf,
+                        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                        "frac": a_tf / peaks["bf16_tflops_sustained"],
+                        "peak_source": f"{peak_src} bf16 sustained",
+                        "algorithmic": "useful flops pairs*4*H*I per launch"}
+    else:
+        a_gbs = ((n_live * H * 2 * I * 2 + pairs * (2 * I + H) * 2)
+                 / (ph["gemm_a_bwd"] / 1e3) / 1e9)
+        bwd_roofline = {"kernel": "ffn_gemm_pair_kernel<1, K-major W1> (backward A)",
+                        "bound": "hbm", "achieved": a_gbs, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": a_gbs / peaks["hbm_gbs"],
+                        "peak_source": f"{peak_src} HBM copy",
+                        "algorithmic": "bytes per launch: W1 of the live experts + live rows "
+                                       "of d(g, u) read + of d(pool) written"}
     cb_bytes = T * H * 2 + 2 * pairs * H * 2 + T * cfg.k * 8
     db_bytes = pairs * H * 2 + T * H * 2
     return {"ms_per_call": total, "tokens_per_s": world * T / (total / 1e3),
@@ -422,12 +442,7 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
                              "note": "dW1 [E,H,2I] + dW2 [E,I,H] in bf16; the writes bound it"},
             "combine_bwd_gbs": cb_bytes / (ph["combine_bwd"] / 1e3) / 1e9,
             "dispatch_bwd_gbs": db_bytes / (ph["dispatch_bwd"] / 1e3) / 1e9,
-            "roofline": {"kernel": "ffn_gemm_pair_kernel<1, K-major W1> (backward A)",
-                         "bound": "tensor", "achieved": a_tf,
-                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": a_tf / peaks["bf16_tflops_sustained"],
-                         "peak_source": f"{peak_src} bf16 sustained",
-                         "algorithmic": "useful flops pairs*4*H*I per launch"},
+            "roofline": bwd_roofline,
             "weights": "as given (read K-major by the backward GEMMs)",
             "calls": steps, "gpu_launches": 9 * steps,
             "note": "after a forward that kept g | u (no recompute); every call computes the "
