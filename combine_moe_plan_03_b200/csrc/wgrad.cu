@@ -12,11 +12,12 @@
 // zero_pad_rows_kernel ensures for the operands that are not zero there already). Both
 // operands are read MN-major straight from the activations (for A the rows of D are
 // contiguous in memory, for B its columns), two TMA boxes of 64 columns x 64 rows each per
-// operand and CTA: 32 KB per stage, 4 stages. One accumulator of 256 TMEM columns per unit
+// operand and CTA: 32 KB per stage, 5 stages. One accumulator of 256 TMEM columns per unit
 // in two buffers, so the epilogue of one unit overlaps the MMAs of the next. In the epilogue
 // each thread holds one row of D (its TMEM lane) and 32 consecutive columns per load; a
-// warp's 32 x 128 share of a unit goes through shared memory (128-byte swizzled) to two
-// TMA stores, which write whole 128-byte row segments (the gradients are 3·E·H·I bf16
+// warp's 32 x 64 share of a unit goes through shared memory (128-byte swizzled) to one TMA
+// store, which writes whole 128-byte row segments; 16 epilogue warps keep the epilogue of a
+// unit shorter than its MMAs even for the experts with few rows (the gradients are 3·E·H·I bf16
 // values per call and their writes bound the kernel). An expert with no rows gets a zero
 // gradient. Waits are bounded as in the forward kernels; a wait that runs out reports
 // MOE_ERR_PIPE_TIMEOUT and raises both CTAs' abort flags.
@@ -30,16 +31,16 @@ constexpr int kBK = 64;
 constexpr int kBoxBytes = 64 * kBK * 2;       // 8 KB: 64 columns x 64 rows
 constexpr int kOpBytes = 2 * kBoxBytes;       // 16 KB: 128 columns of one operand
 constexpr int kStageBytes = 2 * kOpBytes;     // A and B
-constexpr int kStages = 4;
-constexpr int kRingBytes = kStages * kStageBytes;  // 128 KB
+constexpr int kStages = 5;
+constexpr int kRingBytes = kStages * kStageBytes;  // 160 KB
 constexpr int kTmemCols = 512;
 constexpr int kBufCols = 256;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;                  // 4 per TMEM lane quadrant, 64 columns each
 constexpr int kThreads = 64 + kEpiWarps * 32;
 constexpr int kSchedSlots = 4;
 constexpr int kSchedReaders = 1 + kEpiWarps + 1 + kEpiWarps;
 constexpr int kBarrierBytes = 256;
-constexpr int kStageOutBytes = 32 * 128 * 2;   // a warp's 32 rows x 128 columns of D
+constexpr int kStageOutBytes = 32 * 64 * 2;    // a warp's 32 rows x 64 columns of D
 constexpr int kOutBytes = kEpiWarps * kStageOutBytes;
 // shared memory: stage ring, then the epilogue's blocks (1024-byte aligned, as the 128-byte
 // swizzle of their TMA stores wants), then the barriers
@@ -136,6 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ TMA producer
       uint32_t stage = 0, phase = 0, issued = 0, last_parity = 0;
       uint32_t sslot = 0, sphase = 0;
+      // the first CTA asks for the next ticket one unit ahead, so the atomic's round trip
+      // overlaps the loads of the current unit (the units are short: a few k-steps)
+      int32_t next_ticket = lead ? atomicAdd(prm.sched + 0, 1) : 0;
       for (;;) {
         int32_t u;
         if (lead) {
@@ -143,7 +147,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
             break;
           }
-          const int32_t ticket = atomicAdd(prm.sched + 0, 1);
+          const int32_t ticket = next_ticket;
+          if (ticket < n_units) next_ticket = atomicAdd(prm.sched + 0, 1);
           u = (ticket < n_units && !*abort) ? ticket : -1;
           sched[sslot] = u;
           st_cluster_u32(cluster_map(smem_u32(sched + sslot), peer), (uint32_t)u);
@@ -264,13 +269,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    // warp w reads TMEM lanes 32 (w % 4) ... (32 rows of D) and columns 128 h ... 128 h + 127,
+    // warp w reads TMEM lanes 32 (w % 4) ... (32 rows of D) and columns 64 h ... 64 h + 63,
     // h = (w - 2) / 4, of the unit's 256 columns, 32 at a time: each thread puts its row's
-    // 128 columns into the warp's two 32 x 64 blocks in shared memory, in the 128-byte
-    // swizzled order (16-byte chunk c of row r at c ^ (r % 8), so a warp's stores hit every
-    // bank once), and one thread writes the blocks to D with two TMA stores.
+    // 64 columns into the warp's 32 x 64 block in shared memory, in the 128-byte swizzled
+    // order (16-byte chunk c of row r at c ^ (r % 8), so a warp's stores hit every bank
+    // once), and one thread writes the block to D with a TMA store.
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;
     const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
     uint8_t *stg = smem + kRingBytes + (warp - 2) * kStageOutBytes;
     uint32_t local = 0, sslot = 0, sphase = 0;
@@ -318,25 +323,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int32_t m0 = mb * 256 + (int32_t)rank * 128 + quad * 32;  // first row of D here
-      const int32_t ncol0 = nb * 256 + half * 128;                     // first column of D here
+      const int32_t ncol0 = nb * 256 + part * 64;                      // first column of D here
       const bool store = m0 < prm.M && ncol0 < prm.N;                  // uniform across the warp
       // the previous unit's store has read the block
       if (lane == 0) bulk_wait_group_read<0>();
       __syncwarp();
+      uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 128);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         uint32_t a[32];
         __syncwarp();
         if (live) {
-          tmem_ld_32x32b_x32(tq + buf * kBufCols + half * 128 + q * 32, a);
+          tmem_ld_32x32b_x32(tq + buf * kBufCols + part * 64 + q * 32, a);
           tmem_ld_wait();
         }
-        // block q / 2, 16-byte chunks 4 (q % 2) ... 4 (q % 2) + 3 of this thread's row
-        uint4 *row = reinterpret_cast<uint4 *>(stg + (q >> 1) * (kStageOutBytes / 2) + lane * 128);
         if (store) {
 #pragma unroll
           for (int v = 0; v < 4; ++v)
-            row[(4 * (q & 1) + v) ^ (lane & 7)] =
+            row[(4 * q + v) ^ (lane & 7)] =
                 live ? make_uint4(
                            pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
                            pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
@@ -348,11 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (store) {
         fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
         __syncwarp();
-        // a ragged last block (N a multiple of 64, not of 128) has no second half
         if (lane == 0) {
           tma_store_2d(&tm_d, stg, ncol0, e * prm.M + m0);
-          if (ncol0 + 64 < prm.N)
-            tma_store_2d(&tm_d, stg + kStageOutBytes / 2, ncol0 + 64, e * prm.M + m0);
           bulk_commit_group();
         }
       }
