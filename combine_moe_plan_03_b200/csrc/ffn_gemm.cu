@@ -1,6 +1,9 @@
 // Grouped SwiGLU FFN over the expert-major pool (StreamEP README, How it works,
 // "CuTeDSL compute kernels": the forward grouped GEMMs A and Y), written for
-// sm_100a tensor cores:
+// sm_100a tensor cores. This file holds the one-CTA-per-unit kernel (MOE_FFN_ONE_SM),
+// the host side of both grouped-GEMM kernels (tensor maps, unit geometry, launches of
+// the forward and of the backward's GEMMs) and the TMA tensor-map helpers; the SM-pair
+// kernel, the default, is in ffn_gemm_pair.cu.
 //   GEMM A: act[p, n]   = bf16( silu(pool[p] . W1[e][:, n]) * (pool[p] . W1[e][:, I + n]) )
 //   GEMM Y: ypool[p, m] = bf16( act[p] . W2[e][:, m] )
 // for the live rows p of expert e (pool rows past an expert's count are padding and

@@ -17,8 +17,13 @@
  *                                                   moe_plan's optional host_P
  *   - "CuTeDSL compute kernels": the forward grouped GEMMs A (gate/up) and
  *     Y (down)                                   -> moe_grouped_ffn
+ *     and the backward grouped GEMMs A and Y, with the backward pass mirroring
+ *     dispatch and combine                        -> moe_backward (plus the weight
+ *                                                   gradients)
  * and the StreamEP call stream_moe_func(buffer, x, topk_idx, topk_weights, ...,
  * w1_local, w2_local, streams=...) shown there            -> moe_forward.
+ * The router's softmax / top-k, which StreamEP takes as inputs, is here too
+ *                                                -> moe_route, moe_route_plan.
  *
  * Conventions (all entry points):
  *   - Every pointer argument named as a tensor is a DEVICE pointer owned by the
