@@ -348,6 +348,14 @@ def config_block(cfg, world):
 
 # ------------------------------------------------------------------ the CUDA path
 
+def streams_weights(pairs: float, n_live_experts: float, peaks: dict) -> bool:
+    """True when a grouped GEMM over these routed pairs is bound by streaming its weights
+    from HBM rather than by the tensor pipe: it does 2 * rows flops per weight element
+    (2 bytes), so the ridge is the sustained bf16 rate over the HBM copy rate."""
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    return pairs / max(n_live_experts, 1.0) < ridge
+
+
 def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed, ffn_kernel,
                   pairs, peaks, peak_src, steps):
     """A training step of the layer on micro-batch 0: the forward that also keeps the gate /
@@ -410,9 +418,9 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
     a_tf = pairs * 4.0 * H * I / (ph["gemm_a_bwd"] / 1e3) / 1e12
     # backward A reads W1 K-major: 2*rows flops per weight element, as GEMM A; with fewer
     # live rows per expert than the ridge it streams W1 from HBM
-    n_live = float(len(np.unique(idx.cpu().numpy()[idx.cpu().numpy() >= 0])))
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if pairs / max(n_live, 1.0) >= ridge:
+    idx_h = idx.cpu().numpy()
+    n_live = float(len(np.unique(idx_h[idx_h >= 0])))
+    if not streams_weights(pairs, n_live, peaks):
         bwd_roofline = {"kernel": "ffn_gemm_pair_kernel<1, K-major W1> (backward A)",
                         "bound": "tensor", "achieved": a_tf,
                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
@@ -607,7 +615,7 @@ def run_moe(args):
         # expert than the ridge (sustained flop/s over HBM B/s) it streams weights from HBM.
         ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
         rows_per_expert = pairs_m / max(n_live_experts, 1.0)
-        if rows_per_expert >= ridge:
+        if not streams_weights(pairs_m, n_live_experts, peaks):
             line["roofline"] = {"kernel": f"{kname} (GEMM A + SwiGLU)", "bound": "tensor",
                                 "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                                 "unit": "TFLOP/s",

@@ -76,3 +76,16 @@ def test_reference_arm_line_on_rank_zero(monkeypatch):
     line = json.loads(buf.getvalue())
     assert rc == 0 and line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_roofline_bound_choice():
+    """The bench compares a grouped GEMM with the tensor peak when each weight is used by
+    more rows than the flop/byte ridge, else with HBM (weight streaming): the DeepSeek-V3
+    and Qwen3 shapes (256 rows per expert) are tensor-bound, the decode micro-batches (about
+    6 rows per live expert) stream weights."""
+    import bench
+    peaks = {"hbm_gbs": 6508.8, "bf16_tflops": 1624.0, "bf16_tflops_sustained": 1372.3}
+    assert not bench.streams_weights(65536, 256, peaks)       # DeepSeek-V3-shaped layer
+    assert not bench.streams_weights(32768, 128, peaks)       # Qwen3-shaped layer
+    assert bench.streams_weights(1024, 170, peaks)            # a decode micro-batch
+    assert bench.streams_weights(0, 0, peaks)                 # nothing routed
