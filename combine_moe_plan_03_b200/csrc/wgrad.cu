@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *sched_full = drain + 1;
   uint64_t *sched_empty = sched_full + kSchedSlots;
   int32_t *sched = reinterpret_cast<int32_t *>(sched_empty + kSchedSlots);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched + kSchedSlots);
+  int32_t *sched_k = sched + kSchedSlots;   // the unit's k-steps, published with its id
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched_k + kSchedSlots);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   int *never = abort_flag + 1;
 
@@ -150,8 +151,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int32_t ticket = next_ticket;
           if (ticket < n_units) next_ticket = atomicAdd(prm.sched + 0, 1);
           u = (ticket < n_units && !*abort) ? ticket : -1;
+          const int32_t kc = u >= 0 ? k_steps(prm, u / units_per_e) : 0;
           sched[sslot] = u;
+          sched_k[sslot] = kc;
           st_cluster_u32(cluster_map(smem_u32(sched + sslot), peer), (uint32_t)u);
+          st_cluster_u32(cluster_map(smem_u32(sched_k + sslot), peer), (uint32_t)kc);
           mbar_arrive(sched_full + sslot);
           mbar_arrive_cluster(cluster_map(smem_u32(sched_full + sslot), peer));
         } else {
@@ -162,6 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           u = sched[sslot];
           mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
         }
+        const int32_t kcount = sched_k[sslot];
         if (++sslot == kSchedSlots) {
           sslot = 0;
           sphase ^= 1u;
@@ -171,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t rest = u % units_per_e;
         const int32_t mb = rest / prm.nb_count;
         const int32_t nb = rest % prm.nb_count;
-        const int32_t kcount = k_steps(prm, e);
         const int32_t row0 = prm.offsets[e];
         const int32_t acol = mb * 256 + (int32_t)rank * 128;
         const int32_t bcol = nb * 256 + (int32_t)rank * 128;
@@ -224,13 +228,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const int32_t u = sched[sslot];
+        const int32_t kcount = sched_k[sslot];
         mbar_arrive(sched_empty + sslot);
         if (++sslot == kSchedSlots) {
           sslot = 0;
           sphase ^= 1u;
         }
         if (u < 0) break;
-        const int32_t kcount = k_steps(prm, u / units_per_e);
         const uint32_t buf = local & 1u, use = local >> 1;
         if (!mbar_wait<true>(acc_empty + buf, (use + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
           raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *stg = smem + kRingBytes + (warp - 2) * kStageOutBytes;
     uint32_t local = 0, sslot = 0, sphase = 0;
     for (;; ++local) {
-      int32_t u = -1;
+      int32_t u = -1, kc = 0;
       int got = 1;
       if (lane == 0) {
         got = mbar_wait_parked<true>(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort,
@@ -289,6 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   : 0;
         if (got) {
           u = sched[sslot];
+          kc = sched_k[sslot];
           if (lead)
             mbar_arrive(sched_empty + sslot);
           else
@@ -297,6 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       got = __shfl_sync(0xffffffffu, got, 0);
       u = __shfl_sync(0xffffffffu, u, 0);
+      kc = __shfl_sync(0xffffffffu, kc, 0);
       if (++sslot == kSchedSlots) {
         sslot = 0;
         sphase ^= 1u;
@@ -310,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t rest = u % units_per_e;
       const int32_t mb = rest / prm.nb_count;
       const int32_t nb = rest % prm.nb_count;
-      const bool live = k_steps(prm, e) > 0;
+      const bool live = kc > 0;
       const uint32_t buf = local & 1u, use = local >> 1;
       int ok = 1;
       if (lane == 0)
@@ -325,10 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t m0 = mb * 256 + (int32_t)rank * 128 + quad * 32;  // first row of D here
       const int32_t ncol0 = nb * 256 + part * 64;                      // first column of D here
       const bool store = m0 < prm.M && ncol0 < prm.N;                  // uniform across the warp
-      // the previous unit's store has read the block
-      if (lane == 0) bulk_wait_group_read<0>();
-      __syncwarp();
-      uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 128);
+      // the warp's 64 columns into registers as bf16 pairs, then the TMEM buffer goes back
+      // to the MMA thread before the (possibly waiting) staging and store
+      uint32_t pk[32];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         uint32_t a[32];
@@ -337,25 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32x32b_x32(tq + buf * kBufCols + part * 64 + q * 32, a);
           tmem_ld_wait();
         }
-        if (store) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            row[(4 * q + v) ^ (lane & 7)] =
-                live ? make_uint4(
-                           pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
-                           pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
-                           pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5])),
-                           pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7])))
-                     : make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      if (store) {
-        fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_d, stg, ncol0, e * prm.M + m0);
-          bulk_commit_group();
-        }
+        for (int i = 0; i < 16; ++i)
+          pk[16 * q + i] =
+              live ? pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])) : 0u;
       }
       tc_fence_before();
       __syncwarp();
@@ -364,6 +354,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(acc_empty + buf);
         else
           mbar_arrive_cluster(cluster_map(smem_u32(acc_empty + buf), 0));
+      }
+      if (store) {
+        // the previous unit's store has read the block
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          row[c ^ (lane & 7)] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_d, stg, ncol0, e * prm.M + m0);
+          bulk_commit_group();
+        }
       }
     }
     if (lane == 0) bulk_wait_group_all();   // every block written before the CTA exits
