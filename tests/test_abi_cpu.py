@@ -118,3 +118,17 @@ def test_backward_rejects_unsupported_configs_on_the_host():
         with pytest.raises(moe.MoEError) as ei:
             call(None, **over)
         assert ei.value.code == code, over
+
+
+def test_gate_up_needs_the_pair_kernel_and_alignment():
+    """moe_config.gate_up (the training step's saved gate / up values) is refused with the
+    one-CTA kernel and when misaligned, on the host."""
+    import combine_moe_plan_03_b200 as moe
+    s = moe.moe_shape(16, 128, 128, 8, 2, 64)
+    p = moe.moe_plan_bind(s, 1 << 20)
+    for cfg, code in ((moe.moe_config(0, 0, 0, 0, moe.MOE_FFN_ONE_SM, None, 1 << 24),
+                       moe.MOE_ERR_INVALID_ARG),
+                      (moe.moe_config(0, 0, 0, 0, 0, None, (1 << 24) + 8), moe.MOE_ERR_MISALIGNED)):
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_grouped_ffn(s, 1 << 20, 1 << 21, 1 << 21, p, 1 << 22, 1 << 23, cfg)
+        assert ei.value.code == code

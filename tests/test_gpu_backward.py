@@ -233,3 +233,38 @@ def test_weight_gradients_full_deepseek_two_experts():
         _close(to_f64(gW1[e]), r1, f"deepseek dW1[{e}] ({cnt[e]} rows)")
         _close(to_f64(gW2[e]), r2, f"deepseek dW2[{e}] ({cnt[e]} rows)")
     buf.close()
+
+
+def test_packed_forward_saving_gate_up_then_backward():
+    """The training step as the benchmark runs it: the forward with prepacked weights keeping
+    g | u, the backward reading the weights in their given layout; output, saved g / u and
+    gradients against the oracle."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import assert_layer_close, bf16_dev, f32_dev, i32_dev, to_f64, weights_dev
+    cfg = si.custom("packed-train", T=300, H=256, I=384, E=4, k=2, tile=128, seed=31337)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    idx, w = si.make_routing(cfg)
+    dy = si.make_dy(cfg)
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    W1p, W2p = buf.pack_weights(W1, W2)
+    wd = f32_dev(w)
+    out = buf.forward(bf16_dev(x), i32_dev(idx), wd, W1p, W2p, moe.moe_config(packed_weights=1),
+                      save_for_backward=True)
+    gW1 = torch.empty((cfg.E, cfg.H, 2 * cfg.I), dtype=torch.bfloat16, device=W1.device)
+    gW2 = torch.empty((cfg.E, cfg.I, cfg.H), dtype=torch.bfloat16, device=W1.device)
+    dx, dw = buf.backward(bf16_dev(dy), wd, W1, W2, dW1=gW1, dW2=gW2)
+    torch.cuda.synchronize()
+    code, aux = moe.moe_get_status(buf.plan)
+    assert code == 0, (moe.moe_strerror(code), aux)
+    W1l = [si.make_w1_expert(cfg, e) for e in range(cfg.E)]
+    W2l = [si.make_w2_expert(cfg, e) for e in range(cfg.E)]
+    assert_layer_close(to_f64(out), oracle.get().moe_forward(x, idx, w, W1l, W2l), "packed forward")
+    rdx, rdw = oracle.get().moe_backward(x, idx, w, W1l, W2l, dy)
+    _close(to_f64(dx), rdx, "packed dx")
+    _close(dw.cpu().numpy().astype(np.float64), rdw, "packed dw")
+    for e in range(cfg.E):
+        r1, r2 = oracle.get().expert_weight_grads(x, idx, w, W1l[e], W2l[e], e, dy)
+        _close(to_f64(gW1[e]), r1, f"packed dW1[{e}]")
+        _close(to_f64(gW2[e]), r2, f"packed dW2[{e}]")
+    buf.close()
