@@ -84,3 +84,17 @@ def test_config_shapes():
     assert x.shape == (256, 256) and x.dtype == np.uint16
     rows = si.make_x_rows(si.CONFIGS["tiny"], np.array([3, 200]))
     np.testing.assert_array_equal(rows, x[[3, 200]])
+
+
+def test_dy_stream_is_seeded_normal_and_independent_of_x():
+    """The backward's upstream gradient: its own seeded stream, N(0, 1) in bf16, the same
+    bits on every call, different from x of the same workload, one slice per micro-batch."""
+    import numpy as np
+    import synth_inputs as si
+    cfg = si.custom("dy", T=256, H=256, I=128, E=4, k=2, tile=64, seed=77, micro_batches=2)
+    a, b = si.make_dy(cfg), si.make_dy(cfg)
+    assert a.dtype == np.uint16 and a.shape == (256, 256) and np.array_equal(a, b)
+    assert not np.array_equal(a, si.make_x(cfg))
+    assert not np.array_equal(a, si.make_dy(cfg, 1))
+    v = si.bf16_to_f64(a)
+    assert abs(v.mean()) < 0.02 and abs(v.std() - 1.0) < 0.02
