@@ -94,8 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *sched_full = drain + 1;
   uint64_t *sched_empty = sched_full + kSchedSlots;
   int32_t *sched = reinterpret_cast<int32_t *>(sched_empty + kSchedSlots);
-  int32_t *sched_rows = sched + kSchedSlots;  // the unit's live rows, published with its id
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched_rows + kSchedSlots);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched + kSchedSlots);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   int *never = abort_flag + 1;
 
@@ -157,8 +156,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int32_t ticket = atomicAdd(prm.sched + 0, 1);
           u = (ticket < n_units && !*abort) ? ticket : -1;
-          // the MMA thread takes the unit's size from the ring, not from global memory
-          sched_rows[sslot] = u >= 0 ? prm.mblk[3 * (u / prm.n_blocks) + 2] : 0;
           sched[sslot] = u;
           st_cluster_u32(cluster_map(smem_u32(sched + sslot), peer), (uint32_t)u);
           mbar_arrive(sched_full + sslot);
@@ -268,13 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const int32_t u = sched[sslot];
-        const int32_t rows = sched_rows[sslot];
         mbar_arrive(sched_empty + sslot);
         if (++sslot == kSchedSlots) {
           sslot = 0;
           sphase ^= 1u;
         }
         if (u < 0) break;
+        const int mb = u / prm.n_blocks;
+        const int32_t rows = prm.mblk[3 * mb + 2];
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32_ab(2 * kBM, n_mma, /*a_mn=*/!kAK, /*b_mn=*/false);
         // Both CTAs' epilogues have read the previous unit's accumulators.
