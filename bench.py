@@ -366,10 +366,11 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
     H, I, T = cfg.H, cfg.I, cfg.T
     fwd_ev = moe.moe_timing_events_create(7 * steps)
     farr = [(ctypes.c_void_p * 7)(*fwd_ev[7 * c: 7 * c + 7]) for c in range(steps)]
-    fcfg = [moe.moe_config(0, 0, 0, packed, ffn_kernel, ctypes.cast(a, ctypes.c_void_p))
+    # the training step keeps g | u, which needs the SM-pair kernels (the default)
+    fcfg = [moe.moe_config(0, 0, 0, packed, moe.MOE_FFN_SM_PAIR, ctypes.cast(a, ctypes.c_void_p))
             for a in farr]
     for _ in range(3):
-        buf.forward(x, idx, w, W1, W2, moe.moe_config(0, 0, 0, packed, ffn_kernel, None),
+        buf.forward(x, idx, w, W1, W2, moe.moe_config(0, 0, 0, packed, moe.MOE_FFN_SM_PAIR, None),
                     save_for_backward=True)
     torch.cuda.synchronize()
     barrier(world)
