@@ -356,8 +356,8 @@ def streams_weights(pairs: float, n_live_experts: float, peaks: dict) -> bool:
     return pairs / max(n_live_experts, 1.0) < ridge
 
 
-def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed, ffn_kernel,
-                  pairs, peaks, peak_src, steps):
+def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed, pairs, peaks,
+                  peak_src, steps):
     """A training step of the layer on micro-batch 0: the forward that also keeps the gate /
     up values (moe_config.gate_up) and the backward that reads them, each timed over
     `steps` calls back to back with per-phase CUDA events (max over ranks)."""
@@ -683,8 +683,8 @@ def run_moe(args):
     # every call recomputes the same gradients from the forward's plan, pool and ypool
     if do_bwd:
         line["backward"] = time_backward(moe, buf, cfg, dev, world, dx[0], didx[0], dw[0], W1,
-                                         W2, W1u, W2u, packed, ffn_kernel, pairs[0], peaks,
-                                         peak_src, args.steps)
+                                         W2, W1u, W2u, packed, pairs[0], peaks, peak_src,
+                                         args.steps)
 
     # ---------------- e2e: pinned host inputs in, result out, copies inside the timed region
     hx = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in xs]
