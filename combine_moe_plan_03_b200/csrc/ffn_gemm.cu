@@ -559,7 +559,18 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
                         const moe_config &cfg, int num_sms, cudaStream_t st,
                         cudaEvent_t const *tev) {
   const PlanGeom g = plan_geom(s);
-  if (g.pmax == 0) return MOE_OK;
+  if (g.pmax == 0) {
+    // no rows at all (T = 0): the weight gradients are zero, the phases empty
+    if (dW1 != nullptr &&
+        cudaMemsetAsync(dW1, 0, (size_t)s.E * s.H * 2 * s.I * sizeof(uint16_t), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (dW2 != nullptr &&
+        cudaMemsetAsync(dW2, 0, (size_t)s.E * s.I * s.H * sizeof(uint16_t), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    for (int i = 2; tev != nullptr && i <= 6; ++i)
+      if (cudaEventRecord(tev[i], st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
   CUtensorMap tw1_mn, tw2_k, tw1_k, tx_pool, tx_dy, tx_dgu;
   if (!make_tmap(&tw1_mn, W1, 2ull * s.I, (uint64_t)s.E * s.H, kBK) ||
       !make_tmap(&tw2_k, W2, (uint64_t)s.H, (uint64_t)s.E * s.I, 128) ||

@@ -163,7 +163,8 @@ def test_backward_edge_cases(case):
 
 
 def test_backward_no_live_pairs_and_no_tokens():
-    """Every pair dropped: dx = 0 and dw = 0 with no device error. T = 0: nothing to do."""
+    """Every pair dropped: dx = 0 and dw = 0 with no device error. T = 0: no rows, so the
+    weight gradients are exactly zero."""
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import bf16_dev, f32_dev, i32_dev, weights_dev
     cfg = si.custom("alldrop", T=40, H=128, I=128, E=4, k=2, tile=64, seed=5)
@@ -179,9 +180,12 @@ def test_backward_no_live_pairs_and_no_tokens():
     ei = torch.empty((0, 2), dtype=torch.int32, device="cuda")
     ew = torch.empty((0, 2), dtype=torch.float32, device="cuda")
     buf.forward(e, ei, ew, W1, W2)
-    dx, dw = buf.backward(e, ew, W1, W2)
+    gW1 = torch.full((4, 128, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gW2 = torch.full((4, 128, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dx, dw = buf.backward(e, ew, W1, W2, dW1=gW1, dW2=gW2)
     torch.cuda.synchronize()
     assert moe.moe_get_status(buf.plan)[0] == 0 and dx.numel() == 0 and dw.numel() == 0
+    assert not gW1.float().abs().sum().item() and not gW2.float().abs().sum().item()
     buf.close()
 
 
