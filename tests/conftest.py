@@ -9,3 +9,8 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the CUDA library")
     config.addinivalue_line("markers", "slow: full-size case (minutes)")
+    # A fresh checkout has no built libraries (they are not committed): build them once,
+    # as __graft_entry__.build() does, so that the package and the oracle import.
+    if not os.path.exists(os.path.join(ROOT, "combine_moe_plan_03_b200", "libmoe.so")):
+        import __graft_entry__
+        __graft_entry__.build()
