@@ -458,9 +458,30 @@ def time_backward(moe, buf, cfg, dev, world, x, idx, w, W1, W2, W1u, W2u, packed
                     "same gradients"}
 
 
+def ensure_library(local: int) -> None:
+    """Build libmoe.so when it is missing (a checkout without built libraries): the first
+    local rank builds, the others wait for the file to appear and stop growing."""
+    lib = os.path.join(ROOT, "combine_moe_plan_03_b200", "libmoe.so")
+    if os.path.exists(lib):
+        return
+    if local == 0:
+        import __graft_entry__
+        __graft_entry__.build()
+        return
+    t0, last = time.time(), -1
+    while time.time() - t0 < 900:
+        size = os.path.getsize(lib) if os.path.exists(lib) else -1
+        if size > 0 and size == last:
+            return
+        last = size
+        time.sleep(2.0)
+    raise RuntimeError("libmoe.so was not built in time by local rank 0")
+
+
 def run_moe(args):
     import torch
     rank, world, local = dist_env()
+    ensure_library(local)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
