@@ -94,6 +94,7 @@ def _load():
         "moe_route_plan": [P(moe_shape), vp, vp, vp, vp, P(moe_plan_buffers), vp, vp],
         "moe_packed_weight_bytes": [P(moe_shape), P(ctypes.c_size_t), P(ctypes.c_size_t)],
         "moe_pack_weights": [P(moe_shape), vp, vp, vp, vp, vp],
+        "moe_hbm_probe": [vp, vp, ctypes.c_size_t, i32, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -114,7 +115,7 @@ EXPORTS = ["moe_route", "moe_route_plan", "moe_packed_weight_bytes", "moe_pack_w
            "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
            "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
-           "moe_version"]
+           "moe_hbm_probe", "moe_version"]
 
 
 def lib():
@@ -151,6 +152,13 @@ def moe_pack_weights(shape, w1_ptr: int, w2_ptr: int, w1p_ptr: int, w2p_ptr: int
                      stream: int = 0) -> None:
     _check("moe_pack_weights", _lib.moe_pack_weights(ctypes.byref(_shape(shape)), w1_ptr, w2_ptr,
                                                      w1p_ptr, w2p_ptr, stream or None))
+
+
+def moe_hbm_probe(dst_ptr: int, src_ptr: int, nbytes: int, mode: int, stream: int = 0) -> None:
+    """One write-only (mode 0: 16-byte stores, 1: 16 KB bulk stores) or copy (mode 2) pass
+    over nbytes of device memory: the HBM rates the layer's copy kernels are compared with."""
+    _check("moe_hbm_probe", _lib.moe_hbm_probe(dst_ptr, src_ptr or None, nbytes, mode,
+                                               stream or None))
 
 
 def moe_pool_rows_max(shape) -> int:

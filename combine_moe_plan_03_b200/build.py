@@ -25,7 +25,10 @@ def sources():
 
 def build(verbose: bool = False, out: str = LIB) -> str:
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, "-o", out, *sources()]
+    # nvcc writes a file of this process's own, renamed into place once complete: no other
+    # process can load a half-written library
+    tmp = f"{out}.tmp{os.getpid()}"
+    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd))
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -33,7 +36,10 @@ def build(verbose: bool = False, out: str = LIB) -> str:
         sys.stdout.write(res.stdout)
         sys.stderr.write(res.stderr)
     if res.returncode != 0:
+        if os.path.exists(tmp):
+            os.unlink(tmp)
         raise RuntimeError("nvcc failed")
+    os.replace(tmp, out)
     return out
 
 

@@ -15,6 +15,8 @@
 //                           w / kPadPieces (all padding rows are in the expert's last tile)
 //   item kPadPieces*E + t   token t
 // HBM traffic per call: T*H*2 read + (live pairs + padding rows)*H*2 written.
+#include <mutex>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -161,16 +163,23 @@ __global__ void __launch_bounds__(32)
 cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_buffers &p,
                             void *pool, int signal, int num_sms, cudaStream_t st) {
   const uint32_t row_bytes = (uint32_t)s.H * 2;
-  const size_t smem = 3 * (size_t)row_bytes + 2 * sizeof(uint64_t) + 16;
+  const size_t smem = dispatch_smem_bytes(s.H);
+  if (smem > kMaxSmemPerBlock) return cudaErrorInvalidValue;  // refused by check_shape first
+  // the kernel's shared-memory limit only grows, under a lock (host threads may launch
+  // on the same device at once)
+  static std::mutex mu;
   static size_t attr_smem[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (attr_smem[dev] < smem) {
-    cudaError_t e = cudaFuncSetAttribute(dispatch_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_smem[dev] = smem;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (attr_smem[dev] < smem) {
+      cudaError_t e = cudaFuncSetAttribute(
+          dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr_smem[dev] = smem;
+    }
   }
   const int per_sm = (int)(200 * 1024 / smem) > 0 ? (int)(200 * 1024 / smem) : 1;
   const int64_t items = (int64_t)kPadPieces * s.E + s.T;

@@ -238,14 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (*abort) {
-        if (lead)
-          for (int s = 0; s < kStages; ++s)
-            if (issued & (1u << s))
-              mbar_wait(full + s, (last_parity >> s) & 1u, prm.timeout_ns, never);
-      } else if (lead) {
-        // Every cluster has taken its end ticket before it counts itself done, so the
-        // last one may zero the counters for the next launch.
+      if (*abort && lead)
+        for (int s = 0; s < kStages; ++s)
+          if (issued & (1u << s))
+            mbar_wait(full + s, (last_parity >> s) & 1u, prm.timeout_ns, never);
+      if (lead) {
+        // Every cluster has taken its last ticket (the end ticket, or the one before an
+        // abort) before it counts itself done, so the last one may zero the counters for
+        // the next launch, on the abort path too.
         __threadfence();
         if (atomicAdd(prm.sched + 1, 1) == (int)(gridDim.x >> 1) - 1) {
           atomicExch(prm.sched + 0, 0);

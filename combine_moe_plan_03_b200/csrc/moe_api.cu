@@ -36,6 +36,7 @@ int check_shape(const moe_shape *s, bool need_ffn) {
   if (s->k > kMaxTopK || s->E > kMaxExperts) return MOE_ERR_INVALID_ARG;
   if (s->tile != 64 && s->tile != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s->H % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dispatch_smem_bytes(s->H) > kMaxSmemPerBlock) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (need_ffn && (s->I <= 0 || s->I % 64 != 0)) return MOE_ERR_UNSUPPORTED_SHAPE;
   const PlanGeom g = plan_geom(*s);
   if (g.pairs > INT32_MAX || g.pmax > INT32_MAX) return MOE_ERR_INVALID_ARG;
@@ -383,8 +384,12 @@ int moe_get_status(const moe_plan_buffers *p, int32_t *code, int32_t *aux) {
 
 int moe_clear_status(const moe_plan_buffers *p, void *stream) {
   if (p == nullptr || p->status == nullptr) return MOE_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(p->status, 0, 4 * sizeof(int32_t), static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(p->status, 0, 4 * sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+  // the grouped GEMMs' unit counters (meta[4..7]), so that a GEMM run again on the same
+  // plan after a failed one starts from its first unit
+  if (p->meta != nullptr &&
+      cudaMemsetAsync(p->meta + 4, 0, 4 * sizeof(int32_t), st) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

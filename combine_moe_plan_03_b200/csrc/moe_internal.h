@@ -15,6 +15,13 @@ constexpr int kPlanWarps = 8;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kGemmBlockM = 256;  // most live rows of one expert in one grouped-GEMM unit
+constexpr size_t kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per block (227 KB)
+
+// Dynamic shared memory of the dispatch kernel: two staging rows of x, one row of zeros
+// (H bf16 each) and its barriers. Shapes whose rows do not fit are refused on the host.
+inline size_t dispatch_smem_bytes(int32_t H) {
+  return 3 * (size_t)H * 2 + 2 * sizeof(uint64_t) + 16;
+}
 
 // Rows per grouped-GEMM chunk for an expert with c live rows: the rows are cut into
 // ceil(c / 256) chunks of equal size, rounded up to a multiple of 16 (the MMA's N step).

@@ -20,9 +20,11 @@
 //     reads and zeroes the finalize counter, so no state leaks between calls
 //     that run one after the other; calls that overlap on the GPU (concurrent
 //     streams) race on the buffer and must not be issued.
-//   - The device address of the buffer is looked up once per device, on the first
-//     call made with that device current (cudaGetSymbolAddress). Make that first
-//     call before any stream capture.
+//   - The device address of the buffer is looked up once per device context, on the
+//     first call made with that device current (cudaGetSymbolAddress). Make that first
+//     call before any stream capture. The address is cached per CUDA context, so a
+//     call after cudaDeviceReset (which gives the device a new context and reloads the
+//     module) looks it up again instead of reusing a stale one.
 //   - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include <mutex>
 
@@ -37,22 +39,66 @@ static __device__ __align__(256) int32_t g_plan_scratch[kNoallocScratchInts];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+// Cached addresses, one per CUDA context, keyed by the context's process-unique id (a
+// device's primary context gets a new id when a device reset re-creates it); the oldest
+// entry is replaced when the table is full.
+constexpr int kCacheSlots = 64;
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  int32_t *ptr;
+};
 std::mutex g_scratch_mu;
-int32_t *g_scratch_ptr[kMaxDevices] = {nullptr};
+ScratchSlot g_scratch_cache[kCacheSlots] = {};
+int g_scratch_next = 0;
 
-// Device address of g_plan_scratch on the current device (looked up once per device).
-int scratch_for_current_device(int32_t **out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_plan_scratch) != cudaSuccess || ptr == nullptr)
-      return MOE_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<int32_t *>(ptr);
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+void *driver_entry(const char *name) {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
+}
+
+// Id of the context the runtime uses on the current device.
+int current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_ctx = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (get_ctx == nullptr) get_ctx = reinterpret_cast<CtxGetCurrentFn>(driver_entry("cuCtxGetCurrent"));
+  if (get_id == nullptr) get_id = reinterpret_cast<CtxGetIdFn>(driver_entry("cuCtxGetId"));
+  if (get_ctx == nullptr || get_id == nullptr) return MOE_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+  if (ctx == nullptr) {
+    // no context current yet: cudaSetDevice makes the device's primary context current
+    // (it allocates nothing)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MOE_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  return get_id(ctx, id) == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Device address of g_plan_scratch in the current context (looked up once per context).
+int scratch_for_current_device(int32_t **out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  unsigned long long id = 0;
+  int rc = current_context_id(&id);
+  if (rc != MOE_OK) return rc;
+  for (int i = 0; i < kCacheSlots; ++i)
+    if (g_scratch_cache[i].ptr != nullptr && g_scratch_cache[i].ctx_id == id) {
+      *out = g_scratch_cache[i].ptr;
+      return MOE_OK;
+    }
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_plan_scratch) != cudaSuccess || ptr == nullptr)
+    return MOE_ERR_CUDA;
+  g_scratch_cache[g_scratch_next] = ScratchSlot{id, static_cast<int32_t *>(ptr)};
+  g_scratch_next = (g_scratch_next + 1) % kCacheSlots;
+  *out = static_cast<int32_t *>(ptr);
   return MOE_OK;
 }
 

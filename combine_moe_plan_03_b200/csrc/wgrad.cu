@@ -203,12 +203,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (*abort) {
-        if (lead)
-          for (int s = 0; s < kStages; ++s)
-            if (issued & (1u << s))
-              mbar_wait(full + s, (last_parity >> s) & 1u, prm.timeout_ns, never);
-      } else if (lead) {
+      if (*abort && lead)
+        for (int s = 0; s < kStages; ++s)
+          if (issued & (1u << s))
+            mbar_wait(full + s, (last_parity >> s) & 1u, prm.timeout_ns, never);
+      if (lead) {
+        // counted done on the abort path too (its last ticket is taken), so the last
+        // cluster zeroes the counters for the next launch in every case
         __threadfence();
         if (atomicAdd(prm.sched + 1, 1) == (int)(gridDim.x >> 1) - 1) {
           atomicExch(prm.sched + 0, 0);

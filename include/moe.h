@@ -63,7 +63,9 @@ extern "C" {
 /* ---- error codes ------------------------------------------------------------------- */
 #define MOE_OK 0
 #define MOE_ERR_INVALID_ARG (-1)       /* null pointer, negative size, k > 32, E > 1024 ... */
-#define MOE_ERR_UNSUPPORTED_SHAPE (-2) /* H or I not a multiple of 64, tile not 64 or 128 */
+#define MOE_ERR_UNSUPPORTED_SHAPE (-2) /* H or I not a multiple of 64, tile not 64 or 128,
+                                          H above 38,720 (3 rows of x must fit in the 227 KB
+                                          of shared memory of one dispatch block) */
 #define MOE_ERR_MISALIGNED (-3)        /* a tensor pointer not 16-byte aligned */
 #define MOE_ERR_CUDA (-4)              /* a CUDA runtime / driver call failed */
 #define MOE_ERR_NO_DEVICE (-5)         /* current device is not sm_100 */
@@ -282,7 +284,10 @@ int moe_event_elapsed_ms(void *start, void *end, float *ms);
 /* Read the status word (synchronous: waits for work already queued that writes it). */
 int moe_get_status(const moe_plan_buffers *p, int32_t *code, int32_t *aux);
 
-/* Zero the status word on `stream`. */
+/* Zero the status word on `stream`, and (when p->meta is set) the grouped GEMMs' unit
+ * counters meta[4..7], so that an FFN re-run on the same plan after a device error starts
+ * from its first unit. Call it while no layer call that uses these plan buffers is in
+ * flight. */
 int moe_clear_status(const moe_plan_buffers *p, void *stream);
 
 /* Text for an error code. */
@@ -307,12 +312,26 @@ const char *moe_strerror(int code);
  *     back-to-back calls are independent, but calls that overlap on the GPU
  *     (issued on concurrent streams) race on it.
  *   - The first call on a device (with that device current) looks up the
- *     buffer's device address; make it before any stream capture.
+ *     buffer's device address; make it before any stream capture. The address
+ *     is kept per CUDA context: after a device reset the next call looks it up
+ *     again.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 #define MOE_PLAN_NOALLOC_SCRATCH_INTS ((1 << 19) + 64)
 int moe_plan_noalloc(const moe_shape *s, const int32_t *topk_idx, const moe_plan_buffers *p,
                      int32_t *host_P, void *stream);
+
+/*
+ * HBM rate probe (a measurement aid, not part of the pages' method): one launch on `stream`
+ * that only writes `bytes` of zeros to dst (mode 0: 16-byte vector stores; mode 1:
+ * cp.async.bulk stores of 16 KB blocks from shared memory, the store form of moe_dispatch;
+ * bytes a multiple of 16 KB), or copies src to dst (mode 2: 16-byte vector loads and
+ * stores). Timed with events around it on a buffer far larger than L2 it gives the write and
+ * copy rates this library's own kernels reach, the ceilings dispatch and combine are
+ * compared with. dst (and src) are caller-owned device buffers, 16-byte aligned; bytes a
+ * multiple of 16. Errors: MOE_ERR_INVALID_ARG, MOE_ERR_MISALIGNED, MOE_ERR_CUDA.
+ */
+int moe_hbm_probe(void *dst, const void *src, size_t bytes, int32_t mode, void *stream);
 
 /* Library version string. */
 const char *moe_version(void);

@@ -28,10 +28,14 @@ CFLAGS = ["-O2", "-ffp-contract=off", "-fopenmp", "-shared", "-fPIC", "-std=c11"
 
 def build(src: str = SRC, out: str = LIB_PATH, verbose: bool = False) -> str:
     """Compile the oracle (gcc, strict IEEE double: no fast-math, no FMA contraction)."""
-    cmd = ["gcc", *CFLAGS, "-o", out, src, "-lm"]
+    # written under a name of this process, then renamed into place: another process never
+    # loads a half-written library, and two builds at once do not mix their output
+    tmp = f"{out}.tmp{os.getpid()}"
+    cmd = ["gcc", *CFLAGS, "-o", tmp, src, "-lm"]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
     return out
 
 

@@ -49,10 +49,14 @@ def build(verbose: bool = False) -> str:
     import subprocess
 
     src = os.path.join(_HERE, "gen.c")
-    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11", "-o", _LIB_PATH, src, "-lm"]
+    # written under a name of this process, then renamed into place: another process never
+    # loads a half-written library, and two builds at once do not mix their output
+    tmp = f"{_LIB_PATH}.tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11", "-o", tmp, src, "-lm"]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
 

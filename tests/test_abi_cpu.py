@@ -42,6 +42,7 @@ def test_sizes_and_bind_are_host_only():
     ((16, 128, 128, 8, 33, 64), -1),    # k > 32
     ((16, 128, 128, 2000, 2, 64), -1),  # E > 1024
     ((-1, 128, 128, 8, 2, 64), -1),
+    ((16, 38784, 128, 8, 2, 64), -2),   # 3 rows of x exceed a dispatch block's shared memory
 ])
 def test_bad_shapes_rejected(shape, code):
     import combine_moe_plan_03_b200 as moe

@@ -89,3 +89,32 @@ def test_roofline_bound_choice():
     assert not bench.streams_weights(32768, 128, peaks)       # Qwen3-shaped layer
     assert bench.streams_weights(1024, 170, peaks)            # a decode micro-batch
     assert bench.streams_weights(0, 0, peaks)                 # nothing routed
+
+
+def test_tensor_peak_follows_the_clock_record():
+    import bench
+    peaks = {"hbm_gbs": 6508.8, "bf16_tflops": 1624.0, "bf16_tflops_sustained": 1372.3}
+    # a short region at the maximum clock: the burst rate
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.tensor_peak(full, 0.12, peaks, "measured")[0] == 1624.0
+    # the power cap seen briefly, clock still near its maximum: burst
+    brief = {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.tensor_peak(brief, 5.0, peaks, "measured")[0] == 1624.0
+    # seconds under the cap with the clock held well down: sustained
+    capped = {"sm_mhz": 1310.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    pk, why = bench.tensor_peak(capped, 4.0, peaks, "measured")
+    assert pk == 1372.3 and "sustained" in why
+    # held down, but the region is short: burst
+    assert bench.tensor_peak(capped, 0.6, peaks, "measured")[0] == 1624.0
+    # no clock record at all: burst
+    assert bench.tensor_peak({"sm_mhz": None, "sm_max_mhz": None, "reasons": []}, 3.0, peaks,
+                             "fallback")[0] == 1624.0
+
+
+def test_copy_bound_takes_the_slower_of_writes_and_all_bytes():
+    import bench
+    rates = {"write_v4_gbs": 4000.0, "write_bulk_gbs": 5000.0, "copy_gbs": 6000.0}
+    # write-heavy (dispatch-like): the writes at the best write rate bound it
+    assert abs(bench.copy_bound_ms(1e9, 9e9, rates) - 1e3 * 9e9 / 5e12) < 1e-9
+    # read-heavy (combine-like): all bytes at the copy rate
+    assert abs(bench.copy_bound_ms(8e9, 1e9, rates) - 1e3 * 9e9 / 6e12) < 1e-9

@@ -54,3 +54,32 @@ def test_silu_emulation_matches_definition():
     got = g.astype(np.float64) * u * y
     ref = g.astype(np.float64) * u / (1.0 + np.exp(-g.astype(np.float64)))
     assert np.all(np.abs(got - ref) <= 2e-5 * np.abs(ref) + 1e-30)
+
+
+def test_reciprocal_magic_constant_is_the_minimax_first_estimate():
+    """The reciprocal's first estimate takes the bit pattern M - bits(d). Over one binade
+    of d (the error repeats in every binade) the best M is the one whose largest relative
+    error is smallest; a scan finds it, and the constant in the kernels' header must be
+    within 1e-6 of that optimum (and its two Newton steps below 1e-5)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "combine_moe_plan_03_b200", "csrc",
+                            "ffn_gemm.cuh")).read()
+    M_hdr = int(re.search(r"constexpr int32_t kRecipMagic = (0x[0-9A-Fa-f]+);", src).group(1), 16)
+    d = np.linspace(1.0, 2.0, 400_001).astype(np.float32)
+    db = d.view(np.int32).astype(np.int64)
+    dd = d.astype(np.float64)
+
+    def first(M):
+        return (np.int64(M) - db).astype(np.int32).view(np.float32).astype(np.float64)
+
+    def err(M):
+        return np.abs(first(M) * dd - 1.0).max()
+
+    coarse = min(range(0x7EF00000, 0x7EF60000, 0x100), key=err)
+    best = min(range(coarse - 0x100, coarse + 0x100), key=err)
+    assert err(M_hdr) - err(best) < 1e-6
+    y = first(M_hdr)
+    for _ in range(2):
+        y = y * (2.0 - dd * y)
+    assert np.abs(y * dd - 1.0).max() < 1e-5

@@ -29,6 +29,13 @@ def _routing(case):
         cfg = si.CONFIGS["deepseek_v3"]
         idx, _ = si.make_routing(cfg)
         return cfg.T, cfg.E, cfg.k, cfg.tile, idx
+    if case == "largest_accepted":
+        # E = 256 experts and 524,288 pairs: 256 * 2048 chunk counts + 8 = 524,296 of the
+        # buffer's 524,352 ints, the largest shape of this E that fits
+        rng = np.random.default_rng(11)
+        T, E, k, tile = 65536, 256, 8, 128
+        idx = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+        return T, E, k, tile, idx
     rng = np.random.default_rng(7)
     T, E, k, tile = 3000, 40, 6, 64
     idx = rng.integers(0, 5, size=(T, k)).astype(np.int32)   # skewed: 5 hot experts
@@ -38,7 +45,7 @@ def _routing(case):
 
 def test_noalloc_plan_matches_moe_plan_two_calls_in_a_row():
     import combine_moe_plan_03_b200 as moe
-    for case in ("deepseek_v3", "skewed_with_drops"):       # two calls in a row, different shapes
+    for case in ("deepseek_v3", "skewed_with_drops", "largest_accepted"):  # calls in a row
         T, E, k, tile, idx = _routing(case)
         d_idx = torch.from_numpy(idx).cuda()
         ref = moe.MoELayerBuffers(T, 64, 64, E, k, tile, identity=True)
@@ -64,9 +71,13 @@ def test_noalloc_plan_matches_moe_plan_two_calls_in_a_row():
 
 def test_noalloc_plan_rejects_shapes_beyond_its_scratch():
     import combine_moe_plan_03_b200 as moe
-    # E=1024 experts with 1M pairs needs 1024 * 4096 + 8 ints > 2^19 + 64
-    s = moe.moe_shape(131072, 64, 64, 1024, 8, 128)
     p = moe.moe_plan_buffers(*([1 << 20] * 10))
-    with pytest.raises(moe.MoEError) as ei:
-        moe.moe_plan_noalloc(s, 1 << 20, p, 0, 0)
-    assert ei.value.code == moe.MOE_ERR_SCRATCH_LIMIT
+    # E=1024 experts with 1M pairs needs 1024 * 4096 + 8 ints > 2^19 + 64;
+    # one 256-pair chunk past the largest accepted E=256 shape needs 256 * 2049 + 8;
+    # one expert more than that shape needs 257 * 2048 + 8
+    for s in (moe.moe_shape(131072, 64, 64, 1024, 8, 128),
+              moe.moe_shape(65536 + 32, 64, 64, 256, 8, 128),
+              moe.moe_shape(65536, 64, 64, 257, 8, 128)):
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_plan_noalloc(s, 1 << 20, p, 0, 0)
+        assert ei.value.code == moe.MOE_ERR_SCRATCH_LIMIT
