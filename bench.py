@@ -49,6 +49,12 @@ def parse_args(argv=None):
                     help="1: prepack the weights once before timing (moe_pack_weights)")
     ap.add_argument("--ffn-kernel", type=int, default=0,
                     help="grouped-GEMM kernel: 1 one CTA per unit, 2 SM pairs; 0: default")
+    ap.add_argument("--early-combine", type=int, default=-1,
+                    help="1: combine fused into GEMM Y (early combine); 0: separate combine; "
+                         "-1: default")
+    ap.add_argument("--ab", type=int, default=1,
+                    help="1: also time early combine and streaming against the timed "
+                         "configuration, alternating on this GPU (reported under 'ab')")
     ap.add_argument("--backward", type=int, default=1,
                     help="1: also time moe_backward (after one forward), reported under 'backward'")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
@@ -409,6 +415,34 @@ def streams_weights(pairs: float, n_live_experts: float, peaks: dict) -> bool:
     return pairs / max(n_live_experts, 1.0) < ridge
 
 
+def ab_layer_ms(moe, buf, dx, didx, dw, W1, W2, variants: dict, rounds: int = 4,
+                calls: int = 10) -> dict:
+    """Layer time per call of each named moe_config, measured in alternating rounds of
+    `calls` calls (CUDA events from the communicate stream's start to the compute stream's
+    end), so that every variant sees the same clock and power state; the median round."""
+    import torch
+    mbs = len(dx)
+    res = {k: [] for k in variants}
+    for k, c in variants.items():                      # warm-up of each variant
+        for m in range(mbs):
+            buf.forward(dx[m], didx[m], dw[m], W1, W2, c)
+    torch.cuda.synchronize()
+    for _ in range(rounds):
+        for k, c in variants.items():
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(buf.comm)
+            for _ in range(calls):
+                for m in range(mbs):
+                    buf.forward(dx[m], didx[m], dw[m], W1, W2, c)
+            s1.record(buf.compute)
+            torch.cuda.synchronize()
+            res[k].append(s0.elapsed_time(s1) / calls)
+    code, aux = moe.moe_get_status(buf.plan)
+    if code != 0:
+        raise RuntimeError(f"device status after the A/B: {moe.moe_strerror(code)} ({aux})")
+    return {k: statistics.median(v) for k, v in res.items()}
+
+
 def time_backward(moe, buf, cfg, dev, world, local, x, idx, w, W1, W2, W1u, W2u, packed, pairs,
                   peaks, peak_src, steps):
     """A training step of the layer on micro-batch 0: the forward that also keeps the gate /
@@ -556,6 +590,7 @@ def run_moe(args):
     cfg = si.CONFIGS[args.workload]
     peaks, peak_src = load_peaks()
     streaming = 0 if args.streaming < 0 else args.streaming
+    early = 0 if args.early_combine < 0 else args.early_combine
     mbs = cfg.micro_batches
     want_cpu = (world == 1 and rank == 0 and not args.no_cpu_baseline)
 
@@ -593,10 +628,11 @@ def run_moe(args):
     tev = moe.moe_timing_events_create(7 * calls)
     import ctypes
     ev_arrays = [(ctypes.c_void_p * 7)(*tev[7 * c: 7 * c + 7]) for c in range(calls)]
+    early = early if not cfg.identity else 0
     cfgs = [moe.moe_config(streaming, 0, 0, packed, ffn_kernel,
-                           ctypes.cast(ev_arrays[c], ctypes.c_void_p))
+                           ctypes.cast(ev_arrays[c], ctypes.c_void_p), None, early)
             for c in range(calls)]
-    plain = moe.moe_config(streaming, 0, 0, packed, ffn_kernel, None)
+    plain = moe.moe_config(streaming, 0, 0, packed, ffn_kernel, None, None, early)
 
     def step_plain():
         for m in range(mbs):
@@ -661,7 +697,8 @@ def run_moe(args):
     disp_bytes = T * H * 2 + P_m * H * 2
     comb_bytes = pairs_m * H * 2 + T * H * 2 + pairs_m * 8
     dc_ms = ph["dispatch"] + ph["combine"]
-    dc_gbs = (disp_bytes + comb_bytes) / (dc_ms / 1000.0) / 1e9
+    # with early combine the combine runs inside GEMM Y: no rate of its own
+    dc_gbs = (disp_bytes + comb_bytes) / (dc_ms / 1000.0) / 1e9 if not early else None
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -669,14 +706,16 @@ def run_moe(args):
             "config": dict(config_block(cfg, world),
                            weights="prepacked tiles (moe_pack_weights, once before timing)"
                            if packed else "as given: W1 [E,H,2I], W2 [E,I,H]"),
-            "streaming": streaming, "ffn_kernel": ffn_kernel,
+            "streaming": streaming, "ffn_kernel": ffn_kernel, "early_combine": early,
             "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
             "phases_mcycles_per_call": ({k: round(v * clocks["sm_mhz"] / 1000.0, 4)
                                          for k, v in ph.items()} if clocks.get("sm_mhz") else None),
             "dispatch_combine": {"bytes_per_call": disp_bytes + comb_bytes,
-                                 "gbs": dc_gbs, "frac_hbm": dc_gbs / peaks["hbm_gbs"],
+                                 "gbs": dc_gbs,
+                                 "frac_hbm": dc_gbs / peaks["hbm_gbs"] if dc_gbs else None,
                                  "dispatch_gbs": disp_bytes / (ph["dispatch"] / 1e3) / 1e9,
-                                 "combine_gbs": comb_bytes / (ph["combine"] / 1e3) / 1e9,
+                                 "combine_gbs": (comb_bytes / (ph["combine"] / 1e3) / 1e9
+                                                 if not early else None),
                                  "padding_bytes": (P_m - pairs_m) * H * 2}}
     # the HBM ceilings of dispatch and combine on this GPU, from this library's own probe kernels
     probe = hbm_probe_rates(moe, dev)
@@ -685,7 +724,8 @@ def run_moe(args):
     line["dispatch_combine"].update({
         "probe": probe,
         "dispatch_bound_ms": d_bound, "dispatch_frac_of_bound": d_bound / ph["dispatch"],
-        "combine_bound_ms": c_bound, "combine_frac_of_bound": c_bound / ph["combine"],
+        "combine_bound_ms": c_bound,
+        "combine_frac_of_bound": c_bound / ph["combine"] if not early else None,
         "bound_note": "shortest time at the probed write-only and copy rates (moe_hbm_probe)"})
     if not cfg.identity:
         flops_a = pairs_m * 4.0 * H * I
@@ -740,6 +780,18 @@ def run_moe(args):
                             "frac": achieved / peaks["hbm_gbs"],
                             "traffic": committed_traffic("dispatch_kernel", cfg.name),
                             "peak_source": f"{peak_src} HBM copy"}
+
+    # ---------------- same-GPU A/B of the layer's options against the timed configuration
+    if args.ab and not cfg.identity and world == 1:
+        def variant(s_, e_):
+            return moe.moe_config(s_, 0, 0, packed, ffn_kernel, None, None, e_)
+        ab = ab_layer_ms(moe, buf, dx, didx, dw, W1, W2, {
+            "timed": plain, "early_combine": variant(streaming, 1 - early),
+            "streaming": variant(1 - streaming, early)})
+        line["ab"] = {"ms_per_call": ab,
+                      "note": "median of 4 alternating rounds of 10 calls; 'early_combine' and "
+                              "'streaming' flip that one option of the timed configuration "
+                              f"(early_combine={early}, streaming={streaming})"}
 
     # ---------------- router on the device (not part of the layer step: the layer takes
     # topk_idx / topk_w as inputs); timed on its own with the workload's logits
@@ -833,7 +885,7 @@ def run_moe(args):
     d2h = mbs * cfg.T * cfg.H * 2
     line["e2e"] = {"value": world * tokens_step * args.steps / (e2e_ms / 1000.0),
                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    kernels_per_call = 5 if cfg.identity else 7
+    kernels_per_call = 5 if cfg.identity else (6 if early else 7)
     line["gpu_launches"] = kernels_per_call * calls   # the forward's timed region
     line["clocks"] = clocks
     if want_cpu and not cfg.identity:

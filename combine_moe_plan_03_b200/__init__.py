@@ -31,6 +31,9 @@ MOE_ERR_BAD_INDEX = -10
 MOE_ERR_FLAG_TIMEOUT = -11
 MOE_ERR_POOL_OVERFLOW = -12
 MOE_ERR_PIPE_TIMEOUT = -13
+MOE_ERR_COMBINE_TIMEOUT = -14
+MOE_DISPATCH_SIGNAL_TILES = 1
+MOE_DISPATCH_ARM_COMBINE = 2
 
 
 class moe_shape(ctypes.Structure):
@@ -41,14 +44,14 @@ class moe_shape(ctypes.Structure):
 class moe_plan_buffers(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "counts", "offsets", "pool_row", "row_src", "tile_expert", "mblk", "meta",
-        "tile_flags", "workspace", "status")]
+        "tile_flags", "workspace", "status", "tok_pending", "ready")]
 
 
 class moe_config(ctypes.Structure):
     _fields_ = [("streaming", ctypes.c_int32), ("ffn_ctas", ctypes.c_int32),
                 ("wait_timeout_us", ctypes.c_int32), ("packed_weights", ctypes.c_int32),
                 ("ffn_kernel", ctypes.c_int32), ("timing_events", ctypes.c_void_p),
-                ("gate_up", ctypes.c_void_p)]
+                ("gate_up", ctypes.c_void_p), ("early_combine", ctypes.c_int32)]
 
 
 MOE_FFN_ONE_SM = 1
@@ -79,6 +82,8 @@ def _load():
         "moe_grouped_ffn": [P(moe_shape), vp, vp, vp, P(moe_plan_buffers), vp, vp,
                             P(moe_config), vp],
         "moe_combine": [P(moe_shape), vp, vp, P(moe_plan_buffers), vp, vp],
+        "moe_grouped_ffn_combine": [P(moe_shape), vp, vp, vp, P(moe_plan_buffers), vp, vp, vp,
+                                    vp, P(moe_config), vp],
         "moe_forward": [P(moe_shape), vp, vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp,
                         P(moe_config), vp, vp, vp, vp],
         "moe_backward": [P(moe_shape), vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp, vp,
@@ -111,7 +116,8 @@ _lib = _load()
 
 # Names exported by include/moe.h, in declaration order.
 EXPORTS = ["moe_route", "moe_route_plan", "moe_packed_weight_bytes", "moe_pack_weights", "moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
-           "moe_dispatch", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_backward",
+           "moe_dispatch", "moe_grouped_ffn", "moe_grouped_ffn_combine", "moe_combine",
+           "moe_forward", "moe_backward",
            "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
            "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
@@ -212,7 +218,7 @@ def moe_route_plan(shape, logits_ptr: int, bias_ptr: int, topk_idx_ptr: int, top
 
 
 def moe_dispatch(shape, x_ptr: int, plan: moe_plan_buffers, pool_ptr: int,
-                 signal_flags: bool = False, stream: int = 0) -> None:
+                 signal_flags: int = 0, stream: int = 0) -> None:
     _check("moe_dispatch", _lib.moe_dispatch(ctypes.byref(_shape(shape)), x_ptr,
                                              ctypes.byref(plan), pool_ptr, int(signal_flags),
                                              stream or None))
@@ -225,6 +231,17 @@ def moe_grouped_ffn(shape, pool_ptr: int, w1_ptr: int, w2_ptr: int, plan: moe_pl
     _check("moe_grouped_ffn", _lib.moe_grouped_ffn(ctypes.byref(_shape(shape)), pool_ptr, w1_ptr,
                                                    w2_ptr, ctypes.byref(plan), act_ptr, ypool_ptr,
                                                    ctypes.byref(cfg), stream or None))
+
+
+def moe_grouped_ffn_combine(shape, pool_ptr: int, w1_ptr: int, w2_ptr: int,
+                            plan: moe_plan_buffers, act_ptr: int, ypool_ptr: int, topk_w_ptr: int,
+                            out_ptr: int, cfg: moe_config | None = None, stream: int = 0) -> None:
+    """Grouped FFN with the combine fused into GEMM Y (cfg.early_combine must be 1; the
+    plan's counters armed by moe_dispatch with MOE_DISPATCH_ARM_COMBINE)."""
+    cfg = cfg or moe_config(early_combine=1)
+    _check("moe_grouped_ffn_combine", _lib.moe_grouped_ffn_combine(
+        ctypes.byref(_shape(shape)), pool_ptr, w1_ptr, w2_ptr, ctypes.byref(plan), act_ptr,
+        ypool_ptr, topk_w_ptr or None, out_ptr or None, ctypes.byref(cfg), stream or None))
 
 
 def moe_combine(shape, ypool_ptr: int, topk_w_ptr: int, plan: moe_plan_buffers, out_ptr: int,

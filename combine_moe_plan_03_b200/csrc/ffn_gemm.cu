@@ -441,8 +441,9 @@ static cudaError_t launch_one(const CUtensorMap &tw, const CUtensorMap &tx, cons
 }
 
 int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void *W2,
-               const moe_plan_buffers &p, void *act, void *ypool, const moe_config &cfg,
-               int num_sms, cudaStream_t st) {
+               const moe_plan_buffers &p, void *act, void *ypool, const float *topk_w,
+               void *out, const moe_config &cfg, int num_sms, cudaStream_t st) {
+  const bool early = cfg.early_combine != 0;
   const PlanGeom g = plan_geom(s);
   if (g.pmax == 0) return MOE_OK;
   CUtensorMap tw1, tx_pool, tw2, tx_act;
@@ -461,7 +462,8 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
     return MOE_ERR_CUDA;
 
   const bool pair = (cfg.ffn_kernel != 0 ? cfg.ffn_kernel : MOE_FFN_DEFAULT) == MOE_FFN_SM_PAIR;
-  int grid = cfg.ffn_ctas > 0 ? cfg.ffn_ctas : (cfg.streaming ? num_sms - 16 : num_sms);
+  int grid = cfg.ffn_ctas > 0 ? cfg.ffn_ctas
+                              : (cfg.streaming ? num_sms - kStreamDispatchSMs : num_sms);
   if (grid < 1) grid = 1;
   int grid_y = cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms;
   if (pair) {
@@ -542,7 +544,18 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
     y.pk_nb = 4 * pg.kb2;
     y.pk_v = pg.kb2;
   }
-  e = pair ? launch_ffn_pair(1, false, tw2, tx_act, y, grid_y, st)
+  if (early) {
+    // GEMM Y combines every token once its k rows are stored (fused early combine)
+    y.row_src = p.row_src;
+    y.pool_row = p.pool_row;
+    y.topk_w = topk_w;
+    y.tok_pending = p.tok_pending;
+    y.ready = p.ready;
+    y.comb_out = static_cast<uint16_t *>(out);
+    y.T = s.T;
+    y.k = s.k;
+  }
+  e = pair ? launch_ffn_pair(1, false, tw2, tx_act, y, grid_y, st, early)
            : launch_one<1>(tw2, tx_act, y, grid_y, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;

@@ -38,6 +38,17 @@ struct FfnParams {
   // mode 3 (GEMM A saving gate / up): out = [g | u], act = bf16(silu(g) u) to out2
   uint16_t *out2;
   int64_t out2_ld;
+  // early combine (GEMM Y of the SM-pair kernel): per stored unit row, tok_pending[t] of the
+  // row's token t = row_src[p] / k drops by one; at zero t + 1 goes to the ready queue
+  // ready[0 .. T) (tail at ready[T + 1]); after their GEMM work the CTAs pop tokens (head
+  // at ready[T]) and write comb_out[t] = bf16(sum_j topk_w[t, j] ypool[pool_row[t, j]]).
+  const int32_t *row_src;
+  const int32_t *pool_row;
+  const float *topk_w;
+  int32_t *tok_pending;
+  int32_t *ready;
+  uint16_t *comb_out;
+  int32_t T, k;
 };
 
 // 2^x on the MUFU (ex2.approx.ftz.f32).
@@ -92,9 +103,10 @@ bool make_tmap_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t ou
 // mode 0: SwiGLU epilogue (GEMM A); 1: plain bf16 (GEMM Y, backward A, gate / up
 // recompute); 2: SwiGLU backward (backward Y); 3: GEMM A that also stores g | u. a_kmajor: the weights are read K-major
 // (rows of the tensor map are output columns: W2 for backward Y, W1 for backward A).
+// early: GEMM Y (mode 1, MN-major) with the combine fused in (prm.row_src ... comb_out).
 cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
                             const CUtensorMap &tx, const FfnParams &prm, int clusters,
-                            cudaStream_t st);
+                            cudaStream_t st, bool early = false);
 // Clusters of two of the pair kernel that fit on the device at once (0 on error).
 int ffn_pair_max_clusters(int mode);
 

@@ -29,6 +29,12 @@
 //           both CTAs and each finished unit to both CTAs' accumulator barriers.
 //   2-9     epilogue (both CTAs), as in the one-CTA kernel, over the CTA's own TMEM;
 //           a warp reports the accumulators read on the first CTA's barrier.
+//   10      early combine only (GEMM Y with the combine fused in): a signal warp. For each
+//           unit it waits until the CTA's epilogue warps have stored the unit's rows, then
+//           counts each row against its token (tok_pending, acquire-release); the count
+//           that reaches zero puts the token in the ready queue. After the GEMM work all
+//           warps of the CTA pop tokens from that queue and combine them (the same fp32
+//           FMA chain as combine.cu) while other CTAs still finish their last units.
 // Every wait is bounded as in the one-CTA kernel (flag T, producer / MMA 2T,
 // epilogue 3T); a wait that runs out raises the abort flag of both CTAs. Both CTAs
 // leave through two cluster barriers (with a grace period between them after an
@@ -51,12 +57,22 @@ constexpr int kHalfRows = kGemmBlockM / 2;            // pool rows per CTA (N / 
 constexpr int kStageBytes = 2 * kWTileBytes + kHalfRows * kBK * 2;  // 48 KB
 constexpr int kTmemCols = 512;
 constexpr int kAccStride = 256;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + kEpiWarps * 32;
+// Epilogue warps per CTA (a multiple of 4: the warps of one TMEM lane quadrant split the
+// unit's 32-row groups between them).
+#ifndef MOE_PAIR_EPI_WARPS
+#define MOE_PAIR_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = MOE_PAIR_EPI_WARPS;
+static_assert(kEpiWarps % 4 == 0 && kEpiWarps >= 8 && kEpiWarps <= 16, "4 lane quadrants");
+constexpr int kEpiParts = kEpiWarps / 4;              // warps per lane quadrant
+// 32-row groups of a unit (<= 256 rows) per warp: warp part p takes groups p, p + kEpiParts, ...
+constexpr int kGroupsPerWarp = (8 + kEpiParts - 1) / kEpiParts;
+constexpr int kSignalWarp = 2 + kEpiWarps;            // early combine only
+constexpr int threads_for(bool early) { return 64 + kEpiWarps * 32 + (early ? 32 : 0); }
 constexpr int kSchedSlots = 4;
 // readers of a unit id, all counted on the first CTA's sched_empty: its MMA thread and
-// epilogue warps, the second CTA's producer and epilogue warps
-constexpr int kSchedReaders = 1 + kEpiWarps + 1 + kEpiWarps;
+// epilogue warps, the second CTA's producer and epilogue warps (and both signal warps)
+constexpr int sched_readers(bool early) { return 1 + kEpiWarps + 1 + kEpiWarps + (early ? 2 : 0); }
 constexpr int kBarrierBytes = 256;
 constexpr int kXposeBytes = 32 * 32 * 2;
 constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kEpiWarps * kXposeBytes + 1024;
@@ -78,10 +94,102 @@ __device__ __forceinline__ void swiglu_backward(float da, float g, float u, floa
   dg = da * u * (s * fmaf(g, 1.0f - s, 1.0f));
 }
 
-template <int kMode, bool kAK>
-__global__ void __launch_bounds__(kThreads, 1)
+// 16-byte load through L2 only (rows that another SM wrote during this kernel).
+__device__ __forceinline__ uint4 ld_cg_v4(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fma_row8(float (&acc)[8], float w, const uint4 &v) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+    acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
+  }
+}
+
+// Early combine, after the CTA's GEMM work: each warp pops positions of the ready queue and
+// combines their tokens, out[t] = bf16(sum_j w[t, j] ypool[pool_row[t, j]]) as an fp32 FMA
+// chain over j ascending (combine.cu's arithmetic, so the result is bit-identical).
+__device__ void early_combine_drain(const FfnParams &prm, int lane, uint64_t timeout_ns) {
+  const int hv = prm.n_out / 8;  // 16-byte vectors per row
+  const uint4 *yp = reinterpret_cast<const uint4 *>(prm.out);
+  uint4 *op = reinterpret_cast<uint4 *>(prm.comb_out);
+  for (;;) {
+    int32_t pos = 0;
+    if (lane == 0) pos = atomicAdd(prm.ready + prm.T, 1);
+    pos = __shfl_sync(0xffffffffu, pos, 0);
+    if (pos >= prm.T) break;
+    int32_t v = 0;
+    if (lane == 0) {
+      v = ld_acquire_gpu_s32(prm.ready + pos);
+      if (v == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t sleep_ns = 64;
+        while ((v = ld_acquire_gpu_s32(prm.ready + pos)) == 0) {
+          if (globaltimer_ns() - t0 > timeout_ns) break;
+          __nanosleep(sleep_ns);
+          if (sleep_ns < 2048) sleep_ns <<= 1;
+        }
+      }
+      if (v == 0) report(prm.status, MOE_ERR_COMBINE_TIMEOUT, pos);
+    }
+    v = __shfl_sync(0xffffffffu, v, 0);
+    if (v == 0) break;
+    __syncwarp();  // lane 0's acquire orders the other lanes' loads of the token's rows
+    const int64_t t = v - 1;
+    int32_t my_row = -1;
+    float my_w = 0.0f;
+    if (lane < prm.k) {
+      my_row = prm.pool_row[t * prm.k + lane];
+      my_w = prm.topk_w[t * prm.k + lane];
+    }
+    for (int c = lane; c < hv; c += 64) {
+      const int c1 = c + 32;
+      float a0[8], a1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.0f;
+      for (int j0 = 0; j0 < prm.k; j0 += 8) {
+        uint4 y0[8], y1[8];
+        int32_t rr[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          rr[jj] = __shfl_sync(0xffffffffu, my_row, (j0 + jj) & 31);
+          if (j0 + jj < prm.k && rr[jj] >= 0) {
+            y0[jj] = ld_cg_v4(yp + (size_t)rr[jj] * hv + c);
+            if (c1 < hv) y1[jj] = ld_cg_v4(yp + (size_t)rr[jj] * hv + c1);
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float w = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
+          if (j0 + jj < prm.k && rr[jj] >= 0) {
+            fma_row8(a0, w, y0[jj]);
+            if (c1 < hv) fma_row8(a1, w, y1[jj]);
+          }
+        }
+      }
+      op[(size_t)t * hv + c] = make_uint4(pack_bf16x2(a0[0], a0[1]), pack_bf16x2(a0[2], a0[3]),
+                                          pack_bf16x2(a0[4], a0[5]), pack_bf16x2(a0[6], a0[7]));
+      if (c1 < hv)
+        op[(size_t)t * hv + c1] =
+            make_uint4(pack_bf16x2(a1[0], a1[1]), pack_bf16x2(a1[2], a1[3]),
+                       pack_bf16x2(a1[4], a1[5]), pack_bf16x2(a1[6], a1[7]));
+    }
+  }
+}
+
+template <int kMode, bool kAK, bool kEarly>
+__global__ void __launch_bounds__(threads_for(kEarly), 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                          const __grid_constant__ CUtensorMap tm_x, const FfnParams prm) {
+  static_assert(!kEarly || (kMode == 1 && !kAK), "early combine is GEMM Y's");
+  constexpr int kSchedReaders = sched_readers(kEarly);
   extern __shared__ uint8_t smem_raw[];
   // The same offsets in both CTAs (the MMA reads both CTAs' operands at one address).
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -97,6 +205,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched + kSchedSlots);
   int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
   int *never = abort_flag + 1;
+  // early combine: per sched slot, how many epilogue warps have stored their rows of the
+  // slot's units so far (monotonic: unit `local` is stored when it reaches
+  // kEpiWarps * (local / kSchedSlots + 1))
+  uint32_t *stored = reinterpret_cast<uint32_t *>(never + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -116,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kSchedSlots; ++i) {
       mbar_init(sched_full + i, 1);
       mbar_init(sched_empty + i, kSchedReaders);
+      if (kEarly) stored[i] = 0;
     }
     *abort_flag = 0;
     *never = 0;
@@ -318,10 +431,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit_pair_mc(drain, 0x1);
       mbar_wait(drain, 0, prm.timeout_ns, never);
     }
+  } else if (kEarly && warp == kSignalWarp) {
+    // -------------------------------------------------------------- early-combine signals
+    uint32_t sslot = 0, sphase = 0;
+    for (uint32_t local = 0;; ++local) {
+      int32_t u = -1;
+      int got = 1;
+      if (lane == 0) {
+        got = mbar_wait_parked<true>(sched_full + sslot, sphase, 3 * prm.timeout_ns, abort,
+                                     kParkNs)
+                  ? 1
+                  : 0;
+        if (got) {
+          u = sched[sslot];
+          if (lead)
+            mbar_arrive(sched_empty + sslot);
+          else
+            mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
+        }
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (++sslot == kSchedSlots) {
+        sslot = 0;
+        sphase ^= 1u;
+      }
+      if (!got) {
+        if (lane == 0) raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
+        break;
+      }
+      if (u < 0) break;
+      int ok = 1;
+      if (lane == 0) {
+        // all of this CTA's epilogue warps have stored the unit (bounded, sleeping poll)
+        const uint32_t want = kEpiWarps * (local / kSchedSlots + 1);
+        uint32_t *cnt = stored + (local % kSchedSlots);
+        if (ld_acquire_cta_shared(cnt) < want) {
+          const uint64_t t0 = globaltimer_ns();
+          uint32_t sleep_ns = 64;
+          while (ld_acquire_cta_shared(cnt) < want) {
+            if (*abort || globaltimer_ns() - t0 > 3 * prm.timeout_ns) {
+              ok = 0;
+              break;
+            }
+            __nanosleep(sleep_ns);
+            if (sleep_ns < 1024) sleep_ns <<= 1;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+        break;
+      }
+      // every row of the unit once per CTA: the token's count drops by one (release: the
+      // epilogue's stores before it; acquire: the other CTAs' stores, for the combine)
+      const int mb = u / prm.n_blocks;
+      const int32_t row0 = prm.mblk[3 * mb + 0];
+      const int32_t rows = prm.mblk[3 * mb + 2];
+      for (int r = lane; r < rows; r += 32) {
+        const int32_t f = prm.row_src[row0 + r];
+        if (f < 0) continue;
+        const int32_t t = f / prm.k;
+        if (atom_add_acq_rel_gpu(prm.tok_pending + t, -1) == 1) {
+          const int32_t qpos = atomicAdd(prm.ready + prm.T + 1, 1);
+          if (qpos < prm.T)
+            st_release_gpu(prm.ready + qpos, t + 1);
+          else  // more tokens completed than exist: counters armed twice for one plan
+            report(prm.status, MOE_ERR_COMBINE_TIMEOUT, qpos);
+        }
+      }
+    }
   } else {
     // -------------------------------------------------------------- epilogue
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;   // which of the quadrant's row-group parts
     const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
     uint16_t *xp = reinterpret_cast<uint16_t *>(smem + kStages * kStageBytes + kBarrierBytes) +
                    (warp - 2) * (kXposeBytes / 2);
@@ -372,15 +556,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t cb1 = cb0 + prm.col1_off;
       const bool ok0 = cb0 < prm.n_out;
       const bool ok1 = kMode != 0 && cb1 < prm.n_out1;
-      // First the warp's whole share of both accumulators (at most four 32-row groups)
+      // First the warp's whole share of both accumulators (kGroupsPerWarp 32-row groups)
       // into registers as bf16 pairs (rows 2i, 2i+1 of a group in pk[.][i]), and the TMEM
       // back to the MMA thread; then the slower turn through shared memory and the
       // global stores, while the next unit's MMAs already run.
       constexpr int kOuts = kMode == 0 ? 1 : 2;  // output tiles per 32-row group
-      uint32_t pk[4 * kOuts][16];
+      uint32_t pk[kGroupsPerWarp * kOuts][16];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int c = half * 32 + g * 64;
+      for (int g = 0; g < kGroupsPerWarp; ++g) {
+        const int c = part * 32 + g * 32 * kEpiParts;
         if (c < rows) {  // uniform across the warp
           __syncwarp();
           if (kMode == 0) {
@@ -417,8 +601,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_cluster(acc_empty_lead);
       }
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int c = half * 32 + g * 64;
+      for (int g = 0; g < kGroupsPerWarp; ++g) {
+        const int c = part * 32 + g * 32 * kEpiParts;
         if (c < rows) {
           const int lim = min(32, rows - c);
 #pragma unroll
@@ -500,6 +684,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (kEarly) {
+        // the unit's rows of this warp are stored: made visible at GPU scope, then counted
+        // on the slot's counter, which the signal warp waits for
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) red_release_cta_shared_add(stored + (local % kSchedSlots), 1u);
+      }
     }
   }
 
@@ -517,9 +708,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+  if (kEarly && !*abort) early_combine_drain(prm, lane, 3 * prm.timeout_ns);
 }
 
-template <int kMode, bool kAK>
+template <int kMode, bool kAK, bool kEarly = false>
 cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnParams &prm,
                         int clusters, cudaStream_t st) {
   static bool attr_set[64] = {false};
@@ -527,7 +719,7 @@ cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnP
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK>,
+    cudaError_t e = cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK, kEarly>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -539,23 +731,23 @@ cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnP
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
   lc.gridDim = dim3(2 * clusters, 1, 1);
-  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.blockDim = dim3(threads_for(kEarly), 1, 1);
   lc.dynamicSmemBytes = kSmemBytes;
   lc.stream = st;
   lc.attrs = at;
   lc.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&lc, ffn_gemm_pair_kernel<kMode, kAK>, tw, tx, prm);
+  cudaError_t e = cudaLaunchKernelEx(&lc, ffn_gemm_pair_kernel<kMode, kAK, kEarly>, tw, tx, prm);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <int kMode, bool kAK>
+template <int kMode, bool kAK, bool kEarly = false>
 int max_clusters_mode() {
   static int cached[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev] == 0) {
-    if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK>,
+    if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK, kEarly>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBytes) != cudaSuccess)
       return 0;
@@ -566,12 +758,12 @@ int max_clusters_mode() {
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
     lc.gridDim = dim3(2, 1, 1);
-    lc.blockDim = dim3(kThreads, 1, 1);
+    lc.blockDim = dim3(threads_for(kEarly), 1, 1);
     lc.dynamicSmemBytes = kSmemBytes;
     lc.attrs = at;
     lc.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, ffn_gemm_pair_kernel<kMode, kAK>, &lc) != cudaSuccess)
+    if (cudaOccupancyMaxActiveClusters(&n, ffn_gemm_pair_kernel<kMode, kAK, kEarly>, &lc) != cudaSuccess)
       return 0;
     cached[dev] = n;
   }
@@ -582,7 +774,14 @@ int max_clusters_mode() {
 
 cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
                             const CUtensorMap &tx, const FfnParams &prm, int clusters,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool early) {
+  if (early) {
+    if (mode != 1 || a_kmajor) return cudaErrorInvalidValue;
+    // the extra signal warp: as many clusters as fit with it (at most those asked for)
+    const int fit = max_clusters_mode<1, false, true>();
+    if (fit < 1) return cudaErrorInvalidConfiguration;
+    return launch_mode<1, false, true>(tw, tx, prm, clusters < fit ? clusters : fit, st);
+  }
   if (!a_kmajor)
     return mode == 0   ? launch_mode<0, false>(tw, tx, prm, clusters, st)
            : mode == 3 ? launch_mode<3, false>(tw, tx, prm, clusters, st)
@@ -591,7 +790,8 @@ cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
                    : launch_mode<1, true>(tw, tx, prm, clusters, st);
 }
 
-// All instantiations have the same block size and shared memory, hence the same count.
+// All instantiations without early combine have the same block size and shared memory,
+// hence the same count.
 int ffn_pair_max_clusters(int) { return max_clusters_mode<0, false>(); }
 
 }  // namespace moe

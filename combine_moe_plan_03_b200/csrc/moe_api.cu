@@ -61,11 +61,17 @@ int check_config(const moe_config &c) {
                                (MOE_FFN_DEFAULT == MOE_FFN_ONE_SM && c.ffn_kernel == 0)))
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(c.gate_up)) return MOE_ERR_MISALIGNED;
+  if (c.early_combine != 0 && c.early_combine != 1) return MOE_ERR_INVALID_ARG;
+  if (c.early_combine && (c.ffn_kernel == MOE_FFN_ONE_SM ||
+                          (MOE_FFN_DEFAULT == MOE_FFN_ONE_SM && c.ffn_kernel == 0)))
+    return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
+constexpr int kPlanFields = 12;
+
 // Sizes (in 4-byte words) of the plan buffers, in moe_plan_buffers field order.
-void plan_sizes(const moe_shape &s, size_t words[10]) {
+void plan_sizes(const moe_shape &s, size_t words[kPlanFields]) {
   const PlanGeom g = plan_geom(s);
   words[0] = (size_t)s.E;
   words[1] = (size_t)s.E + 1;
@@ -77,6 +83,8 @@ void plan_sizes(const moe_shape &s, size_t words[10]) {
   words[7] = (size_t)g.n_tiles;
   words[8] = plan_workspace_ints(s);
   words[9] = 4;
+  words[10] = (size_t)s.T;
+  words[11] = (size_t)s.T + 4;
 }
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
@@ -123,10 +131,10 @@ int moe_plan_arena_bytes(const moe_shape *s, size_t *bytes_out) {
   int rc = check_shape(s, false);
   if (rc != MOE_OK) return rc;
   if (bytes_out == nullptr) return MOE_ERR_INVALID_ARG;
-  size_t w[10];
+  size_t w[kPlanFields];
   plan_sizes(*s, w);
   size_t total = 0;
-  for (int i = 0; i < 10; ++i) total += round256(w[i] * 4);
+  for (int i = 0; i < kPlanFields; ++i) total += round256(w[i] * 4);
   *bytes_out = total;
   return MOE_OK;
 }
@@ -136,11 +144,11 @@ int moe_plan_bind(const moe_shape *s, void *arena, moe_plan_buffers *out) {
   if (rc != MOE_OK) return rc;
   if (arena == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(arena) & 255u) != 0) return MOE_ERR_MISALIGNED;
-  size_t w[10];
+  size_t w[kPlanFields];
   plan_sizes(*s, w);
   char *base = static_cast<char *>(arena);
-  void *ptrs[10];
-  for (int i = 0; i < 10; ++i) {
+  void *ptrs[kPlanFields];
+  for (int i = 0; i < kPlanFields; ++i) {
     ptrs[i] = base;
     base += round256(w[i] * 4);
   }
@@ -154,6 +162,8 @@ int moe_plan_bind(const moe_shape *s, void *arena, moe_plan_buffers *out) {
   out->tile_flags = static_cast<uint32_t *>(ptrs[7]);
   out->workspace = static_cast<int32_t *>(ptrs[8]);
   out->status = static_cast<int32_t *>(ptrs[9]);
+  out->tok_pending = static_cast<int32_t *>(ptrs[10]);
+  out->ready = static_cast<int32_t *>(ptrs[11]);
   return MOE_OK;
 }
 
@@ -215,9 +225,16 @@ int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, v
   if ((rc = check_plan(p)) != MOE_OK) return rc;
   if ((x == nullptr && s->T > 0) || pool == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(pool)) return MOE_ERR_MISALIGNED;
+  // a mask of MOE_DISPATCH_SIGNAL_TILES and MOE_DISPATCH_ARM_COMBINE; any other non-zero
+  // value keeps its old meaning (tile flags only)
+  int flags = signal_flags;
+  if (flags & ~(MOE_DISPATCH_SIGNAL_TILES | MOE_DISPATCH_ARM_COMBINE))
+    flags = MOE_DISPATCH_SIGNAL_TILES;
+  if ((flags & MOE_DISPATCH_ARM_COMBINE) && (!p->tok_pending || !p->ready))
+    return MOE_ERR_INVALID_ARG;
   int nsm;
   if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
-  if (launch_dispatch(*s, x, *p, pool, signal_flags != 0, nsm, static_cast<cudaStream_t>(stream)) !=
+  if (launch_dispatch(*s, x, *p, pool, flags, nsm, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
@@ -236,9 +253,34 @@ int moe_grouped_ffn(const moe_shape *s, const void *pool, const void *W1, const 
   moe_config c{};
   if (cfg != nullptr) c = *cfg;
   if ((rc = check_config(c)) != MOE_OK) return rc;
+  if (c.early_combine) return MOE_ERR_INVALID_ARG;   // moe_grouped_ffn_combine does that
   int nsm;
   if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
-  return launch_ffn(*s, pool, W1, W2, *p, act, ypool, c, nsm, static_cast<cudaStream_t>(stream));
+  return launch_ffn(*s, pool, W1, W2, *p, act, ypool, nullptr, nullptr, c, nsm,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int moe_grouped_ffn_combine(const moe_shape *s, const void *pool, const void *W1, const void *W2,
+                            const moe_plan_buffers *p, void *act, void *ypool,
+                            const float *topk_w, void *out, const moe_config *cfg,
+                            void *stream) {
+  int rc = check_shape(s, true);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (!pool || !W1 || !W2 || !act || !ypool || !p->tok_pending || !p->ready)
+    return MOE_ERR_INVALID_ARG;
+  if (s->T > 0 && (!topk_w || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned16(W1) || !aligned16(W2) || !aligned16(act) ||
+      !aligned16(ypool) || !aligned16(out))
+    return MOE_ERR_MISALIGNED;
+  moe_config c{};
+  if (cfg != nullptr) c = *cfg;
+  if ((rc = check_config(c)) != MOE_OK) return rc;
+  if (!c.early_combine) return MOE_ERR_INVALID_ARG;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  return launch_ffn(*s, pool, W1, W2, *p, act, ypool, topk_w, out, c, nsm,
+                    static_cast<cudaStream_t>(stream));
 }
 
 int moe_combine(const moe_shape *s, const void *ypool, const float *topk_w,
@@ -319,10 +361,22 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
   if ((rc = moe_plan(s, topk_idx, p, nullptr, comm)) != MOE_OK) return rc;
   if (cudaEventRecord(evp, comm) != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[1], comm) != cudaSuccess) return MOE_ERR_CUDA;
-  const int signal = (!identity && c.streaming) ? 1 : 0;
+  const bool early = !identity && c.early_combine;
+  const int signal = ((!identity && c.streaming) ? MOE_DISPATCH_SIGNAL_TILES : 0) |
+                     (early ? MOE_DISPATCH_ARM_COMBINE : 0);
   if ((rc = moe_dispatch(s, x, p, pool, signal, comm)) != MOE_OK) return rc;
   if (cudaEventRecord(evd, comm) != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[2], comm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (early) {
+    // GEMM Y combines each token as its rows complete; no separate combine launch
+    if (cudaStreamWaitEvent(comp, c.streaming ? evp : evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((rc = moe_grouped_ffn_combine(s, pool, W1, W2, p, act, ypool, topk_w, out, &c, comp)) !=
+        MOE_OK)
+      return rc;
+    if (cudaStreamWaitEvent(comp, evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (tev != nullptr && cudaEventRecord(tev[6], comp) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
   if (!identity) {
     if (cudaStreamWaitEvent(comp, c.streaming ? evp : evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
     if ((rc = moe_grouped_ffn(s, pool, W1, W2, p, act, ypool, &c, comp)) != MOE_OK) return rc;
@@ -408,6 +462,7 @@ const char *moe_strerror(int code) {
     case MOE_ERR_FLAG_TIMEOUT: return "streaming FFN timed out waiting for a pool tile";
     case MOE_ERR_POOL_OVERFLOW: return "pool rows exceeded the dropless bound";
     case MOE_ERR_PIPE_TIMEOUT: return "FFN pipeline wait timed out";
+    case MOE_ERR_COMBINE_TIMEOUT: return "early combine timed out waiting for a token's rows";
     default: return "unknown error";
   }
 }

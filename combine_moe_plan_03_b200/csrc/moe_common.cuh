@@ -36,6 +36,30 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---- plan buffers reset before every plan (its first kernel, grid-stride) ---------------
+struct PlanResets {
+  int32_t *row_src;      // [pmax] -> -1
+  int64_t pmax;
+  int32_t *tile_expert;  // [n_tiles] -> -1
+  uint32_t *flags;       // [n_tiles] -> 0
+  int64_t n_tiles;
+  int32_t *tok_pending;  // [T] -> 0 (early combine; may be null)
+  int32_t *ready;        // [T + 4] -> 0 (early combine; may be null)
+  int64_t T;
+};
+
+__device__ __forceinline__ void plan_reset_slice(const PlanResets &r, int64_t gtid, int64_t gsz) {
+  for (int64_t i = gtid; i < r.pmax; i += gsz) r.row_src[i] = -1;
+  for (int64_t i = gtid; i < r.n_tiles; i += gsz) {
+    r.tile_expert[i] = -1;
+    r.flags[i] = 0;
+  }
+  if (r.tok_pending != nullptr)
+    for (int64_t i = gtid; i < r.T; i += gsz) r.tok_pending[i] = 0;
+  if (r.ready != nullptr)
+    for (int64_t i = gtid; i < r.T + 4; i += gsz) r.ready[i] = 0;
+}
+
 // ---- global acquire / release ---------------------------------------------------------
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
   uint32_t v;
@@ -45,6 +69,37 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 
 __device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Shared-memory counter between the warps of one CTA: add with release, read with acquire.
+__device__ __forceinline__ void red_release_cta_shared_add(uint32_t *p, uint32_t v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_cta_shared(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p))
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int32_t *p, int32_t v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t ld_acquire_gpu_s32(const int32_t *p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Atomic add with acquire-release order at GPU scope; returns the old value.
+__device__ __forceinline__ int32_t atom_add_acq_rel_gpu(int32_t *p, int32_t v) {
+  int32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
 }
 
 // Order this thread's earlier generic-proxy accesses with its later async-proxy

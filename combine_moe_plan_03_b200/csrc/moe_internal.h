@@ -16,6 +16,9 @@ constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kGemmBlockM = 256;  // most live rows of one expert in one grouped-GEMM unit
 constexpr size_t kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per block (227 KB)
+// Streaming (moe_config.streaming): SMs left to the tile-ordered dispatch while GEMM A
+// claims tiles on the others.
+constexpr int kStreamDispatchSMs = 16;
 
 // Dynamic shared memory of the dispatch kernel: two staging rows of x, one row of zeros
 // (H bf16 each) and its barriers. Shapes whose rows do not fit are refused on the host.
@@ -50,6 +53,9 @@ PackGeom pack_geom(const moe_shape &s);
 cudaError_t launch_pack(const moe_shape &s, const void *W1, const void *W2, void *W1p, void *W2p,
                         int num_sms, cudaStream_t st);
 size_t plan_workspace_ints(const moe_shape &s);
+struct PlanResets;
+// What the plan's first kernel resets (row_src, tile tables, flags, early-combine counters).
+PlanResets plan_resets(const moe_shape &s, const moe_plan_buffers &p);
 
 cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_plan_buffers &p,
                         cudaStream_t st);
@@ -60,8 +66,9 @@ cudaError_t launch_plan_scan_rank(const moe_shape &s, const int32_t *topk_idx,
 cudaError_t launch_route(const moe_shape &s, const float *logits, const float *bias,
                          int32_t *topk_idx, float *topk_w, const moe_plan_buffers *p,
                          int num_sms, cudaStream_t st);
+// flags: MOE_DISPATCH_SIGNAL_TILES | MOE_DISPATCH_ARM_COMBINE
 cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_buffers &p,
-                            void *pool, int signal, int num_sms, cudaStream_t st);
+                            void *pool, int flags, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const moe_shape &s, const void *ypool, const float *topk_w,
                            const moe_plan_buffers &p, void *out, int num_sms, cudaStream_t st);
 cudaError_t launch_combine_backward(const moe_shape &s, const void *dy, const void *ypool,
@@ -80,9 +87,17 @@ int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, in
                  int num_sms, cudaStream_t st);
 cudaError_t launch_zero_pad_rows(const moe_shape &s, void *buf, int32_t width,
                                  const moe_plan_buffers &p, int num_sms, cudaStream_t st);
-// Returns MOE_OK or a MOE_ERR_* code.
+// Returns MOE_OK or a MOE_ERR_* code. With topk_w / out (cfg.early_combine) GEMM Y also
+// combines the tokens into out as their rows complete.
 int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void *W2,
-               const moe_plan_buffers &p, void *act, void *ypool, const moe_config &cfg,
-               int num_sms, cudaStream_t st);
+               const moe_plan_buffers &p, void *act, void *ypool, const float *topk_w,
+               void *out, const moe_config &cfg, int num_sms, cudaStream_t st);
+
+// Early combine: GEMM Y units of the SM-pair kernel cover 512 output columns, and both CTAs
+// of a pair count a unit's rows once each, so a token with n live pairs waits for
+// n * early_combine_arrivals(H) row counts.
+__host__ __device__ inline int32_t early_combine_arrivals(int32_t H) {
+  return 2 * ((H + 511) / 512);
+}
 
 }  // namespace moe

@@ -43,9 +43,7 @@ size_t plan_workspace_ints(const moe_shape &s) {
 __global__ void __launch_bounds__(kPlanWarps * 32)
     plan_hist_kernel(const int32_t *__restrict__ idx, int64_t pairs, int32_t E, int32_t n_chunks,
                      int32_t *__restrict__ ws, int32_t *__restrict__ done_counter,
-                     int32_t *__restrict__ row_src, int64_t pmax,
-                     int32_t *__restrict__ tile_expert, uint32_t *__restrict__ flags,
-                     int64_t n_tiles, int32_t *__restrict__ status) {
+                     const PlanResets resets, int32_t *__restrict__ status) {
   extern __shared__ int32_t hist[];  // [kPlanWarps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kPlanWarps * E; i += blockDim.x) hist[i] = 0;
@@ -71,11 +69,13 @@ __global__ void __launch_bounds__(kPlanWarps * 32)
   const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t gsz = (int64_t)gridDim.x * blockDim.x;
   if (gtid == 0) *done_counter = 0;
-  for (int64_t i = gtid; i < pmax; i += gsz) row_src[i] = -1;
-  for (int64_t i = gtid; i < n_tiles; i += gsz) {
-    tile_expert[i] = -1;
-    flags[i] = 0;
-  }
+  plan_reset_slice(resets, gtid, gsz);
+}
+
+PlanResets plan_resets(const moe_shape &s, const moe_plan_buffers &p) {
+  const PlanGeom g = plan_geom(s);
+  return PlanResets{p.row_src, g.pmax, p.tile_expert, p.tile_flags, g.n_tiles,
+                    p.tok_pending, p.ready, (int64_t)s.T};
 }
 
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
@@ -221,8 +221,7 @@ cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_p
   const int nblk = g.n_chunks > 0 ? (g.n_chunks + kPlanWarps - 1) / kPlanWarps : 0;
   const int hist_blocks = nblk > 0 ? nblk : 1;
   plan_hist_kernel<<<hist_blocks, kPlanWarps * 32, smem, st>>>(
-      topk_idx, g.pairs, s.E, g.n_chunks, p.workspace, done, p.row_src, g.pmax, p.tile_expert,
-      p.tile_flags, g.n_tiles, p.status);
+      topk_idx, g.pairs, s.E, g.n_chunks, p.workspace, done, plan_resets(s, p), p.status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   return launch_plan_scan_rank(s, topk_idx, p, st);

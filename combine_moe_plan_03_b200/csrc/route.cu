@@ -94,9 +94,7 @@ __global__ void __launch_bounds__(kPlanWarps * 32)
     route_hist_kernel(const float *__restrict__ logits, const float *__restrict__ bias,
                       int32_t T, int32_t E, int32_t k, int32_t *__restrict__ topk_idx,
                       float *__restrict__ topk_w, int32_t n_chunks, int32_t *__restrict__ ws,
-                      int32_t *__restrict__ done_counter, int32_t *__restrict__ row_src,
-                      int64_t pmax, int32_t *__restrict__ tile_expert,
-                      uint32_t *__restrict__ flags, int64_t n_tiles) {
+                      int32_t *__restrict__ done_counter, const PlanResets resets) {
   extern __shared__ int32_t hist[];  // [E] for this block's chunk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
@@ -124,11 +122,7 @@ __global__ void __launch_bounds__(kPlanWarps * 32)
   const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t gsz = (int64_t)gridDim.x * blockDim.x;
   if (gtid == 0) *done_counter = 0;
-  for (int64_t i = gtid; i < pmax; i += gsz) row_src[i] = -1;
-  for (int64_t i = gtid; i < n_tiles; i += gsz) {
-    tile_expert[i] = -1;
-    flags[i] = 0;
-  }
+  plan_reset_slice(resets, gtid, gsz);
 }
 
 template <int kPer>
@@ -150,8 +144,8 @@ static cudaError_t launch_route_t(const moe_shape &s, const float *logits, const
   int32_t *done = p->workspace + (size_t)s.E * (size_t)(g.n_chunks > 0 ? g.n_chunks : 1);
   const int nblk = g.n_chunks > 0 ? g.n_chunks : 1;
   route_hist_kernel<kPer><<<nblk, kPlanWarps * 32, smem, st>>>(
-      logits, bias, s.T, s.E, s.k, topk_idx, topk_w, g.n_chunks, p->workspace, done, p->row_src,
-      g.pmax, p->tile_expert, p->tile_flags, g.n_tiles);
+      logits, bias, s.T, s.E, s.k, topk_idx, topk_w, g.n_chunks, p->workspace, done,
+      plan_resets(s, *p));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_plan_scan_rank(s, topk_idx, *p, st);

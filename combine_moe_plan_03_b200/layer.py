@@ -19,7 +19,7 @@ def ctypes_copy(dst: ctypes.Structure, src: ctypes.Structure) -> None:
 
 
 _PLAN_FIELDS = ("counts", "offsets", "pool_row", "row_src", "tile_expert", "mblk", "meta",
-                "tile_flags", "workspace", "status")
+                "tile_flags", "workspace", "status", "tok_pending", "ready")
 
 
 class MoELayerBuffers:

@@ -75,6 +75,8 @@ extern "C" {
 #define MOE_ERR_FLAG_TIMEOUT (-11)  /* streaming FFN gave up waiting on a tile flag; aux = tile */
 #define MOE_ERR_POOL_OVERFLOW (-12) /* plan produced more rows than P_max (cannot happen for valid input) */
 #define MOE_ERR_PIPE_TIMEOUT (-13)  /* an FFN pipeline barrier wait ran out of time; aux = unit */
+#define MOE_ERR_COMBINE_TIMEOUT (-14) /* early combine gave up waiting for a token's expert rows;
+                                         aux = position in the ready queue */
 
 /* Layer shape. T tokens, hidden H, expert intermediate I, E experts, top-k,
  * pool tile rows (64 or 128). */
@@ -96,6 +98,10 @@ typedef struct moe_plan_buffers {
   uint32_t *tile_flags; /* [P_max/tile] rows landed per tile (streaming) */
   int32_t *workspace;   /* plan scratch: per-(expert, 256-pair chunk) counts + 1 counter */
   int32_t *status;      /* [4]          code, aux, 0, 0 (first device error wins) */
+  /* early combine (moe_config.early_combine); may be NULL otherwise. moe_plan zeroes both. */
+  int32_t *tok_pending; /* [T]          expert-row stores still missing per token */
+  int32_t *ready;       /* [T + 4]      queue of finished tokens (t + 1; 0 = not yet), then
+                                        its head and tail counters */
 } moe_plan_buffers;
 
 #define MOE_FFN_ONE_SM 1
@@ -127,6 +133,13 @@ typedef struct moe_config {
      act = bf16(silu(g) * u) from those bf16 values. moe_backward: g and u are read from
      there (from the forward call made with the same buffer) instead of being recomputed. */
   void *gate_up;
+  /* 1: early combine ("Per-tile streaming": combine handles a token as soon as its compute is
+     done), SM-pair kernels only. GEMM Y counts, per token, the expert rows it has stored;
+     the store that completes a token puts the token in a ready queue (p->ready), and the
+     GEMM's CTAs, once they run out of GEMM work, combine the queued tokens into out while
+     the last GEMM units still run. Needs p->tok_pending and p->ready, and moe_dispatch with
+     MOE_DISPATCH_ARM_COMBINE (moe_forward does both); out is bit-identical to moe_combine's. */
+  int32_t early_combine;
 } moe_config;
 
 /*
@@ -192,7 +205,12 @@ int moe_route_plan(const moe_shape *s, const float *logits, const float *bias, i
  * each expert's segment set to zero, and (signal_flags != 0) tile_flags[p / tile]
  * incremented with release order once row p has landed. Reads x [T, H], writes
  * pool [P_max, H] (rows >= P are not touched). Runs after moe_plan on `stream`.
+ * signal_flags is a mask of MOE_DISPATCH_SIGNAL_TILES and MOE_DISPATCH_ARM_COMBINE (any
+ * other non-zero value counts as MOE_DISPATCH_SIGNAL_TILES alone).
  */
+#define MOE_DISPATCH_SIGNAL_TILES 1  /* count landed rows in tile_flags (streaming FFN) */
+#define MOE_DISPATCH_ARM_COMBINE 2   /* set p->tok_pending for early combine, queue the tokens
+                                        that have no live pair */
 int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, void *pool,
                  int32_t signal_flags, void *stream);
 
@@ -210,6 +228,21 @@ int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, v
 int moe_grouped_ffn(const moe_shape *s, const void *pool, const void *W1, const void *W2,
                     const moe_plan_buffers *p, void *act, void *ypool, const moe_config *cfg,
                     void *stream);
+
+/*
+ * moe_grouped_ffn with the combine fused in (early combine; StreamEP README, How it works,
+ * "Per-tile streaming": combine starts on a token as soon as its compute is done). The same
+ * GEMMs A and Y, and out[t] = bf16(sum_j topk_w[t,j] * ypool[pool_row[t,j]]) exactly as
+ * moe_combine computes it (fp32 FMA chain, j ascending), each token combined by the GEMM Y
+ * kernel's CTAs as soon as its k rows are stored. Needs cfg->early_combine = 1, the SM-pair
+ * kernel, p->tok_pending / p->ready, and moe_dispatch run with MOE_DISPATCH_ARM_COMBINE
+ * after this call's moe_plan. A token whose rows never arrive (the counters were not armed)
+ * gives MOE_ERR_COMBINE_TIMEOUT in the status word after cfg->wait_timeout_us.
+ */
+int moe_grouped_ffn_combine(const moe_shape *s, const void *pool, const void *W1, const void *W2,
+                            const moe_plan_buffers *p, void *act, void *ypool,
+                            const float *topk_w, void *out, const moe_config *cfg,
+                            void *stream);
 
 /*
  * Combine (StreamEP README, How it works, "Per-tile streaming": combine of a token

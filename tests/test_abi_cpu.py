@@ -81,7 +81,7 @@ def test_ffn_kernel_constants_and_config_layout():
     fields = re.findall(r"^\s*(?:int32_t|void \*const \*|void \*)\s*(\w+);", body, re.M)
     assert fields == [f for f, _ in moe.moe_config._fields_]
     assert moe.moe_config.timing_events.offset == 24 and moe.moe_config.gate_up.offset == 32
-    assert ctypes.sizeof(moe.moe_config) == 40
+    assert moe.moe_config.early_combine.offset == 40 and ctypes.sizeof(moe.moe_config) == 48
     s = moe.moe_shape(16, 128, 128, 8, 2, 64)
     p = moe.moe_plan_bind(s, 1 << 20)
     for bad in (3, -1):
@@ -133,3 +133,55 @@ def test_gate_up_needs_the_pair_kernel_and_alignment():
         with pytest.raises(moe.MoEError) as ei:
             moe.moe_grouped_ffn(s, 1 << 20, 1 << 21, 1 << 21, p, 1 << 22, 1 << 23, cfg)
         assert ei.value.code == code
+
+
+def test_plan_struct_layout_matches_the_header():
+    """moe_plan_buffers' fields in include/moe.h, in order, are the binding's; the arena
+    gives the early-combine counters T and T + 4 ints after the status word."""
+    import combine_moe_plan_03_b200 as moe
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    body = re.search(r"typedef struct moe_plan_buffers \{(.*?)\} moe_plan_buffers;", src,
+                     re.S).group(1)
+    fields = re.findall(r"^\s*u?int32_t \*(\w+);", body, re.M)
+    assert fields == [f for f, _ in moe.moe_plan_buffers._fields_]
+    s = moe.moe_shape(1000, 128, 128, 8, 2, 64)
+    p = moe.moe_plan_bind(s, 1 << 20)
+    assert p.tok_pending - p.status == 256                       # [4] status, 256-B aligned
+    assert p.ready - p.tok_pending == (1000 * 4 + 255) // 256 * 256
+    assert moe.moe_plan_arena_bytes(s) == p.ready + (1004 * 4 + 255) // 256 * 256 - (1 << 20)
+
+
+def test_early_combine_is_refused_where_it_does_not_apply():
+    """Early combine needs the SM-pair kernel, its own entry point (moe_grouped_ffn refuses
+    it, moe_grouped_ffn_combine requires it) and the plan's counters; dispatch cannot arm
+    counters that are not there. All checked on the host."""
+    import combine_moe_plan_03_b200 as moe
+    s = moe.moe_shape(16, 128, 128, 8, 2, 64)
+    p = moe.moe_plan_bind(s, 1 << 20)
+    args = (s, 1 << 22, 1 << 23, 1 << 23, p, 1 << 24, 1 << 25)
+    cases = (
+        (lambda: moe.moe_grouped_ffn(*args, moe.moe_config(early_combine=1))),
+        (lambda: moe.moe_grouped_ffn_combine(*args, 1 << 26, 1 << 27, moe.moe_config())),
+        (lambda: moe.moe_grouped_ffn_combine(
+            *args, 1 << 26, 1 << 27, moe.moe_config(ffn_kernel=moe.MOE_FFN_ONE_SM,
+                                                    early_combine=1))),
+        (lambda: moe.moe_grouped_ffn_combine(*args, 1 << 26, 1 << 27,
+                                             moe.moe_config(early_combine=2))),
+    )
+    for c in cases:
+        with pytest.raises(moe.MoEError) as ei:
+            c()
+        assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    q = moe.moe_plan_buffers.from_buffer_copy(p)
+    q.tok_pending = None
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_grouped_ffn_combine(s, 1 << 22, 1 << 23, 1 << 23, q, 1 << 24, 1 << 25, 1 << 26,
+                                    1 << 27, moe.moe_config(early_combine=1))
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_dispatch(s, 1 << 22, q, 1 << 23, moe.MOE_DISPATCH_ARM_COMBINE)
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoEError) as ei:                      # out misaligned
+        moe.moe_grouped_ffn_combine(*args, 1 << 26, (1 << 27) + 2, moe.moe_config(early_combine=1))
+    assert ei.value.code == moe.MOE_ERR_MISALIGNED
+    assert "early combine" in moe.moe_strerror(moe.MOE_ERR_COMBINE_TIMEOUT)

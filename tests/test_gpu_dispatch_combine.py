@@ -18,15 +18,19 @@ def _layer(cfg, mb=0):
     return buf, x, idx, w, bf16_dev(x), i32_dev(idx), f32_dev(w)
 
 
-@pytest.mark.parametrize("name", ["tiny", "qwen3_235b_a22b", "dc_sweep_T4096_zipf"])
-def test_dispatch_pool_exact(name):
+@pytest.mark.parametrize("name,signal", [
+    ("tiny", 0), ("tiny", 1), ("qwen3_235b_a22b", 0), ("qwen3_235b_a22b", 1),
+    ("dc_sweep_T4096_zipf", 0), ("dc_sweep_T4096_zipf", 1), ("deepseek_v3", 1)])
+def test_dispatch_pool_exact(name, signal):
+    """signal = 0: the token-order dispatch; 1: the tile-order dispatch of the streaming
+    layer (tiles gathered through row_src in pool order, each tile's flag raised once)."""
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import bf16_host
     cfg = si.CONFIGS[name]
     buf, x, idx, w, dx, didx, dw = _layer(cfg)
     buf.pool.view(torch.int16).fill_(0x7FC0)                  # poison: NaN pattern
     moe.moe_plan(buf.shape, didx.data_ptr(), buf.plan, 0, 0)
-    moe.moe_dispatch(buf.shape, dx.data_ptr(), buf.plan, buf.pool.data_ptr(), True, 0)
+    moe.moe_dispatch(buf.shape, dx.data_ptr(), buf.plan, buf.pool.data_ptr(), signal, 0)
     torch.cuda.synchronize()
     ref = oracle.get().plan(idx, cfg.E, cfg.tile)
     P = ref["P"]
@@ -34,7 +38,7 @@ def test_dispatch_pool_exact(name):
     got = bf16_host(buf.pool[:P])
     np.testing.assert_array_equal(got, want)
     flags = buf.plan_view("tile_flags")[: P // cfg.tile].cpu().numpy().view(np.uint32)
-    assert np.all(flags == cfg.tile)                           # every tile fully landed
+    assert np.all(flags == (cfg.tile if signal else 0))       # every tile fully landed
     assert moe.moe_get_status(buf.plan)[0] == 0
     buf.close()
 

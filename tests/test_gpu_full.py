@@ -83,3 +83,36 @@ def test_dc_sweep_identity(T, routing):
     bound = 2.0 ** -8 * np.abs(ref) + cfg.k * 2.0 ** -23 * aw[:, None] * np.abs(xf) + 1e-30
     assert np.all(np.abs(got[rows] - ref) <= bound)
     buf.close()
+
+
+@pytest.mark.parametrize("name,streaming", [("deepseek_v3", 0), ("deepseek_v3", 1),
+                                            ("qwen3_235b_a22b", 0), ("decode_microbatch", 0)])
+def test_full_layer_early_combine(name, streaming):
+    """Early combine (fused into GEMM Y) at full size in the benchmark's launch configuration
+    (prepacked weights): every token's output equal to the serial combine's bit for bit, and
+    sampled tokens within the layer's tolerance of the oracle."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import assert_layer_close, bf16_dev, f32_dev, i32_dev, sample_tokens, to_f64
+    cfg = si.CONFIGS[name]
+    h1, h2, W1, W2 = _weights(cfg)
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    W1, W2 = buf.pack_weights(W1, W2)
+    W1l = [h1[e] for e in range(cfg.E)]
+    W2l = [h2[e] for e in range(cfg.E)]
+    for mb in range(cfg.micro_batches):
+        x = si.make_x(cfg, mb)
+        idx, w = si.make_routing(cfg, mb)
+        args = (bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2)
+        serial = buf.forward(*args, moe.moe_config(streaming=streaming, packed_weights=1)).clone()
+        buf.out.view(torch.int16).fill_(0x7FC0)
+        early = buf.forward(*args, moe.moe_config(streaming=streaming, packed_weights=1,
+                                                  early_combine=1))
+        torch.cuda.synchronize()
+        code, aux = moe.moe_get_status(buf.plan)
+        assert code == 0, (moe.moe_strerror(code), aux)
+        assert torch.equal(early.view(torch.int16), serial.view(torch.int16)), f"{name} mb{mb}"
+        tok = sample_tokens(cfg.T, N_SAMPLE, seed=100 + mb)
+        ref = oracle.get().moe_forward(x[tok], idx[tok], w[tok], W1l, W2l)
+        got = to_f64(early[torch.from_numpy(tok).to(early.device)])
+        assert_layer_close(got, ref, f"{name} mb{mb} early combine")
+    buf.close()

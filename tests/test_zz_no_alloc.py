@@ -71,7 +71,7 @@ def test_noalloc_plan_matches_moe_plan_two_calls_in_a_row():
 
 def test_noalloc_plan_rejects_shapes_beyond_its_scratch():
     import combine_moe_plan_03_b200 as moe
-    p = moe.moe_plan_buffers(*([1 << 20] * 10))
+    p = moe.moe_plan_buffers(*([1 << 20] * 12))
     # E=1024 experts with 1M pairs needs 1024 * 4096 + 8 ints > 2^19 + 64;
     # one 256-pair chunk past the largest accepted E=256 shape needs 256 * 2049 + 8;
     # one expert more than that shape needs 257 * 2048 + 8
