@@ -154,11 +154,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           sphase ^= 1u;
         }
         if (u < 0) break;
-        const int mb = (int)(u / prm.n_blocks);
-        const int nb = (int)(u % prm.n_blocks);
-        const int32_t row0 = prm.mblk[3 * mb + 0];
-        const int32_t e = prm.mblk[3 * mb + 1];
-        const int32_t rows = prm.mblk[3 * mb + 2];
+        int32_t mb, nb;
+        unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
+        const int32_t row0 = prm.mblk[kMblkInts * mb + 0];
+        const int32_t e = prm.mblk[kMblkInts * mb + 1];
+        const int32_t rows = prm.mblk[kMblkInts * mb + 2];
         const int nbox = (rows + kRowBox - 1) / kRowBox;
         if (kMode == 0 && prm.streaming) {
           const int32_t t_end = (row0 + rows - 1) / prm.tile;
@@ -218,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // before it counts itself done, so the last one may zero the counters for the next
       // launch, on the abort path too.
       __threadfence();
-      if (atomicAdd(prm.sched + 1, 1) == (int)gridDim.x - 1) {
+      const int group = prm.sched_group > 0 ? prm.sched_group : (int)gridDim.x;
+      if (atomicAdd(prm.sched + 1, 1) == group - 1) {
         atomicExch(prm.sched + 0, 0);
         atomicExch(prm.sched + 1, 0);
       }
@@ -241,8 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           sphase ^= 1u;
         }
         if (u < 0) break;
-        const int mb = u / prm.n_blocks;
-        const int32_t rows = prm.mblk[3 * mb + 2];
+        int32_t mb, nb;
+        unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
+        const int32_t rows = prm.mblk[kMblkInts * mb + 2];
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32_ab(kBM, n_mma, /*a_mn=*/true, /*b_mn=*/false);
         // The accumulators may be overwritten once the epilogue read the previous unit
@@ -320,10 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       if (u < 0) break;
-      const int mb = u / prm.n_blocks;
-      const int nb = u % prm.n_blocks;
-      const int32_t row0 = prm.mblk[3 * mb + 0];
-      const int32_t rows = prm.mblk[3 * mb + 2];
+      int32_t mb, nb;
+      unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
+      const int32_t row0 = prm.mblk[kMblkInts * mb + 0];
+      const int32_t rows = prm.mblk[kMblkInts * mb + 2];
       int ok = 1;
       if (lane == 0)
         ok = mbar_wait_sleepy(acc_full, local & 1u, 3 * prm.timeout_ns, abort, 1024) ? 1 : 0;
@@ -442,8 +444,14 @@ static cudaError_t launch_one(const CUtensorMap &tw, const CUtensorMap &tx, cons
 
 int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void *W2,
                const moe_plan_buffers &p, void *act, void *ypool, const float *topk_w,
-               void *out, const moe_config &cfg, int num_sms, cudaStream_t st) {
+               void *out, const moe_config &cfg, int num_sms, cudaStream_t st,
+               cudaStream_t helper_stream, cudaEvent_t helper_done) {
   const bool early = cfg.early_combine != 0;
+  // streaming with a helper stream: GEMM A runs on the SMs dispatch leaves free, and a second
+  // launch of it, queued on the helper stream behind dispatch, takes the remaining SMs'
+  // share of the same unit tickets once dispatch is done
+  const bool helper = cfg.streaming && helper_stream != nullptr && helper_done != nullptr &&
+                      cfg.ffn_ctas == 0;
   const PlanGeom g = plan_geom(s);
   if (g.pmax == 0) return MOE_OK;
   CUtensorMap tw1, tx_pool, tw2, tx_act;
@@ -466,13 +474,16 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
                               : (cfg.streaming ? num_sms - kStreamDispatchSMs : num_sms);
   if (grid < 1) grid = 1;
   int grid_y = cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms;
+  int grid_helper = helper ? num_sms - grid : 0;  // CTAs of the helper launch
   if (pair) {
     // clusters of two CTAs: as many as fit at once, at most half the requested CTAs
     const int fit0 = ffn_pair_max_clusters(0), fit1 = ffn_pair_max_clusters(1);
     if (fit0 < 1 || fit1 < 1) return MOE_ERR_CUDA;
     grid = grid / 2 < 1 ? 1 : (grid / 2 < fit0 ? grid / 2 : fit0);
     grid_y = grid_y / 2 < 1 ? 1 : (grid_y / 2 < fit1 ? grid_y / 2 : fit1);
+    grid_helper = helper ? (fit0 - grid > 0 ? fit0 - grid : 0) : 0;
   }
+  const bool use_helper = helper && grid_helper > 0;
   const uint64_t timeout_ns =
       (uint64_t)(cfg.wait_timeout_us > 0 ? cfg.wait_timeout_us : 2000000) * 1000ull;
 
@@ -516,12 +527,21 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
     a.out2 = static_cast<uint16_t *>(act);
     a.out2_ld = s.I;
   }
+  if (use_helper) a.sched_group = grid + grid_helper;  // both launches count themselves done
   cudaError_t e = pair ? launch_ffn_pair(a_mode, false, tw1, tx_pool, a, grid, st)
                        : launch_one<0>(tw1, tx_pool, a, grid, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (use_helper) {
+    e = pair ? launch_ffn_pair(a_mode, false, tw1, tx_pool, a, grid_helper, helper_stream)
+             : launch_one<0>(tw1, tx_pool, a, grid_helper, helper_stream);
+    if (e != cudaSuccess || cudaEventRecord(helper_done, helper_stream) != cudaSuccess ||
+        cudaStreamWaitEvent(st, helper_done, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
 
   FfnParams y = a;
+  y.sched_group = 0;
   y.out = static_cast<uint16_t *>(ypool);
   y.out_ld = s.H;
   y.K = s.I;

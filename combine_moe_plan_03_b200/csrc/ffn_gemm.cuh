@@ -25,6 +25,8 @@ struct FfnParams {
   int32_t tile;            // pool tile rows
   int32_t streaming;
   int32_t *sched;          // {next unit ticket, CTAs done}: zero at launch, zeroed again at exit
+  int32_t sched_group;     // clusters (pair kernel) or CTAs of all launches sharing sched;
+                           // 0 = this launch's own
   int32_t packed;          // weights are moe_pack_weights tiles (one 16 KB box per tile)
   // packed tile index = e*pk_e + nb*pk_nb + rank*pk_v + j*pk_j + kb
   // (rank = CTA of an SM pair, j = accumulator)
@@ -50,6 +52,33 @@ struct FfnParams {
   uint16_t *comb_out;
   int32_t T, k;
 };
+
+// Order of the grouped GEMMs' units. The units of one expert (its row chunks x the weight
+// column blocks) take consecutive tickets; inside them, chunks are taken kChunkBlock at a
+// time, and for each such block of chunks every column block in turn, so the units that
+// read the same weight columns start close together and share them through L2. Returns the
+// unit's chunk (index into the row-chunk table) and weight column block.
+#ifndef MOE_CHUNK_BLOCK
+#define MOE_CHUNK_BLOCK 1
+#endif
+constexpr int kChunkBlock = MOE_CHUNK_BLOCK;
+
+__device__ __forceinline__ void unit_coords(const int32_t *mblk, int32_t u, int32_t n_blocks,
+                                            int32_t &mb, int32_t &nb) {
+  if (kChunkBlock == 1) {
+    mb = u / n_blocks;
+    nb = u % n_blocks;
+    return;
+  }
+  const int32_t *m = mblk + kMblkInts * (u / n_blocks);  // a chunk of the same expert
+  const int32_t first = m[3], n_ch = m[4];
+  const int32_t local = u - n_blocks * first;
+  const int32_t b = local / (n_blocks * kChunkBlock);
+  const int32_t cb = min(kChunkBlock, n_ch - b * kChunkBlock);
+  const int32_t li = local - b * n_blocks * kChunkBlock;
+  nb = li / cb;
+  mb = first + b * kChunkBlock + li % cb;
+}
 
 // 2^x on the MUFU (ex2.approx.ftz.f32).
 __device__ __forceinline__ float ex2_approx(float x) {

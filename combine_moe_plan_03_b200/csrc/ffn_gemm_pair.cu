@@ -286,11 +286,11 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
           sphase ^= 1u;
         }
         if (u < 0) break;
-        const int mb = u / prm.n_blocks;
-        const int nb = u % prm.n_blocks;
-        const int32_t row0 = prm.mblk[3 * mb + 0];
-        const int32_t e = prm.mblk[3 * mb + 1];
-        const int32_t rows = prm.mblk[3 * mb + 2];
+        int32_t mb, nb;
+        unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
+        const int32_t row0 = prm.mblk[kMblkInts * mb + 0];
+        const int32_t e = prm.mblk[kMblkInts * mb + 1];
+        const int32_t rows = prm.mblk[kMblkInts * mb + 2];
         const int32_t half_rows = ((rows + 15) & ~15) >> 1;   // N / 2
         const int nbox = (half_rows + kRowBox - 1) / kRowBox;  // same in both CTAs
         const int32_t xrow0 = row0 + (int32_t)rank * half_rows;
@@ -360,7 +360,8 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
         // abort) before it counts itself done, so the last one may zero the counters for
         // the next launch, on the abort path too.
         __threadfence();
-        if (atomicAdd(prm.sched + 1, 1) == (int)(gridDim.x >> 1) - 1) {
+        const int group = prm.sched_group > 0 ? prm.sched_group : (int)(gridDim.x >> 1);
+        if (atomicAdd(prm.sched + 1, 1) == group - 1) {
           atomicExch(prm.sched + 0, 0);
           atomicExch(prm.sched + 1, 0);
         }
@@ -384,8 +385,9 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
           sphase ^= 1u;
         }
         if (u < 0) break;
-        const int mb = u / prm.n_blocks;
-        const int32_t rows = prm.mblk[3 * mb + 2];
+        int32_t mb, nb;
+        unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
+        const int32_t rows = prm.mblk[kMblkInts * mb + 2];
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32_ab(2 * kBM, n_mma, /*a_mn=*/!kAK, /*b_mn=*/false);
         // Both CTAs' epilogues have read the previous unit's accumulators.
@@ -486,9 +488,10 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
       }
       // every row of the unit once per CTA: the token's count drops by one (release: the
       // epilogue's stores before it; acquire: the other CTAs' stores, for the combine)
-      const int mb = u / prm.n_blocks;
-      const int32_t row0 = prm.mblk[3 * mb + 0];
-      const int32_t rows = prm.mblk[3 * mb + 2];
+      int32_t mb, nb;
+      unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
+      const int32_t row0 = prm.mblk[kMblkInts * mb + 0];
+      const int32_t rows = prm.mblk[kMblkInts * mb + 2];
       for (int r = lane; r < rows; r += 32) {
         const int32_t f = prm.row_src[row0 + r];
         if (f < 0) continue;
@@ -539,10 +542,10 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
         break;
       }
       if (u < 0) break;
-      const int mb = u / prm.n_blocks;
-      const int nb = u % prm.n_blocks;
-      const int32_t row0 = prm.mblk[3 * mb + 0];
-      const int32_t rows = prm.mblk[3 * mb + 2];
+      int32_t mb, nb;
+      unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
+      const int32_t row0 = prm.mblk[kMblkInts * mb + 0];
+      const int32_t rows = prm.mblk[kMblkInts * mb + 2];
       int ok = 1;
       if (lane == 0)
         ok = mbar_wait_parked(acc_full, local & 1u, 3 * prm.timeout_ns, abort, kParkNs) ? 1 : 0;

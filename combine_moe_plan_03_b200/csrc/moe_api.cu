@@ -78,7 +78,7 @@ void plan_sizes(const moe_shape &s, size_t words[kPlanFields]) {
   words[2] = (size_t)g.pairs;
   words[3] = (size_t)g.pmax;
   words[4] = (size_t)g.n_tiles;
-  words[5] = 3 * (size_t)g.n_tiles;
+  words[5] = kMblkInts * (size_t)g.n_tiles;
   words[6] = 8;
   words[7] = (size_t)g.n_tiles;
   words[8] = plan_workspace_ints(s);
@@ -88,6 +88,32 @@ void plan_sizes(const moe_shape &s, size_t words[kPlanFields]) {
 }
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// The grouped FFN's host checks and launch, for moe_grouped_ffn (topk_w / out NULL),
+// moe_grouped_ffn_combine (both set) and moe_forward (which may pass a helper stream and
+// event for the streaming layer's second GEMM A launch).
+int grouped_ffn_entry(const moe_shape *s, const void *pool, const void *W1, const void *W2,
+                      const moe_plan_buffers *p, void *act, void *ypool, const float *topk_w,
+                      void *out, const moe_config *cfg, bool combine, cudaStream_t st,
+                      cudaStream_t helper_stream, cudaEvent_t helper_done) {
+  int rc = check_shape(s, true);
+  if (rc != MOE_OK) return rc;
+  if ((rc = check_plan(p)) != MOE_OK) return rc;
+  if (!pool || !W1 || !W2 || !act || !ypool) return MOE_ERR_INVALID_ARG;
+  if (combine && (!p->tok_pending || !p->ready)) return MOE_ERR_INVALID_ARG;
+  if (combine && s->T > 0 && (!topk_w || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(pool) || !aligned16(W1) || !aligned16(W2) || !aligned16(act) ||
+      !aligned16(ypool) || !aligned16(out))
+    return MOE_ERR_MISALIGNED;
+  moe_config c{};
+  if (cfg != nullptr) c = *cfg;
+  if ((rc = check_config(c)) != MOE_OK) return rc;
+  if ((c.early_combine != 0) != combine) return MOE_ERR_INVALID_ARG;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  return launch_ffn(*s, pool, W1, W2, *p, act, ypool, combine ? topk_w : nullptr,
+                    combine ? out : nullptr, c, nsm, st, helper_stream, helper_done);
+}
 
 }  // namespace
 
@@ -243,44 +269,17 @@ int moe_dispatch(const moe_shape *s, const void *x, const moe_plan_buffers *p, v
 int moe_grouped_ffn(const moe_shape *s, const void *pool, const void *W1, const void *W2,
                     const moe_plan_buffers *p, void *act, void *ypool, const moe_config *cfg,
                     void *stream) {
-  int rc = check_shape(s, true);
-  if (rc != MOE_OK) return rc;
-  if ((rc = check_plan(p)) != MOE_OK) return rc;
-  if (!pool || !W1 || !W2 || !act || !ypool) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(pool) || !aligned16(W1) || !aligned16(W2) || !aligned16(act) ||
-      !aligned16(ypool))
-    return MOE_ERR_MISALIGNED;
-  moe_config c{};
-  if (cfg != nullptr) c = *cfg;
-  if ((rc = check_config(c)) != MOE_OK) return rc;
-  if (c.early_combine) return MOE_ERR_INVALID_ARG;   // moe_grouped_ffn_combine does that
-  int nsm;
-  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
-  return launch_ffn(*s, pool, W1, W2, *p, act, ypool, nullptr, nullptr, c, nsm,
-                    static_cast<cudaStream_t>(stream));
+  // early combine is moe_grouped_ffn_combine's
+  return grouped_ffn_entry(s, pool, W1, W2, p, act, ypool, nullptr, nullptr, cfg, false,
+                           static_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
 
 int moe_grouped_ffn_combine(const moe_shape *s, const void *pool, const void *W1, const void *W2,
                             const moe_plan_buffers *p, void *act, void *ypool,
                             const float *topk_w, void *out, const moe_config *cfg,
                             void *stream) {
-  int rc = check_shape(s, true);
-  if (rc != MOE_OK) return rc;
-  if ((rc = check_plan(p)) != MOE_OK) return rc;
-  if (!pool || !W1 || !W2 || !act || !ypool || !p->tok_pending || !p->ready)
-    return MOE_ERR_INVALID_ARG;
-  if (s->T > 0 && (!topk_w || !out)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(pool) || !aligned16(W1) || !aligned16(W2) || !aligned16(act) ||
-      !aligned16(ypool) || !aligned16(out))
-    return MOE_ERR_MISALIGNED;
-  moe_config c{};
-  if (cfg != nullptr) c = *cfg;
-  if ((rc = check_config(c)) != MOE_OK) return rc;
-  if (!c.early_combine) return MOE_ERR_INVALID_ARG;
-  int nsm;
-  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
-  return launch_ffn(*s, pool, W1, W2, *p, act, ypool, topk_w, out, c, nsm,
-                    static_cast<cudaStream_t>(stream));
+  return grouped_ffn_entry(s, pool, W1, W2, p, act, ypool, topk_w, out, cfg, true,
+                           static_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
 
 int moe_combine(const moe_shape *s, const void *ypool, const float *topk_w,
@@ -367,19 +366,20 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
   if ((rc = moe_dispatch(s, x, p, pool, signal, comm)) != MOE_OK) return rc;
   if (cudaEventRecord(evd, comm) != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[2], comm) != cudaSuccess) return MOE_ERR_CUDA;
-  if (early) {
-    // GEMM Y combines each token as its rows complete; no separate combine launch
+  if (!identity) {
     if (cudaStreamWaitEvent(comp, c.streaming ? evp : evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((rc = moe_grouped_ffn_combine(s, pool, W1, W2, p, act, ypool, topk_w, out, &c, comp)) !=
+    // streaming: the FFN's second GEMM A launch goes on the communicate stream behind
+    // dispatch; evp, already waited for above, is recorded again after it
+    if ((rc = grouped_ffn_entry(s, pool, W1, W2, p, act, ypool, topk_w, out, &c, early, comp,
+                                c.streaming ? comm : nullptr, c.streaming ? evp : nullptr)) !=
         MOE_OK)
       return rc;
+  }
+  if (early) {
+    // GEMM Y combined each token as its rows completed; no separate combine launch
     if (cudaStreamWaitEvent(comp, evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
     if (tev != nullptr && cudaEventRecord(tev[6], comp) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
-  }
-  if (!identity) {
-    if (cudaStreamWaitEvent(comp, c.streaming ? evp : evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((rc = moe_grouped_ffn(s, pool, W1, W2, p, act, ypool, &c, comp)) != MOE_OK) return rc;
   }
   if (cudaStreamWaitEvent(comp, evd, 0) != cudaSuccess) return MOE_ERR_CUDA;
   if (identity && tev != nullptr) {

@@ -15,6 +15,9 @@ constexpr int kPlanWarps = 8;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kGemmBlockM = 256;  // most live rows of one expert in one grouped-GEMM unit
+// GEMM row-chunk table entry: {first row, expert, live rows, expert's first chunk, expert's
+// chunk count}
+constexpr int kMblkInts = 5;
 constexpr size_t kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per block (227 KB)
 // Streaming (moe_config.streaming): SMs left to the tile-ordered dispatch while GEMM A
 // claims tiles on the others.
@@ -89,9 +92,13 @@ cudaError_t launch_zero_pad_rows(const moe_shape &s, void *buf, int32_t width,
                                  const moe_plan_buffers &p, int num_sms, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* code. With topk_w / out (cfg.early_combine) GEMM Y also
 // combines the tokens into out as their rows complete.
+// With cfg.streaming, helper_stream / helper_done (both or neither) let a second launch of
+// GEMM A, queued on helper_stream after dispatch, join the first one's unit tickets on the
+// SMs dispatch used; st waits for helper_done (recorded after it) before GEMM Y.
 int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void *W2,
                const moe_plan_buffers &p, void *act, void *ypool, const float *topk_w,
-               void *out, const moe_config &cfg, int num_sms, cudaStream_t st);
+               void *out, const moe_config &cfg, int num_sms, cudaStream_t st,
+               cudaStream_t helper_stream = nullptr, cudaEvent_t helper_done = nullptr);
 
 // Early combine: GEMM Y units of the SM-pair kernel cover 512 output columns, and both CTAs
 // of a pair count a unit's rows once each, so a token with n live pairs waits for

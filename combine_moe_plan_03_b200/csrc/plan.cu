@@ -158,10 +158,14 @@ __global__ void __launch_bounds__(256)
     offsets[x] = row;
     for (int32_t r = 0; r < pad; r += tile) tile_expert[(row + r) / tile] = x;
     const int32_t chunk = gemm_chunk_rows(c);
+    const int32_t first = blk, n_ch = c > 0 ? (c + chunk - 1) / chunk : 0;
     for (int32_t r = 0; r < c; r += chunk) {  // live rows only: padding is not computed
-      mblk[3 * blk + 0] = row + r;
-      mblk[3 * blk + 1] = x;
-      mblk[3 * blk + 2] = min(chunk, c - r);
+      int32_t *m = mblk + (int64_t)kMblkInts * blk;
+      m[0] = row + r;
+      m[1] = x;
+      m[2] = min(chunk, c - r);
+      m[3] = first;
+      m[4] = n_ch;
       ++blk;
     }
     row += pad;

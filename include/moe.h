@@ -92,7 +92,8 @@ typedef struct moe_plan_buffers {
   int32_t *pool_row;    /* [T * k]      pool row of pair f, -1 for a dropped pair */
   int32_t *row_src;     /* [P_max]      pair id of pool row p, -1 for padding */
   int32_t *tile_expert; /* [P_max/tile] expert of pool tile i, -1 past P/tile */
-  int32_t *mblk;        /* [3 * P_max/tile] GEMM row chunks: {row_start, expert, live rows <= 256} */
+  int32_t *mblk;        /* [5 * P_max/tile] GEMM row chunks: {row_start, expert, live rows <= 256,
+                                        the expert's first chunk, its number of chunks} */
   int32_t *meta;        /* [8]          num_tiles, P, number of row chunks, 0, and four
                                         grouped-GEMM unit counters (zeroed by moe_plan) */
   uint32_t *tile_flags; /* [P_max/tile] rows landed per tile (streaming) */

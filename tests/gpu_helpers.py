@@ -63,8 +63,9 @@ def check_plan_exact(buf, ref, T, k):
                                   ref["tile_expert"])
     meta = buf.plan_view("meta")[:4].cpu().numpy()
     assert meta[0] == P // buf.shape.tile and meta[1] == P
-    # GEMM row chunks: an expert's live rows in ceil(c/256) equal chunks (multiples of 16)
-    mb = buf.plan_view("mblk")[: 3 * meta[2]].cpu().numpy().reshape(-1, 3)
+    # GEMM row chunks: an expert's live rows in ceil(c/256) equal chunks (multiples of 16),
+    # each entry {first row, expert, rows, the expert's first chunk, its chunk count}
+    mb = buf.plan_view("mblk")[: 5 * meta[2]].cpu().numpy().reshape(-1, 5)
     want = []
     for e in range(E):
         a, c = int(ref["offsets"][e]), int(ref["counts"][e])
@@ -72,9 +73,10 @@ def check_plan_exact(buf, ref, T, k):
             continue
         n = -(-c // 256)
         step = (-(-c // n) + 15) // 16 * 16
+        first = len(want)
         for r in range(a, a + c, step):
-            want.append((r, e, min(step, a + c - r)))
-    np.testing.assert_array_equal(mb, np.array(want, np.int64).reshape(-1, 3))
+            want.append((r, e, min(step, a + c - r), first, -(-c // step)))
+    np.testing.assert_array_equal(mb, np.array(want, np.int64).reshape(-1, 5))
 
 
 def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:

@@ -219,9 +219,26 @@ def test_weight_gradients_small_shapes_every_expert(shape):
     buf.close()
 
 
+def _oracle_weight_grads_threaded(x, idx, w, W1e, W2e, e, dy, threads=8):
+    """The oracle's weight gradients of expert e, with the expert's tokens split into
+    `threads` contiguous slices computed at once (the oracle releases the GIL) and the
+    slices' sums added: the same products, summed in fp64 in slices."""
+    import concurrent.futures as cf
+    tok = np.nonzero((idx == e).any(1))[0]
+    parts = [p for p in np.array_split(tok, threads) if p.size]
+    orc = oracle.get()
+
+    def one(p):
+        return orc.expert_weight_grads(x[p], idx[p], w[p], W1e, W2e, e, dy[p])
+    with cf.ThreadPoolExecutor(len(parts)) as ex:
+        res = list(ex.map(one, parts))
+    return sum(r[0] for r in res), sum(r[1] for r in res)
+
+
 def test_weight_gradients_full_deepseek_two_experts():
     """The DeepSeek-V3-shaped layer at full size: dW1 and dW2 of the two experts with the
-    fewest (non-zero) rows, element by element against the oracle."""
+    fewest (non-zero) rows and of the expert with the most rows (the longest fp32
+    accumulation, up to ~2,400 rows), element by element against the oracle."""
     from gpu_helpers import to_f64
     from test_gpu_full import _weights
     cfg = si.CONFIGS["deepseek_v3"]
@@ -231,11 +248,12 @@ def test_weight_gradients_full_deepseek_two_experts():
     dy = si.make_dy(cfg)
     buf, dx, dw, (gW1, gW2) = _run(cfg, W1, W2, x, idx, w, dy, weight_grads=True)
     cnt = np.bincount(idx[idx >= 0].reshape(-1), minlength=cfg.E)
-    order = [int(e) for e in np.argsort(cnt, kind="stable") if cnt[e] > 0][:2]
-    for e in order:
-        r1, r2 = oracle.get().expert_weight_grads(x, idx, w, h1[e], h2[e], e, dy)
+    order = [int(e) for e in np.argsort(cnt, kind="stable") if cnt[e] > 0]
+    for e in order[:2] + order[-1:]:
+        r1, r2 = _oracle_weight_grads_threaded(x, idx, w, h1[e], h2[e], e, dy)
         _close(to_f64(gW1[e]), r1, f"deepseek dW1[{e}] ({cnt[e]} rows)")
         _close(to_f64(gW2[e]), r2, f"deepseek dW2[{e}] ({cnt[e]} rows)")
+    assert cnt[order[-1]] > 1000                  # the most-loaded expert: a long K loop
     buf.close()
 
 

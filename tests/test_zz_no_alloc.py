@@ -63,7 +63,7 @@ def test_noalloc_plan_matches_moe_plan_two_calls_in_a_row():
         n = {"counts": E, "offsets": E + 1, "pool_row": T * k, "row_src": ref.P_max,
              "tile_expert": ref.P_max // tile, "meta": 4, "tile_flags": ref.P_max // tile}
         for f in FIELDS:
-            m = 3 * int(a["meta"][2]) if f == "mblk" else n[f]
+            m = 5 * int(a["meta"][2]) if f == "mblk" else n[f]
             np.testing.assert_array_equal(b[f][:m], a[f][:m], err_msg=f"{case}: {f}")
         ref.close()
         got.close()
