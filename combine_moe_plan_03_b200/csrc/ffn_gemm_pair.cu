@@ -149,8 +149,11 @@ __device__ void early_combine_drain(const FfnParams &prm, int lane, uint64_t tim
       my_row = prm.pool_row[t * prm.k + lane];
       my_w = prm.topk_w[t * prm.k + lane];
     }
-    for (int c = lane; c < hv; c += 64) {
-      const int c1 = c + 32;
+    // every lane runs every iteration (the shuffles below need the whole warp); a lane's
+    // vectors past the row's end are masked
+    for (int c0 = 0; c0 < hv; c0 += 64) {
+      const int c = c0 + lane, c1 = c + 32;
+      const bool v0 = c < hv, v1 = c1 < hv;
       float a0[8], a1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.0f;
@@ -161,22 +164,24 @@ __device__ void early_combine_drain(const FfnParams &prm, int lane, uint64_t tim
         for (int jj = 0; jj < 8; ++jj) {
           rr[jj] = __shfl_sync(0xffffffffu, my_row, (j0 + jj) & 31);
           if (j0 + jj < prm.k && rr[jj] >= 0) {
-            y0[jj] = ld_cg_v4(yp + (size_t)rr[jj] * hv + c);
-            if (c1 < hv) y1[jj] = ld_cg_v4(yp + (size_t)rr[jj] * hv + c1);
+            if (v0) y0[jj] = ld_cg_v4(yp + (size_t)rr[jj] * hv + c);
+            if (v1) y1[jj] = ld_cg_v4(yp + (size_t)rr[jj] * hv + c1);
           }
         }
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const float w = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
           if (j0 + jj < prm.k && rr[jj] >= 0) {
-            fma_row8(a0, w, y0[jj]);
-            if (c1 < hv) fma_row8(a1, w, y1[jj]);
+            if (v0) fma_row8(a0, w, y0[jj]);
+            if (v1) fma_row8(a1, w, y1[jj]);
           }
         }
       }
-      op[(size_t)t * hv + c] = make_uint4(pack_bf16x2(a0[0], a0[1]), pack_bf16x2(a0[2], a0[3]),
-                                          pack_bf16x2(a0[4], a0[5]), pack_bf16x2(a0[6], a0[7]));
-      if (c1 < hv)
+      if (v0)
+        op[(size_t)t * hv + c] =
+            make_uint4(pack_bf16x2(a0[0], a0[1]), pack_bf16x2(a0[2], a0[3]),
+                       pack_bf16x2(a0[4], a0[5]), pack_bf16x2(a0[6], a0[7]));
+      if (v1)
         op[(size_t)t * hv + c1] =
             make_uint4(pack_bf16x2(a1[0], a1[1]), pack_bf16x2(a1[2], a1[3]),
                        pack_bf16x2(a1[4], a1[5]), pack_bf16x2(a1[6], a1[7]));
