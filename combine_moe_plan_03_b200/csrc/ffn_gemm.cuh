@@ -59,7 +59,7 @@ struct FfnParams {
 // read the same weight columns start close together and share them through L2. Returns the
 // unit's chunk (index into the row-chunk table) and weight column block.
 #ifndef MOE_CHUNK_BLOCK
-#define MOE_CHUNK_BLOCK 1
+#define MOE_CHUNK_BLOCK 16
 #endif
 constexpr int kChunkBlock = MOE_CHUNK_BLOCK;
 

@@ -693,9 +693,10 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
         }
       }
       if (kEarly) {
-        // the unit's rows of this warp are stored: made visible at GPU scope, then counted
-        // on the slot's counter, which the signal warp waits for
-        __threadfence();
+        // the unit's rows of this warp are stored: counted on the slot's counter (the warp
+        // barrier orders every lane's stores before lane 0's release; the signal warp's
+        // acquire of the counter and its GPU-scope release of the token's count pass them
+        // on to the combine, whose acquire reads the queue)
         __syncwarp();
         if (lane == 0) red_release_cta_shared_add(stored + (local % kSchedSlots), 1u);
       }

@@ -75,9 +75,13 @@ def test_early_combine_repeated_calls_on_one_plan_buffer():
         x = si.make_x(cfg, mb)
         idx, w = si.make_routing(cfg, mb)
         args = (bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2)
-        a = buf.forward(*args, moe.moe_config()).clone()
-        b = buf.forward(*args, moe.moe_config(early_combine=1)).clone()
+        # out is ready once the layer's compute stream reaches it: synchronise before copying
+        a = buf.forward(*args, moe.moe_config())
         torch.cuda.synchronize()
+        a = a.clone()
+        b = buf.forward(*args, moe.moe_config(early_combine=1))
+        torch.cuda.synchronize()
+        b = b.clone()
         assert torch.equal(a.view(torch.int16), b.view(torch.int16)), mb
         outs.append(b)
     assert moe.moe_get_status(buf.plan)[0] == 0

@@ -103,7 +103,9 @@ def test_full_layer_early_combine(name, streaming):
         x = si.make_x(cfg, mb)
         idx, w = si.make_routing(cfg, mb)
         args = (bf16_dev(x), i32_dev(idx), f32_dev(w), W1, W2)
-        serial = buf.forward(*args, moe.moe_config(streaming=streaming, packed_weights=1)).clone()
+        serial = buf.forward(*args, moe.moe_config(streaming=streaming, packed_weights=1))
+        torch.cuda.synchronize()               # out is the layer's compute stream's result
+        serial = serial.clone()
         buf.out.view(torch.int16).fill_(0x7FC0)
         early = buf.forward(*args, moe.moe_config(streaming=streaming, packed_weights=1,
                                                   early_combine=1))
