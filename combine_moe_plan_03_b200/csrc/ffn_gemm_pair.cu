@@ -195,10 +195,6 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
                          const __grid_constant__ CUtensorMap tm_x, const FfnParams prm) {
   static_assert(!kEarly || (kMode == 1 && !kAK), "early combine is GEMM Y's");
   constexpr int kSchedReaders = sched_readers(kEarly);
-  // GEMM Y, backward A and backward Y hand their two accumulators back one at a time (the
-  // epilogue only converts them, so it can read them in either order); GEMM A's SwiGLU
-  // needs both accumulators of an element together
-  constexpr bool kSplitRelease = kMode == 1 || kMode == 2;
   extern __shared__ uint8_t smem_raw[];
   // The same offsets in both CTAs (the MMA reads both CTAs' operands at one address).
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -208,8 +204,7 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
   uint64_t *acc_full = empty + kStages;
   uint64_t *acc_empty = acc_full + 1;
   uint64_t *drain = acc_empty + 1;
-  uint64_t *acc_empty1 = drain + 1;   // split release: accumulator 1 read (acc_empty: 0)
-  uint64_t *sched_full = acc_empty1 + 1;
+  uint64_t *sched_full = drain + 1;
   uint64_t *sched_empty = sched_full + kSchedSlots;
   int32_t *sched = reinterpret_cast<int32_t *>(sched_empty + kSchedSlots);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sched + kSchedSlots);
@@ -234,7 +229,6 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kEpiWarps);
-    mbar_init(acc_empty1, 2 * kEpiWarps);
     mbar_init(drain, 1);
     for (int i = 0; i < kSchedSlots; ++i) {
       mbar_init(sched_full + i, 1);
@@ -354,8 +348,12 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
             tma_load_2d_pair(sw1, &tm_w, fb, wcol1, krow);
             tma_load_2d_pair(sw1 + kChunkBytes, &tm_w, fb, wcol1 + 64, krow);
           }
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d_pair(sx + i * kRowBoxBytes, &tm_x, fb, kb * kBK, xrow0 + i * kRowBox);
+          for (int i = 0; i < nbox; ++i) {
+            if (prm.x_panels)
+              tma_load_3d_pair(sx + i * kRowBoxBytes, &tm_x, fb, 0, xrow0 + i * kRowBox, kb);
+            else
+              tma_load_2d_pair(sx + i * kRowBoxBytes, &tm_x, fb, kb * kBK, xrow0 + i * kRowBox);
+          }
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -421,47 +419,13 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
             if (mask & 2) tc_mma_bf16_pair(tmem_base + kAccStride, w1, xdesc, idesc, acc);
           }
         };
-        // Both CTAs' epilogues have read the previous unit's accumulator 0 (all of it
-        // unless the release is split).
+        // Both CTAs' epilogues have read the previous unit's accumulators.
         if (!mbar_wait<true>(acc_empty, (local + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
           raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
           break;
         }
         tc_fence_after();
-        int kb = 0;
-        if (kSplitRelease) {
-          // Split release: the epilogue reads accumulator 0 first and hands it back, then
-          // accumulator 1. Accumulator 0's MMAs of the unit's first stages (all that the
-          // ring holds) run while accumulator 1 is still being read; the stages are
-          // released once accumulator 1's MMAs have caught up.
-          const uint32_t s0 = stage;
-          const int lead_in = kb_count < kStages ? kb_count : kStages;
-          for (; kb < lead_in; ++kb) {
-            if (!mbar_wait(full + stage, phase, 2 * prm.timeout_ns, abort)) {
-              raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            mma_stage(stage, kb, 1);
-            if (++stage == kStages) {
-              stage = 0;
-              phase ^= 1u;
-            }
-          }
-          if (ok && !mbar_wait<true>(acc_empty1, (local + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
-            raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
-            ok = false;
-          }
-          if (!ok) break;
-          tc_fence_after();
-          for (int i = 0; i < lead_in; ++i) {
-            const uint32_t s = (s0 + (uint32_t)i) % kStages;
-            mma_stage(s, i, 2);
-            tc_commit_pair_mc(empty + s, 0x3);
-          }
-        }
-        for (; kb < kb_count; ++kb) {
+        for (int kb = 0; kb < kb_count; ++kb) {
           if (!mbar_wait(full + stage, phase, 2 * prm.timeout_ns, abort)) {
             raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
             ok = false;
@@ -613,41 +577,8 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
       // global stores, while the next unit's MMAs already run.
       constexpr int kOuts = kMode == 0 ? 1 : 2;  // output tiles per 32-row group
       uint32_t pk[kGroupsPerWarp * kOuts][16];
-      // lane 0 of the warp reports accumulator j read (split release: j = 0, 1 in turn)
-      auto release = [&](int j) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          uint64_t *b = j == 0 ? acc_empty : acc_empty1;
-          if (lead)
-            mbar_arrive(b);
-          else
-            mbar_arrive_cluster(cluster_map(smem_u32(b), 0));
-        }
-      };
-      if (kSplitRelease) {
-        // accumulator 0 of every group, handed back, then accumulator 1
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-#pragma unroll
-          for (int g = 0; g < kGroupsPerWarp; ++g) {
-            const int c = part * 32 + g * 32 * kEpiParts;
-            if (c < rows) {  // uniform across the warp
-              __syncwarp();
-              uint32_t a[32];
-              tmem_ld_32x32b_x32(tq + j * kAccStride + c, a);
-              tmem_ld_wait();
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[kOuts * g + j][i] =
-                    pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
-            }
-          }
-          release(j);
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < kGroupsPerWarp && !kSplitRelease; ++g) {
+      for (int g = 0; g < kGroupsPerWarp; ++g) {
         const int c = part * 32 + g * 32 * kEpiParts;
         if (c < rows) {  // uniform across the warp
           __syncwarp();
@@ -676,7 +607,14 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
           }
         }
       }
-      if (!kSplitRelease) release(0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (lead)
+          mbar_arrive(acc_empty);
+        else
+          mbar_arrive_cluster(cluster_map(smem_u32(acc_empty), 0));
+      }
 #pragma unroll
       for (int g = 0; g < kGroupsPerWarp; ++g) {
         const int c = part * 32 + g * 32 * kEpiParts;
@@ -705,7 +643,13 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
                   *reinterpret_cast<uint4 *>(prm.out + (size_t)(row0 + c + r) * prm.out_ld +
                                              cb + part * 8) = val;
                 } else {
-                  const size_t o = (size_t)(row0 + c + r) * prm.out_ld + cb + part * 8;
+                  const int32_t orow = row0 + c + r, ocol = cb + part * 8;
+                  const size_t o = prm.out_panel_rows > 0
+                                       ? panel_index(orow, ocol, prm.out_panel_rows)
+                                       : (size_t)orow * prm.out_ld + ocol;
+                  const size_t o1 = prm.out_panel_rows > 0
+                                        ? panel_index(orow, ocol + prm.aux_off, prm.out_panel_rows)
+                                        : o + prm.aux_off;
                   // 8 columns of one row: da from the turned block, g and u from the
                   // saved pre-activations, dg and du to the same columns of out
                   const size_t a = (size_t)(row0 + c + r) * prm.aux_ld + cb + part * 8;
@@ -728,7 +672,7 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
                   }
                   *reinterpret_cast<uint4 *>(prm.out + o) =
                       make_uint4(dgo[0], dgo[1], dgo[2], dgo[3]);
-                  *reinterpret_cast<uint4 *>(prm.out + o + prm.aux_off) =
+                  *reinterpret_cast<uint4 *>(prm.out + o1) =
                       make_uint4(duo[0], duo[1], duo[2], duo[3]);
                 }
               }
