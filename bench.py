@@ -495,8 +495,8 @@ def time_backward(moe, buf, cfg, dev, world, local, x, idx, w, W1, W2, W1u, W2u,
     code, aux = moe.moe_get_status(buf.plan)
     if code != 0:
         raise RuntimeError(f"device status after the backward: {moe.moe_strerror(code)} ({aux})")
-    names = ("combine_bwd", "recompute_gu", "gemm_y_bwd", "wgrad_w2", "gemm_a_bwd",
-             "dispatch_bwd", "wgrad_w1")
+    names = ("combine_bwd", "recompute_gu", "gemm_y_bwd", "wgrad_w2", "gemm_a_bwd", "wgrad_w1",
+             "dispatch_bwd")
     ph = {k: 0.0 for k in names}
     for c in range(steps):
         e = tev[8 * c: 8 * c + 8]

@@ -10,9 +10,7 @@
 //   dispatch, mirrored:  dx[t]     = bf16(sum_j dpool[pool_row[t,j]])  (fp32 sum, j order)
 // This file holds the combine backward; the GEMMs are the SM-pair kernel (ffn_gemm_pair.cu)
 // with the weights read K-major, and the dispatch backward is the combine kernel with unit
-// weights (combine.cu). dypool and dgu are kept in the panel layout (ffn_gemm.cuh), which
-// the backward and weight-gradient GEMMs read as contiguous boxes; act and pool are copied
-// into it (repack_panels_kernel, wgrad.cu) before their weight gradients.
+// weights (combine.cu).
 #include "ffn_gemm.cuh"
 
 namespace moe {
@@ -40,8 +38,6 @@ __device__ __forceinline__ uint4 scale_bf16x8(const uint4 &a, float w) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// dypool is written in the panel layout (64-column panels of panel_rows rows) that the
-// backward Y GEMM and the dW2 GEMM read as contiguous boxes.
 // One block of 128 threads per token (grid-stride); thread v owns the 16-byte vectors v,
 // v + 128, ... of the row. Per vector, dy is loaded once and the ypool vectors of up to 8
 // pairs are all loaded before they are used; each pair's dypool vector is stored and its
@@ -54,7 +50,7 @@ __global__ void __launch_bounds__(kCbThreads)
     combine_backward_kernel(const uint4 *__restrict__ dy, const uint4 *__restrict__ ypool,
                             const float *__restrict__ topk_w, const int32_t *__restrict__ pool_row,
                             uint4 *__restrict__ dypool, float *__restrict__ dw, int32_t T,
-                            int32_t k, int32_t hv, int64_t panel_rows) {
+                            int32_t k, int32_t hv) {
   __shared__ int32_t s_p[kMaxTopK];
   __shared__ float s_w[kMaxTopK];
   __shared__ float s_red[kCbThreads / 32][kMaxTopK];
@@ -83,9 +79,7 @@ __global__ void __launch_bounds__(kCbThreads)
           const int j = j0 + jj;
           if (j < k && s_p[j] >= 0) {
             part[jj] += dot_bf16x8(d, y[jj]);
-            // 16-byte vector v of row p: panel v / 8, piece v % 8 of the row's 128 bytes
-            dypool[((size_t)(v >> 3) * panel_rows + s_p[j]) * 8 + (v & 7)] =
-                scale_bf16x8(d, s_w[j]);
+            dypool[(size_t)s_p[j] * hv + v] = scale_bf16x8(d, s_w[j]);
           }
         }
       }
@@ -116,7 +110,7 @@ cudaError_t launch_combine_backward(const moe_shape &s, const void *dy, const vo
   if (grid > s.T) grid = s.T;
   combine_backward_kernel<<<(int)grid, kCbThreads, 0, st>>>(
       static_cast<const uint4 *>(dy), static_cast<const uint4 *>(ypool), topk_w, p.pool_row,
-      static_cast<uint4 *>(dypool), dw, s.T, s.k, s.H / 8, plan_geom(s).pmax);
+      static_cast<uint4 *>(dypool), dw, s.T, s.k, s.H / 8);
   return cudaGetLastError();
 }
 

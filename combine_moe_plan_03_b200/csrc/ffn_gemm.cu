@@ -420,20 +420,6 @@ bool make_tmap_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t ou
   return r == CUDA_SUCCESS;
 }
 
-bool make_tmap_panels(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
-                      uint32_t box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr || cols % 64 != 0) return false;
-  cuuint64_t dims[3] = {64, rows, cols / 64};
-  cuuint64_t strides[2] = {128, rows * 128};
-  cuuint32_t box[3] = {64, box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
                uint32_t box_outer) {
   return make_tmap_box(m, base, inner, outer, 64, box_outer, true);
@@ -603,7 +589,7 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
 int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
                         const moe_plan_buffers &p, const void *pool, void *act,
                         void *dypool_dpool, void *gu, void *dgu, void *dW1, void *dW2,
-                        void *dx, const moe_config &cfg, int num_sms, cudaStream_t st,
+                        const moe_config &cfg, int num_sms, cudaStream_t st,
                         cudaEvent_t const *tev) {
   const PlanGeom g = plan_geom(s);
   if (g.pmax == 0) {
@@ -614,18 +600,17 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
     if (dW2 != nullptr &&
         cudaMemsetAsync(dW2, 0, (size_t)s.E * s.I * s.H * sizeof(uint16_t), st) != cudaSuccess)
       return MOE_ERR_CUDA;
-    for (int i = 2; tev != nullptr && i <= 7; ++i)
+    for (int i = 2; tev != nullptr && i <= 6; ++i)
       if (cudaEventRecord(tev[i], st) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  // dypool (in dypool_dpool) and dgu are kept in the panel layout; dpool is row-major
   CUtensorMap tw1_mn, tw2_k, tw1_k, tx_pool, tx_dy, tx_dgu;
   if (!make_tmap(&tw1_mn, W1, 2ull * s.I, (uint64_t)s.E * s.H, kBK) ||
       !make_tmap(&tw2_k, W2, (uint64_t)s.H, (uint64_t)s.E * s.I, 128) ||
       !make_tmap(&tw1_k, W1, 2ull * s.I, (uint64_t)s.E * s.H, 128) ||
       !make_tmap(&tx_pool, pool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
-      !make_tmap_panels(&tx_dy, dypool_dpool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
-      !make_tmap_panels(&tx_dgu, dgu, 2ull * s.I, (uint64_t)g.pmax, kRowBox))
+      !make_tmap(&tx_dy, dypool_dpool, (uint64_t)s.H, (uint64_t)g.pmax, kRowBox) ||
+      !make_tmap(&tx_dgu, dgu, 2ull * s.I, (uint64_t)g.pmax, kRowBox))
     return MOE_ERR_CUDA;
   const int fit = ffn_pair_max_clusters(0);
   if (fit < 1) return MOE_ERR_CUDA;
@@ -678,18 +663,15 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   y.aux = static_cast<const uint16_t *>(gu);
   y.aux_ld = 2 * s.I;
   y.aux_off = s.I;
-  y.x_panels = 1;                    // dypool
-  y.out_panel_rows = g.pmax;         // dgu
   if (launch_ffn_pair(2, true, tw2_k, tx_dy, y, clusters, st) != cudaSuccess) return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
 
   // dW2 = act^T . dypool per expert (before backward A overwrites dypool)
   if (dW2 != nullptr) {
-    if (launch_zero_pad_rows(s, act, s.I, p, num_sms, st, false) != cudaSuccess ||
-        launch_zero_pad_rows(s, dypool_dpool, s.H, p, num_sms, st, true) != cudaSuccess)
+    if (launch_zero_pad_rows(s, act, s.I, p, num_sms, st) != cudaSuccess ||
+        launch_zero_pad_rows(s, dypool_dpool, s.H, p, num_sms, st) != cudaSuccess)
       return MOE_ERR_CUDA;
-    const int rc = launch_wgrad(s, act, s.I, false, dypool_dpool, s.H, true, dW2, p, p.meta + 6,
-                                cfg, num_sms, st);
+    const int rc = launch_wgrad(s, act, s.I, dypool_dpool, s.H, dW2, p, p.meta + 6, cfg, num_sms, st);
     if (rc != MOE_OK) return rc;
   }
   if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -706,28 +688,17 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   a.n_out1 = s.H;
   a.k_rows = s.H;
   a.sched = p.meta + 4;
-  a.x_panels = 1;                    // dgu
   if (launch_ffn_pair(1, true, tw1_k, tx_dgu, a, clusters, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
 
-  // dispatch backward: dx[t] = bf16(sum_j dpool[pool_row[t, j]]) (the combine with unit
-  // weights), before dW1 takes the dpool buffer
-  if (launch_combine(s, dypool_dpool, nullptr, p, dx, num_sms, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (tev != nullptr && cudaEventRecord(tev[6], st) != cudaSuccess) return MOE_ERR_CUDA;
-
-  // dW1 = pool^T . dgu per expert, with pool copied into the panel layout (in the dpool
-  // buffer, free now); the pool's padding rows are zero already
+  // dW1 = pool^T . dgu per expert (the pool's padding rows are zero already)
   if (dW1 != nullptr) {
-    if (launch_repack_panels(s, pool, dypool_dpool, s.H, p, num_sms, st) != cudaSuccess ||
-        launch_zero_pad_rows(s, dgu, 2 * s.I, p, num_sms, st, true) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    const int rc = launch_wgrad(s, dypool_dpool, s.H, true, dgu, 2 * s.I, true, dW1, p,
-                                p.meta + 4, cfg, num_sms, st);
+    if (launch_zero_pad_rows(s, dgu, 2 * s.I, p, num_sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+    const int rc = launch_wgrad(s, pool, s.H, dgu, 2 * s.I, dW1, p, p.meta + 4, cfg, num_sms, st);
     if (rc != MOE_OK) return rc;
   }
-  if (tev != nullptr && cudaEventRecord(tev[7], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[6], st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -51,10 +51,6 @@ struct FfnParams {
   int32_t *ready;
   uint16_t *comb_out;
   int32_t T, k;
-  // the rows operand (tm_x) in the panel layout: boxes at {0, row, k / 64}
-  int32_t x_panels;
-  // mode 2: dg | du written in the panel layout with out_panel_rows rows per panel
-  int64_t out_panel_rows;
 };
 
 // Order of the grouped GEMMs' units. The units of one expert (its row chunks x the weight
@@ -131,18 +127,6 @@ bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
 // The same with any box and no swizzle or the 128-byte one (for TMA stores, no swizzle).
 bool make_tmap_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
                    uint32_t box_inner, uint32_t box_outer, bool swizzle128);
-
-// Panel layout of a bf16 matrix [rows, cols] (cols a multiple of 64): 64-column panels, each
-// [rows, 64] row-major (128-byte rows), one after the other; element (r, c) at
-// ((c / 64) * rows + r) * 64 + c % 64. Any box of 64 columns x n rows inside a panel is
-// n * 128 contiguous bytes, read by TMA at the contiguous rate (a 64 x 64 box of a
-// row-major matrix is 64 pieces of 128 bytes at the row pitch). 3-D tensor map {64, rows,
-// cols / 64}, box {64, box_rows, 1}, 128-byte swizzle.
-bool make_tmap_panels(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
-                      uint32_t box_rows);
-__host__ __device__ inline size_t panel_index(int64_t r, int64_t c, int64_t rows) {
-  return (size_t)(((c >> 6) * rows + r) * 64 + (c & 63));
-}
 
 // Pair-kernel launch (ffn_gemm_pair.cu): grid = 2 * clusters CTAs, clusters of two.
 // mode 0: SwiGLU epilogue (GEMM A); 1: plain bf16 (GEMM Y, backward A, gate / up

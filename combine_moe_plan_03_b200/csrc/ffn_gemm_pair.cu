@@ -348,12 +348,8 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
             tma_load_2d_pair(sw1, &tm_w, fb, wcol1, krow);
             tma_load_2d_pair(sw1 + kChunkBytes, &tm_w, fb, wcol1 + 64, krow);
           }
-          for (int i = 0; i < nbox; ++i) {
-            if (prm.x_panels)
-              tma_load_3d_pair(sx + i * kRowBoxBytes, &tm_x, fb, 0, xrow0 + i * kRowBox, kb);
-            else
-              tma_load_2d_pair(sx + i * kRowBoxBytes, &tm_x, fb, kb * kBK, xrow0 + i * kRowBox);
-          }
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d_pair(sx + i * kRowBoxBytes, &tm_x, fb, kb * kBK, xrow0 + i * kRowBox);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -399,26 +395,6 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
         const int32_t rows = prm.mblk[kMblkInts * mb + 2];
         const uint32_t n_mma = (uint32_t)((rows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32_ab(2 * kBM, n_mma, /*a_mn=*/!kAK, /*b_mn=*/false);
-        // The MMAs of one k-step into accumulator j (mask bit j) from stage s.
-        auto mma_stage = [&](uint32_t s, int kb, int mask) {
-          const uint32_t sw0 = smem_u32(smem + s * kStageBytes);
-          const uint32_t sw1 = sw0 + kWTileBytes;
-          const uint32_t sx = sw0 + 2 * kWTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            // weights: MN-major, 64-column chunks kChunkBytes apart, +2048 B per 16 k;
-            // pool rows: K-major 128-byte rows, 8-row groups 1024 B apart, +32 B per 16 k
-            // (K-major weights: the same form as the pool rows)
-            const uint64_t xdesc = smem_desc_sw128(sx + kk * 32, 16, 1024);
-            const uint64_t w0 = kAK ? smem_desc_sw128(sw0 + kk * 32, 16, 1024)
-                                    : smem_desc_sw128(sw0 + kk * 2048, kChunkBytes, 1024);
-            const uint64_t w1 = kAK ? smem_desc_sw128(sw1 + kk * 32, 16, 1024)
-                                    : smem_desc_sw128(sw1 + kk * 2048, kChunkBytes, 1024);
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            if (mask & 1) tc_mma_bf16_pair(tmem_base, w0, xdesc, idesc, acc);
-            if (mask & 2) tc_mma_bf16_pair(tmem_base + kAccStride, w1, xdesc, idesc, acc);
-          }
-        };
         // Both CTAs' epilogues have read the previous unit's accumulators.
         if (!mbar_wait<true>(acc_empty, (local + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
           raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
@@ -432,7 +408,23 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
             break;
           }
           tc_fence_after();
-          mma_stage(stage, kb, 3);
+          const uint32_t sw0 = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sw1 = sw0 + kWTileBytes;
+          const uint32_t sx = sw0 + 2 * kWTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            // weights: MN-major, 64-column chunks kChunkBytes apart, +2048 B per 16 k;
+            // pool rows: K-major 128-byte rows, 8-row groups 1024 B apart, +32 B per 16 k
+            // (K-major weights: the same form as the pool rows)
+            const uint64_t xdesc = smem_desc_sw128(sx + kk * 32, 16, 1024);
+            const uint64_t w0 = kAK ? smem_desc_sw128(sw0 + kk * 32, 16, 1024)
+                                    : smem_desc_sw128(sw0 + kk * 2048, kChunkBytes, 1024);
+            const uint64_t w1 = kAK ? smem_desc_sw128(sw1 + kk * 32, 16, 1024)
+                                    : smem_desc_sw128(sw1 + kk * 2048, kChunkBytes, 1024);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            tc_mma_bf16_pair(tmem_base, w0, xdesc, idesc, acc);
+            tc_mma_bf16_pair(tmem_base + kAccStride, w1, xdesc, idesc, acc);
+          }
           tc_commit_pair_mc(empty + stage, 0x3);
           if (++stage == kStages) {
             stage = 0;
@@ -525,6 +517,7 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
     const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
     uint16_t *xp = reinterpret_cast<uint16_t *>(smem + kStages * kStageBytes + kBarrierBytes) +
                    (warp - 2) * (kXposeBytes / 2);
+    const uint32_t acc_empty_lead = cluster_map(smem_u32(acc_empty), 0);
     uint32_t local = 0;
     uint32_t sslot = 0, sphase = 0;
     for (;; ++local) {
@@ -613,7 +606,7 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
         if (lead)
           mbar_arrive(acc_empty);
         else
-          mbar_arrive_cluster(cluster_map(smem_u32(acc_empty), 0));
+          mbar_arrive_cluster(acc_empty_lead);
       }
 #pragma unroll
       for (int g = 0; g < kGroupsPerWarp; ++g) {
@@ -643,13 +636,7 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
                   *reinterpret_cast<uint4 *>(prm.out + (size_t)(row0 + c + r) * prm.out_ld +
                                              cb + part * 8) = val;
                 } else {
-                  const int32_t orow = row0 + c + r, ocol = cb + part * 8;
-                  const size_t o = prm.out_panel_rows > 0
-                                       ? panel_index(orow, ocol, prm.out_panel_rows)
-                                       : (size_t)orow * prm.out_ld + ocol;
-                  const size_t o1 = prm.out_panel_rows > 0
-                                        ? panel_index(orow, ocol + prm.aux_off, prm.out_panel_rows)
-                                        : o + prm.aux_off;
+                  const size_t o = (size_t)(row0 + c + r) * prm.out_ld + cb + part * 8;
                   // 8 columns of one row: da from the turned block, g and u from the
                   // saved pre-activations, dg and du to the same columns of out
                   const size_t a = (size_t)(row0 + c + r) * prm.aux_ld + cb + part * 8;
@@ -672,7 +659,7 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
                   }
                   *reinterpret_cast<uint4 *>(prm.out + o) =
                       make_uint4(dgo[0], dgo[1], dgo[2], dgo[3]);
-                  *reinterpret_cast<uint4 *>(prm.out + o1) =
+                  *reinterpret_cast<uint4 *>(prm.out + o + prm.aux_off) =
                       make_uint4(duo[0], duo[1], duo[2], duo[3]);
                 }
               }

@@ -325,8 +325,12 @@ int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const 
   if (launch_combine_backward(*s, dy, ypool, topk_w, *p, dpool, dw, nsm, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[1], st) != cudaSuccess) return MOE_ERR_CUDA;
-  return launch_ffn_backward(*s, W1, W2, *p, pool, act, dpool, gu, dgu, dW1, dW2, dx, c, nsm, st,
-                             tev);
+  if ((rc = launch_ffn_backward(*s, W1, W2, *p, pool, act, dpool, gu, dgu, dW1, dW2, c, nsm, st,
+                                tev)) != MOE_OK)
+    return rc;
+  if (launch_combine(*s, dpool, nullptr, *p, dx, nsm, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (tev != nullptr && cudaEventRecord(tev[7], st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, const float *topk_w,

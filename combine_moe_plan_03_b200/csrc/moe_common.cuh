@@ -304,18 +304,6 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
       : "memory");
 }
 
-// The same for a 3-D tensor map (the panel layout: x within a 64-column panel, y the row,
-// z the panel).
-__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *m,
-                                                 uint32_t bar_cluster_addr, int32_t x, int32_t y,
-                                                 int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
 // 2-D tiled store of the box at (x, y) from shared memory (bulk-group completion; x must
 // start on a 16-byte boundary, and neither coordinate may be negative).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *src, int32_t x,

@@ -78,23 +78,17 @@ cudaError_t launch_combine_backward(const moe_shape &s, const void *dy, const vo
                                     const float *topk_w, const moe_plan_buffers &p,
                                     void *dypool, float *dw, int num_sms, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* code. With dW1 / dW2 (and act) also the weight gradients.
-// Also runs the dispatch backward into dx (between backward A and dW1).
 int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
                         const moe_plan_buffers &p, const void *pool, void *act,
                         void *dypool_dpool, void *gu, void *dgu, void *dW1, void *dW2,
-                        void *dx, const moe_config &cfg, int num_sms, cudaStream_t st,
+                        const moe_config &cfg, int num_sms, cudaStream_t st,
                         cudaEvent_t const *tev);
 // wgrad.cu: D [E, M, N] = per expert A_e^T B_e over its pool segment (rows past the live
-// ones must be zero in A and B; either operand row-major or in the panel layout); the
-// kernel that zeroes those rows of a buffer; and the copy of a row-major [P, width] matrix
-// into the panel layout.
-int launch_wgrad(const moe_shape &s, const void *A, int32_t M, bool a_panels, const void *B,
-                 int32_t N, bool b_panels, void *D, const moe_plan_buffers &p, int32_t *sched,
-                 const moe_config &cfg, int num_sms, cudaStream_t st);
+// ones must be zero in A and B); and the kernel that zeroes those rows of a buffer.
+int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, int32_t N,
+                 void *D, const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg,
+                 int num_sms, cudaStream_t st);
 cudaError_t launch_zero_pad_rows(const moe_shape &s, void *buf, int32_t width,
-                                 const moe_plan_buffers &p, int num_sms, cudaStream_t st,
-                                 bool panels);
-cudaError_t launch_repack_panels(const moe_shape &s, const void *src, void *dst, int32_t width,
                                  const moe_plan_buffers &p, int num_sms, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* code. With topk_w / out (cfg.early_combine) GEMM Y also
 // combines the tokens into out as their rows complete.

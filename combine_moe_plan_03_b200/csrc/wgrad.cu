@@ -5,12 +5,6 @@
 //   D[e] [M, N] = sum over the segment's rows p of A[p, 0:M]^T (x) B[p, 0:N]
 // with A, B row-major [P_max, M] / [P_max, N] activations and D [E, M, N] bf16.
 //
-// Operands in the panel layout (ffn_gemm.cuh: 64-column panels) are read as contiguous
-// 64 x 64 boxes; a row-major operand as 64 rows of 128 bytes at its row pitch, which TMA
-// reads at about two thirds of the contiguous rate. The backward keeps dgu and dypool in
-// panels and copies pool into panels (repack_panels_kernel) before dW1; act stays
-// row-major (no free buffer of its size while dW2 runs).
-//
 // Design (tcgen05, SM pairs as in ffn_gemm_pair.cu): a work unit is (expert, 256 rows of D,
 // 256 columns of D); one cta_group::2 MMA has M = 256 (128 rows of D per CTA) and N = 256
 // (each CTA holds 128 of B's columns), K = 16; the K loop runs over the expert's rows in
@@ -63,7 +57,6 @@ struct WgradParams {
   int32_t mb_count, nb_count;  // blocks of 256 rows / columns of D
   int32_t *sched;           // {ticket, clusters done}
   uint64_t timeout_ns;
-  int32_t a_panels, b_panels;  // operand in the panel layout (3-D tensor map)
 };
 
 __device__ __forceinline__ void raise_abort_w(volatile int *abort, uint32_t peer_abort,
@@ -200,20 +193,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           }
           const int32_t r = row0 + kb * kBK;
-          if (prm.a_panels) {
-            tma_load_3d_pair(sa, &tm_a, fb, 0, r, acol >> 6);
-            tma_load_3d_pair(sa + kBoxBytes, &tm_a, fb, 0, r, (acol >> 6) + 1);
-          } else {
-            tma_load_2d_pair(sa, &tm_a, fb, acol, r);
-            tma_load_2d_pair(sa + kBoxBytes, &tm_a, fb, acol + 64, r);
-          }
-          if (prm.b_panels) {
-            tma_load_3d_pair(sb, &tm_b, fb, 0, r, bcol >> 6);
-            tma_load_3d_pair(sb + kBoxBytes, &tm_b, fb, 0, r, (bcol >> 6) + 1);
-          } else {
-            tma_load_2d_pair(sb, &tm_b, fb, bcol, r);
-            tma_load_2d_pair(sb + kBoxBytes, &tm_b, fb, bcol + 64, r);
-          }
+          tma_load_2d_pair(sa, &tm_a, fb, acol, r);
+          tma_load_2d_pair(sa + kBoxBytes, &tm_a, fb, acol + 64, r);
+          tma_load_2d_pair(sb, &tm_b, fb, bcol, r);
+          tma_load_2d_pair(sb + kBoxBytes, &tm_b, fb, bcol + 64, r);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -408,72 +391,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Rows [offsets[e] + counts[e], offsets[e] + roundup(counts[e], 64)) of a [P, width] bf16
 // buffer set to zero: the rows the weight-gradient GEMMs read past an expert's live rows.
-// Row-major (panel_rows = 0) or in the panel layout with panel_rows rows per panel. One
-// block per expert, 16-byte stores.
+// One block per expert, 16-byte stores.
 __global__ void __launch_bounds__(256)
     zero_pad_rows_kernel(uint16_t *__restrict__ buf, int32_t width, const int32_t *__restrict__ offsets,
-                         const int32_t *__restrict__ counts, int32_t E, int64_t panel_rows) {
+                         const int32_t *__restrict__ counts, int32_t E) {
   for (int e = blockIdx.x; e < E; e += gridDim.x) {
     const int32_t c = counts[e];
     const int32_t r0 = offsets[e] + c;
     const int32_t r1 = offsets[e] + ((c + kBK - 1) / kBK) * kBK;
     const int32_t vpr = width / 8;
     const int64_t n = (int64_t)(r1 - r0) * vpr;
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-      const int64_t r = r0 + i / vpr, col = (i % vpr) * 8;
-      const size_t off = panel_rows > 0 ? panel_index(r, col, panel_rows) : (size_t)r * width + col;
-      *reinterpret_cast<uint4 *>(buf + off) = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-}
-
-// Copy of the first meta[1] (= P) rows of a row-major [P_max, width] bf16 matrix into the
-// panel layout with panel_rows rows per panel: each row's 128-byte pieces go to their
-// panels. Grid-stride over 16-byte vectors, consecutive threads on consecutive vectors of a
-// row (reads coalesced; each 8 threads write one 128-byte line).
-__global__ void __launch_bounds__(256)
-    repack_panels_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int32_t width,
-                         const int32_t *__restrict__ meta, int64_t panel_rows) {
-  const int64_t vpr = width / 8;
-  const int64_t n = (int64_t)meta[1] * vpr;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / vpr, v = i % vpr;
-    dst[((v >> 3) * panel_rows + r) * 8 + (v & 7)] = src[i];
+    uint4 *base = reinterpret_cast<uint4 *>(buf + (size_t)r0 * width);
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_zero_pad_rows(const moe_shape &s, void *buf, int32_t width,
-                                 const moe_plan_buffers &p, int num_sms, cudaStream_t st,
-                                 bool panels) {
+                                 const moe_plan_buffers &p, int num_sms, cudaStream_t st) {
   const int grid = s.E < num_sms * 4 ? s.E : num_sms * 4;
   zero_pad_rows_kernel<<<grid, 256, 0, st>>>(static_cast<uint16_t *>(buf), width, p.offsets,
-                                            p.counts, s.E, panels ? plan_geom(s).pmax : 0);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_repack_panels(const moe_shape &s, const void *src, void *dst, int32_t width,
-                                 const moe_plan_buffers &p, int num_sms, cudaStream_t st) {
-  repack_panels_kernel<<<num_sms * 8, 256, 0, st>>>(static_cast<const uint4 *>(src),
-                                                     static_cast<uint4 *>(dst), width, p.meta,
-                                                     plan_geom(s).pmax);
+                                            p.counts, s.E);
   return cudaGetLastError();
 }
 
 // D [E, M, N] = per expert A_e^T B_e over the expert's segment; A [P_max, M], B [P_max, N].
-int launch_wgrad(const moe_shape &s, const void *A, int32_t M, bool a_panels, const void *B,
-                 int32_t N, bool b_panels, void *D, const moe_plan_buffers &p, int32_t *sched,
-                 const moe_config &cfg, int num_sms, cudaStream_t st) {
+int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, int32_t N,
+                 void *D, const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg,
+                 int num_sms, cudaStream_t st) {
   const PlanGeom g = plan_geom(s);
   CUtensorMap ta, tb, td;
   const uint64_t rows = g.pmax > 0 ? (uint64_t)g.pmax : 1;
-  const bool ok_a = a_panels ? make_tmap_panels(&ta, A, (uint64_t)M, rows, kBK)
-                             : make_tmap(&ta, A, (uint64_t)M, rows, kBK);
-  const bool ok_b = b_panels ? make_tmap_panels(&tb, B, (uint64_t)N, rows, kBK)
-                             : make_tmap(&tb, B, (uint64_t)N, rows, kBK);
-  if (!ok_a || !ok_b || !make_tmap_box(&td, D, (uint64_t)N, (uint64_t)s.E * M, 64, 32, true))
+  if (!make_tmap(&ta, A, (uint64_t)M, rows, kBK) || !make_tmap(&tb, B, (uint64_t)N, rows, kBK) ||
+      !make_tmap_box(&td, D, (uint64_t)N, (uint64_t)s.E * M, 64, 32, true))
     return MOE_ERR_CUDA;
   static bool attr_set[64] = {false};
   static int fit_cache[64] = {0};
@@ -516,8 +467,6 @@ int launch_wgrad(const moe_shape &s, const void *A, int32_t M, bool a_panels, co
   prm.nb_count = (N + 255) / 256;
   prm.sched = sched;
   prm.timeout_ns = (uint64_t)(cfg.wait_timeout_us > 0 ? cfg.wait_timeout_us : 2000000) * 1000ull;
-  prm.a_panels = a_panels ? 1 : 0;
-  prm.b_panels = b_panels ? 1 : 0;
   lc.gridDim = dim3(2 * clusters, 1, 1);
   lc.stream = st;
   if (cudaLaunchKernelEx(&lc, wgrad_pair_kernel, ta, tb, td, prm) != cudaSuccess)

@@ -291,13 +291,12 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
  *   dW1[e] = sum over e's rows p of pool[p]^T dgu[p]             [E, H, 2I]
  * act is the forward call's act buffer (needed for dW2; its padding rows are set to zero).
  * Work buffers (device, caller-owned, 16-byte aligned): gu and dgu [P_max, 2I] bf16,
- * dpool [P_max, H] bf16; their contents are internal (dgu, and dypool / a copy of pool in
- * dpool, are kept in a 64-column panel layout that the GEMMs read as contiguous tiles). Outputs: dx [T, H] bf16, dw [T, k] fp32, dW1, dW2 bf16. The grouped
+ * dpool [P_max, H] bf16. Outputs: dx [T, H] bf16, dw [T, k] fp32, dW1, dW2 bf16. The grouped
  * GEMMs run on SM pairs (cfg->ffn_kernel must be 0 or MOE_FFN_SM_PAIR; cfg->packed_weights
  * and cfg->streaming must be 0). cfg->timing_events, if set, holds 8 events recorded on
  * `stream`: [0] before, [1] after the combine backward, [2] after the recompute, [3] after
- * backward Y, [4] after dW2, [5] after backward A, [6] after the dispatch backward, [7] after
- * dW1.
+ * backward Y, [4] after dW2, [5] after backward A, [6] after dW1, [7] after the dispatch
+ * backward.
  */
 int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
                  const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
