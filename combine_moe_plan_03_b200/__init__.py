@@ -54,6 +54,14 @@ class moe_config(ctypes.Structure):
                 ("gate_up", ctypes.c_void_p), ("early_combine", ctypes.c_int32)]
 
 
+MOE_EP_MAX_RANKS = 8
+
+
+class moe_ep_plan(ctypes.Structure):
+    _fields_ = [("local", moe_plan_buffers)] + [(n, ctypes.c_void_p) for n in (
+        "counts", "offsets", "src_base", "tile_expert", "mblk", "meta")]
+
+
 MOE_FFN_ONE_SM = 1
 MOE_FFN_SM_PAIR = 2
 MOE_FFN_DEFAULT = MOE_FFN_SM_PAIR      # moe.h: the kernel that ffn_kernel = 0 selects
@@ -100,6 +108,15 @@ def _load():
         "moe_packed_weight_bytes": [P(moe_shape), P(ctypes.c_size_t), P(ctypes.c_size_t)],
         "moe_pack_weights": [P(moe_shape), vp, vp, vp, vp, vp],
         "moe_hbm_probe": [vp, vp, ctypes.c_size_t, i32, vp],
+        "moe_ep_local_shape": [P(moe_shape), i32, P(moe_shape)],
+        "moe_ep_pool_rows": [P(moe_shape), i32, P(ctypes.c_int64)],
+        "moe_ep_arena_bytes": [P(moe_shape), i32, P(ctypes.c_size_t)],
+        "moe_ep_bind": [P(moe_shape), i32, vp, P(moe_ep_plan)],
+        "moe_ep_layout": [P(moe_shape), i32, i32, vp, P(moe_ep_plan), vp, vp],
+        "moe_ep_dispatch": [P(moe_shape), i32, i32, vp, P(moe_plan_buffers), P(moe_ep_plan),
+                            P(vp), vp],
+        "moe_ep_combine": [P(moe_shape), i32, i32, P(vp), vp, P(moe_plan_buffers),
+                           P(moe_ep_plan), vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -121,7 +138,8 @@ EXPORTS = ["moe_route", "moe_route_plan", "moe_packed_weight_bytes", "moe_pack_w
            "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
            "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
-           "moe_hbm_probe", "moe_version"]
+           "moe_hbm_probe", "moe_ep_local_shape", "moe_ep_pool_rows", "moe_ep_arena_bytes",
+           "moe_ep_bind", "moe_ep_layout", "moe_ep_dispatch", "moe_ep_combine", "moe_version"]
 
 
 def lib():
@@ -165,6 +183,62 @@ def moe_hbm_probe(dst_ptr: int, src_ptr: int, nbytes: int, mode: int, stream: in
     over nbytes of device memory: the HBM rates the layer's copy kernels are compared with."""
     _check("moe_hbm_probe", _lib.moe_hbm_probe(dst_ptr, src_ptr or None, nbytes, mode,
                                                stream or None))
+
+
+# ---- expert parallelism inside one node (R ranks; shapes are per rank) --------------------
+
+def moe_ep_local_shape(shape, R: int) -> moe_shape:
+    out = moe_shape()
+    _check("moe_ep_local_shape", _lib.moe_ep_local_shape(ctypes.byref(_shape(shape)), R,
+                                                         ctypes.byref(out)))
+    return out
+
+
+def moe_ep_pool_rows(shape, R: int) -> int:
+    out = ctypes.c_int64(0)
+    _check("moe_ep_pool_rows", _lib.moe_ep_pool_rows(ctypes.byref(_shape(shape)), R,
+                                                     ctypes.byref(out)))
+    return int(out.value)
+
+
+def moe_ep_arena_bytes(shape, R: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moe_ep_arena_bytes", _lib.moe_ep_arena_bytes(ctypes.byref(_shape(shape)), R,
+                                                         ctypes.byref(out)))
+    return int(out.value)
+
+
+def moe_ep_bind(shape, R: int, arena_ptr: int) -> moe_ep_plan:
+    out = moe_ep_plan()
+    _check("moe_ep_bind", _lib.moe_ep_bind(ctypes.byref(_shape(shape)), R, arena_ptr,
+                                           ctypes.byref(out)))
+    return out
+
+
+def _ptr_array(ptrs):
+    return (ctypes.c_void_p * len(ptrs))(*ptrs)
+
+
+def moe_ep_layout(shape, R: int, rank: int, all_counts_ptr: int, ep: moe_ep_plan,
+                  pool_ptr: int, stream: int = 0) -> None:
+    _check("moe_ep_layout", _lib.moe_ep_layout(ctypes.byref(_shape(shape)), R, rank,
+                                               all_counts_ptr, ctypes.byref(ep), pool_ptr,
+                                               stream or None))
+
+
+def moe_ep_dispatch(shape, R: int, rank: int, x_ptr: int, own: moe_plan_buffers,
+                    ep: moe_ep_plan, pool_ptrs, stream: int = 0) -> None:
+    _check("moe_ep_dispatch", _lib.moe_ep_dispatch(ctypes.byref(_shape(shape)), R, rank, x_ptr,
+                                                   ctypes.byref(own), ctypes.byref(ep),
+                                                   _ptr_array(pool_ptrs), stream or None))
+
+
+def moe_ep_combine(shape, R: int, rank: int, ypool_ptrs, topk_w_ptr: int,
+                   own: moe_plan_buffers, ep: moe_ep_plan, out_ptr: int, stream: int = 0) -> None:
+    _check("moe_ep_combine", _lib.moe_ep_combine(ctypes.byref(_shape(shape)), R, rank,
+                                                 _ptr_array(ypool_ptrs), topk_w_ptr,
+                                                 ctypes.byref(own), ctypes.byref(ep), out_ptr,
+                                                 stream or None))
 
 
 def moe_pool_rows_max(shape) -> int:

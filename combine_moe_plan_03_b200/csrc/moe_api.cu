@@ -89,6 +89,32 @@ void plan_sizes(const moe_shape &s, size_t words[kPlanFields]) {
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
+// Expert parallelism: rank shape checks, and the EP plan arena (the all-expert prefix, then
+// the rank's pool plan, whose scratch must also hold the per-source counts of its experts).
+int check_ep(const moe_shape *s, int32_t R) {
+  int rc = check_shape(s, false);
+  if (rc != MOE_OK) return rc;
+  if (R < 1 || R > kMaxEpRanks || s->E % R != 0) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)s->T * R > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  const moe_shape g = ep_global_shape(*s, R);
+  return check_shape(&g, false);
+}
+
+constexpr int kEpFields = 6;
+void ep_sizes(const moe_shape &s, int32_t R, size_t words[kEpFields + kPlanFields]) {
+  const moe_shape g = ep_global_shape(s, R), l = ep_local_shape(s, R);
+  const PlanGeom gg = plan_geom(g);
+  words[0] = (size_t)s.E;
+  words[1] = (size_t)s.E + 1;
+  words[2] = (size_t)s.E * R + 8;
+  words[3] = (size_t)gg.n_tiles;
+  words[4] = kMblkInts * (size_t)gg.n_tiles;
+  words[5] = 8;
+  plan_sizes(l, words + kEpFields);
+  const size_t need = (size_t)(s.E / R) * R + 8;
+  if (words[kEpFields + 8] < need) words[kEpFields + 8] = need;
+}
+
 // The grouped FFN's host checks and launch, for moe_grouped_ffn (topk_w / out NULL),
 // moe_grouped_ffn_combine (both set) and moe_forward (which may pass a helper stream and
 // event for the streaming layer's second GEMM A launch).
@@ -467,6 +493,135 @@ const char *moe_strerror(int code) {
   }
 }
 
-const char *moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+int moe_ep_local_shape(const moe_shape *s, int32_t R, moe_shape *out) {
+  int rc = check_ep(s, R);
+  if (rc != MOE_OK) return rc;
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = ep_local_shape(*s, R);
+  return MOE_OK;
+}
+
+int moe_ep_pool_rows(const moe_shape *s, int32_t R, int64_t *rows_out) {
+  int rc = check_ep(s, R);
+  if (rc != MOE_OK) return rc;
+  if (rows_out == nullptr) return MOE_ERR_INVALID_ARG;
+  *rows_out = plan_geom(ep_local_shape(*s, R)).pmax;
+  return MOE_OK;
+}
+
+int moe_ep_arena_bytes(const moe_shape *s, int32_t R, size_t *bytes_out) {
+  int rc = check_ep(s, R);
+  if (rc != MOE_OK) return rc;
+  if (bytes_out == nullptr) return MOE_ERR_INVALID_ARG;
+  size_t w[kEpFields + kPlanFields];
+  ep_sizes(*s, R, w);
+  size_t total = 0;
+  for (int i = 0; i < kEpFields + kPlanFields; ++i) total += round256(w[i] * 4);
+  *bytes_out = total;
+  return MOE_OK;
+}
+
+int moe_ep_bind(const moe_shape *s, int32_t R, void *arena, moe_ep_plan *out) {
+  int rc = check_ep(s, R);
+  if (rc != MOE_OK) return rc;
+  if (arena == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(arena) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  size_t w[kEpFields + kPlanFields];
+  ep_sizes(*s, R, w);
+  char *base = static_cast<char *>(arena);
+  int32_t *ptrs[kEpFields + kPlanFields];
+  for (int i = 0; i < kEpFields + kPlanFields; ++i) {
+    ptrs[i] = reinterpret_cast<int32_t *>(base);
+    base += round256(w[i] * 4);
+  }
+  out->counts = ptrs[0];
+  out->offsets = ptrs[1];
+  out->src_base = ptrs[2];
+  out->tile_expert = ptrs[3];
+  out->mblk = ptrs[4];
+  out->meta = ptrs[5];
+  int32_t *const *q = ptrs + kEpFields;
+  moe_plan_buffers &l = out->local;
+  l.counts = q[0];
+  l.offsets = q[1];
+  l.pool_row = q[2];
+  l.row_src = q[3];
+  l.tile_expert = q[4];
+  l.mblk = q[5];
+  l.meta = q[6];
+  l.tile_flags = reinterpret_cast<uint32_t *>(q[7]);
+  l.workspace = q[8];
+  l.status = q[9];
+  l.tok_pending = q[10];
+  l.ready = q[11];
+  return MOE_OK;
+}
+
+int moe_ep_layout(const moe_shape *s, int32_t R, int32_t rank, const int32_t *all_counts,
+                  const moe_ep_plan *ep, void *pool, void *stream) {
+  int rc = check_ep(s, R);
+  if (rc != MOE_OK) return rc;
+  if (rank < 0 || rank >= R || all_counts == nullptr || ep == nullptr || pool == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((rc = check_plan(&ep->local)) != MOE_OK) return rc;
+  if (!ep->counts || !ep->offsets || !ep->src_base || !ep->tile_expert || !ep->mblk || !ep->meta)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(pool)) return MOE_ERR_MISALIGNED;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  if (launch_ep_layout(*s, R, rank, all_counts, *ep, pool, nsm,
+                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+namespace {
+int check_ep_call(const moe_shape *s, int32_t R, int32_t rank, const moe_plan_buffers *own,
+                  const moe_ep_plan *ep, void *const *peers) {
+  int rc = check_ep(s, R);
+  if (rc != MOE_OK) return rc;
+  if (rank < 0 || rank >= R || own == nullptr || ep == nullptr || peers == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((rc = check_plan(own)) != MOE_OK) return rc;
+  if (!ep->offsets || !ep->src_base) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < R; ++i) {
+    if (peers[i] == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(peers[i])) return MOE_ERR_MISALIGNED;
+  }
+  return MOE_OK;
+}
+}  // namespace
+
+int moe_ep_dispatch(const moe_shape *s, int32_t R, int32_t rank, const void *x,
+                    const moe_plan_buffers *own, const moe_ep_plan *ep, void *const *pools,
+                    void *stream) {
+  int rc = check_ep_call(s, R, rank, own, ep, pools);
+  if (rc != MOE_OK) return rc;
+  if (x == nullptr && s->T > 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x)) return MOE_ERR_MISALIGNED;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  if (launch_ep_dispatch(*s, R, rank, x, *own, *ep, pools, nsm,
+                         static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_ep_combine(const moe_shape *s, int32_t R, int32_t rank, void *const *ypools,
+                   const float *topk_w, const moe_plan_buffers *own, const moe_ep_plan *ep,
+                   void *out, void *stream) {
+  int rc = check_ep_call(s, R, rank, own, ep, ypools);
+  if (rc != MOE_OK) return rc;
+  if (s->T > 0 && (topk_w == nullptr || out == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out)) return MOE_ERR_MISALIGNED;
+  int nsm;
+  if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
+  if (launch_ep_combine(*s, R, rank, ypools, topk_w, *own, *ep, out, nsm,
+                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+const char *moe_version(void) { return "moe-b200 0.2 (sm_100a)"; }
 
 }  // extern "C"

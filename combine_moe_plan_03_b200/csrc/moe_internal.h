@@ -19,6 +19,17 @@ constexpr int kGemmBlockM = 256;  // most live rows of one expert in one grouped
 // chunk count}
 constexpr int kMblkInts = 5;
 constexpr size_t kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per block (227 KB)
+constexpr int kMaxEpRanks = MOE_EP_MAX_RANKS;  // expert-parallel ranks (GPUs of one node)
+
+// Expert parallelism: the shapes of the plan over all ranks' pairs (E global experts) and of
+// one rank's pool (its E / R experts), for R ranks of T tokens each.
+inline moe_shape ep_global_shape(const moe_shape &s, int32_t R) {
+  return moe_shape{s.T * R, s.H, s.I, s.E, s.k, s.tile};
+}
+inline moe_shape ep_local_shape(const moe_shape &s, int32_t R) {
+  return moe_shape{s.T * R, s.H, s.I, s.E / R, s.k, s.tile};
+}
+
 // Streaming (moe_config.streaming): SMs left to the tile-ordered dispatch while GEMM A
 // claims tiles on the others.
 constexpr int kStreamDispatchSMs = 16;
@@ -62,6 +73,23 @@ PlanResets plan_resets(const moe_shape &s, const moe_plan_buffers &p);
 
 cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_plan_buffers &p,
                         cudaStream_t st);
+// The plan's per-expert scan over n_src sources (ws [E][n_src] of counts, scanned in place;
+// *done zero) and the tables it builds: counts, offsets, tile table, row-chunk table, meta.
+cudaError_t launch_plan_scan_only(const moe_shape &s, int32_t n_src, int32_t *ws, int32_t *done,
+                                  int32_t *counts, int32_t *offsets, int32_t *tile_expert,
+                                  int32_t *mblk, int32_t *meta, int32_t *status, cudaStream_t st);
+// ep.cu: expert parallelism (layout from all ranks' counts, dispatch into the owners' pools,
+// combine from the owners' ypools).
+cudaError_t launch_ep_layout(const moe_shape &rank_shape, int32_t R, int32_t rank,
+                             const int32_t *C, const moe_ep_plan &ep, void *pool,
+                             int num_sms, cudaStream_t st);
+cudaError_t launch_ep_dispatch(const moe_shape &rank_shape, int32_t R, int32_t rank,
+                               const void *x, const moe_plan_buffers &own, const moe_ep_plan &ep,
+                               void *const *pools, int num_sms, cudaStream_t st);
+cudaError_t launch_ep_combine(const moe_shape &rank_shape, int32_t R, int32_t rank,
+                              void *const *ypools, const float *topk_w,
+                              const moe_plan_buffers &own, const moe_ep_plan &ep, void *out,
+                              int num_sms, cudaStream_t st);
 // The plan's second and third launches (per-expert scan + tables, stable rank), after
 // ws[e][chunk] holds the per-chunk counts (written by plan_hist_kernel or the router).
 cudaError_t launch_plan_scan_rank(const moe_shape &s, const int32_t *topk_idx,

@@ -141,16 +141,37 @@ __global__ void __launch_bounds__(256)
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int e0 = threadIdx.x * per;
   const int e1 = min(E, e0 + per);
-  int32_t my_rows = 0, my_blk = 0;
+  __shared__ unsigned long long s_rows;
+  if (threadIdx.x == 0) s_rows = 0;
+  __syncthreads();
+  int64_t rows64 = 0;
+  int32_t my_blk = 0;
   for (int x = e0; x < e1; ++x) {
     const int32_t c = __ldcg(counts + x);
-    const int32_t pad = (c + tile - 1) / tile * tile;
-    my_rows += pad;
+    rows64 += ((int64_t)c + tile - 1) / tile * tile;
     const int32_t chunk = gemm_chunk_rows(c);
     if (c > 0) my_blk += (c + chunk - 1) / chunk;
   }
+  atomicAdd(&s_rows, (unsigned long long)rows64);
+  __syncthreads();
+  // Counts beyond the dropless bound (only counts passed in by a caller, as in expert
+  // parallelism, can do this): leave an empty plan, whose tables fit any arena, and report.
+  if (s_rows > (unsigned long long)pmax) {
+    for (int x = e0; x < e1; ++x) {
+      counts[x] = 0;
+      offsets[x] = 0;
+    }
+    if (threadIdx.x == 0) {
+      offsets[E] = 0;
+      for (int i = 0; i < 8; ++i) meta[i] = 0;
+      report(status, MOE_ERR_POOL_OVERFLOW,
+             s_rows > (unsigned long long)INT32_MAX ? INT32_MAX : (int32_t)s_rows);
+    }
+    return;
+  }
+  // the total is at most pmax (< 2^31), so the int32 scans below cannot overflow
   int32_t tot_rows, tot_blk;
-  int32_t row = block_excl_scan(my_rows, warp_sums, &tot_rows);
+  int32_t row = block_excl_scan((int32_t)rows64, warp_sums, &tot_rows);
   int32_t blk = block_excl_scan(my_blk, warp_sums, &tot_blk);
   for (int x = e0; x < e1; ++x) {
     const int32_t c = __ldcg(counts + x);
@@ -177,7 +198,6 @@ __global__ void __launch_bounds__(256)
     meta[2] = tot_blk;
     meta[3] = 0;
     for (int i = 4; i < 8; ++i) meta[i] = 0;  // grouped-GEMM unit counters
-    if ((int64_t)tot_rows > pmax) report(status, MOE_ERR_POOL_OVERFLOW, tot_rows);
   }
 }
 
@@ -229,6 +249,14 @@ cudaError_t launch_plan(const moe_shape &s, const int32_t *topk_idx, const moe_p
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   return launch_plan_scan_rank(s, topk_idx, p, st);
+}
+
+cudaError_t launch_plan_scan_only(const moe_shape &s, int32_t n_src, int32_t *ws, int32_t *done,
+                                  int32_t *counts, int32_t *offsets, int32_t *tile_expert,
+                                  int32_t *mblk, int32_t *meta, int32_t *status, cudaStream_t st) {
+  plan_scan_kernel<<<s.E, 256, 0, st>>>(ws, n_src, s.E, s.tile, done, counts, offsets,
+                                         tile_expert, mblk, meta, plan_geom(s).pmax, status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_plan_scan_rank(const moe_shape &s, const int32_t *topk_idx,

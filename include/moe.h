@@ -367,6 +367,72 @@ int moe_plan_noalloc(const moe_shape *s, const int32_t *topk_idx, const moe_plan
  */
 int moe_hbm_probe(void *dst, const void *src, size_t bytes, int32_t mode, void *stream);
 
+/*
+ * Expert parallelism inside one node (StreamEP README: dispatch and combine "intranode over
+ * NVLink"; "Pool-layout dispatch"). R ranks (one per GPU, R <= MOE_EP_MAX_RANKS, E a
+ * multiple of R); rank d owns experts [d E/R, (d+1) E/R). Shapes below are per rank:
+ * rank_shape = {T tokens of this rank, H, I, E global experts, k, tile}. A layer call on
+ * rank r:
+ *   1. moe_plan(rank_shape, topk_idx, own)        this rank's pairs over the E experts
+ *   2. all-gather own.counts ([E] int32) over the ranks into all_counts [R][E] (device; by the
+ *      caller, e.g. one NCCL all-gather); it orders this step after every rank's previous
+ *      use of its pool
+ *   3. moe_ep_layout(rank_shape, R, r, all_counts, ep, pool)   every rank's pool layout, this
+ *      rank's pool plan (ep->local) and zero padding rows
+ *   4. moe_ep_dispatch(..., pools)                 x rows into their owners' pools
+ *   5. a barrier over the ranks (every rank's dispatch done)
+ *   6. moe_grouped_ffn(local_shape, pool, W1 / W2 of this rank's experts, &ep->local, ...)
+ *      with local_shape from moe_ep_local_shape (T = R * rank T, E = E / R)
+ *   7. a barrier (every rank's FFN done)
+ *   8. moe_ep_combine(..., ypools, topk_w, own, ep, out)   out[t] from the owners' ypools
+ * The pool of rank d holds the rows of d's experts from rank 0's pairs, then rank 1's, ...,
+ * each in flat pair order, padded per expert to the tile: the part of one dropless pool over
+ * all ranks' pairs that holds d's experts. pools / ypools: host arrays of R device pointers
+ * (every rank's pool [moe_ep_pool_rows, H] / ypool, mapped for peer access); x rows are
+ * stored into peers' pools and ypool rows loaded from peers' ypools with plain 16-byte
+ * accesses. No collective is issued by the library.
+ */
+#define MOE_EP_MAX_RANKS 8
+typedef struct moe_ep_plan {
+  moe_plan_buffers local; /* this rank's pool: the grouped FFN's plan (local shape) */
+  int32_t *counts;        /* [E]       pairs of all ranks per expert */
+  int32_t *offsets;       /* [E + 1]   padded prefix over all experts (rank d's pool starts at
+                                       offsets[d E / R]) */
+  int32_t *src_base;      /* [E * R + 8] rows of expert e from ranks before s: [e * R + s] */
+  int32_t *tile_expert;   /* tile and row-chunk tables and meta of the all-expert prefix */
+  int32_t *mblk;
+  int32_t *meta;
+} moe_ep_plan;
+
+/* Local shape {R * T, H, I, E / R, k, tile} of a rank's pool; pool rows (dropless bound for
+ * all ranks' pairs on E / R experts); bytes of the EP plan arena; binding the arena. */
+int moe_ep_local_shape(const moe_shape *rank_shape, int32_t R, moe_shape *out);
+int moe_ep_pool_rows(const moe_shape *rank_shape, int32_t R, int64_t *rows_out);
+int moe_ep_arena_bytes(const moe_shape *rank_shape, int32_t R, size_t *bytes_out);
+int moe_ep_bind(const moe_shape *rank_shape, int32_t R, void *arena, moe_ep_plan *out);
+
+/* Step 3: from all_counts [R][E] (device int32), the layout of every rank's pool, this rank's
+ * pool plan ep->local (reset and built; its status word is the layer's) and zeroed padding
+ * rows in this rank's pool. A count outside [0, T k], or totals beyond the pool, give
+ * MOE_ERR_POOL_OVERFLOW in ep->local's status word and an empty pool plan. */
+int moe_ep_layout(const moe_shape *rank_shape, int32_t R, int32_t rank,
+                  const int32_t *all_counts, const moe_ep_plan *ep, void *pool, void *stream);
+
+/* Step 4: pool_{owner(e)}[row of pair f] = x[t] for every live pair f = t*k + j of this rank
+ * (own: this rank's moe_plan). This rank's row of all_counts must equal own's counts, else
+ * MOE_ERR_POOL_OVERFLOW (aux = expert) in own's status word. A row that all_counts would
+ * place outside the owner's pool is skipped and reported the same way (aux = pair id);
+ * moe_ep_combine checks rows the same way. */
+int moe_ep_dispatch(const moe_shape *rank_shape, int32_t R, int32_t rank, const void *x,
+                    const moe_plan_buffers *own, const moe_ep_plan *ep, void *const *pools,
+                    void *stream);
+
+/* Step 8: out[t] = bf16(sum_j topk_w[t,j] * ypool_{owner}[row of pair t*k + j]), fp32 FMA
+ * chain over j ascending (moe_combine's arithmetic); dropped pairs add nothing. */
+int moe_ep_combine(const moe_shape *rank_shape, int32_t R, int32_t rank, void *const *ypools,
+                   const float *topk_w, const moe_plan_buffers *own, const moe_ep_plan *ep,
+                   void *out, void *stream);
+
 /* Library version string. */
 const char *moe_version(void);
 

@@ -1,0 +1,195 @@
+"""Expert parallelism inside one node (StreamEP README: dispatch and combine intranode over
+NVLink), with R ranks emulated on one GPU: every rank's buffers live on the same device and
+the "peer" pointers are plain pointers, which is what the kernels see on several GPUs too.
+Each rank's pool must be bit for bit the part of one dropless pool over all ranks' pairs
+that holds the rank's experts, and each rank's output must be bit for bit the single-GPU
+layer's output for its tokens (the GEMMs compute each row independently of the others in
+its chunk, and combine keeps the same FMA chain), and within the layer's tolerance of the
+oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_ep(cfg, R, drop=0.0, check_pools=True):
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import DEV, bf16_dev, bf16_host, f32_dev, i32_dev, weights_dev
+    W1, W2 = weights_dev(cfg)
+    rs = moe.moe_shape(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    ls = moe.moe_ep_local_shape(rs, R)
+    Er = cfg.E // R
+    rows = moe.moe_ep_pool_rows(rs, R)
+    xs, idxs, ws = [], [], []
+    for r in range(R):
+        x = si.make_x(cfg, r)
+        idx, w = si.make_routing(cfg, r)
+        if drop > 0:
+            idx = idx.copy()
+            idx[np.random.default_rng(r).random(idx.shape) < drop] = -1
+        xs.append(x), idxs.append(idx), ws.append(w)
+    own = [moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile, identity=True)
+           for _ in range(R)]
+    ep_arena = [torch.zeros(moe.moe_ep_arena_bytes(rs, R), dtype=torch.uint8, device=DEV)
+                for _ in range(R)]
+    ep = [moe.moe_ep_bind(rs, R, a.data_ptr()) for a in ep_arena]
+    pools = [torch.full((rows, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+             for _ in range(R)]
+    acts = [torch.empty((rows, cfg.I), dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    ypools = [torch.empty((rows, cfg.H), dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    outs = [torch.full((cfg.T, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+            for _ in range(R)]
+    dx = [bf16_dev(x) for x in xs]
+    dw = [f32_dev(w) for w in ws]
+    # 1. each rank's own plan over the E global experts
+    for r in range(R):
+        moe.moe_plan(rs, i32_dev(idxs[r]).data_ptr(), own[r].plan, 0, 0)
+    # 2. the all-gather of the counts (here: stacking the ranks' rows)
+    C = torch.stack([own[r].plan_view("counts")[: cfg.E] for r in range(R)]).contiguous()
+    pool_ptrs = [p.data_ptr() for p in pools]
+    ypool_ptrs = [p.data_ptr() for p in ypools]
+    # 3.-8. layout, dispatch into the owners' pools, each rank's FFN, combine from the owners
+    for r in range(R):
+        moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pools[r].data_ptr(), 0)
+    for r in range(R):
+        moe.moe_ep_dispatch(rs, R, r, dx[r].data_ptr(), own[r].plan, ep[r], pool_ptrs, 0)
+    for r in range(R):
+        w1 = W1[r * Er:(r + 1) * Er].contiguous()
+        w2 = W2[r * Er:(r + 1) * Er].contiguous()
+        moe.moe_grouped_ffn(ls, pools[r].data_ptr(), w1.data_ptr(), w2.data_ptr(), ep[r].local,
+                            acts[r].data_ptr(), ypools[r].data_ptr(), moe.moe_config(), 0)
+    for r in range(R):
+        moe.moe_ep_combine(rs, R, r, ypool_ptrs, dw[r].data_ptr(), own[r].plan, ep[r],
+                           outs[r].data_ptr(), 0)
+    torch.cuda.synchronize()
+    for r in range(R):
+        assert moe.moe_get_status(own[r].plan)[0] == 0
+        assert moe.moe_get_status(ep[r].local)[0] == 0
+    if check_pools:
+        # every rank's pool = its experts' part of one pool over all ranks' pairs
+        idx_all = np.concatenate(idxs)
+        x_all = np.concatenate(xs)
+        ref = oracle.get().plan(idx_all, cfg.E, cfg.tile)
+        pool_all = oracle.get().pool(ref["row_src"], ref["P"], x_all, cfg.k)
+        for r in range(R):
+            a, b = int(ref["offsets"][r * Er]), int(ref["offsets"][(r + 1) * Er])
+            np.testing.assert_array_equal(bf16_host(pools[r][: b - a]), pool_all[a:b],
+                                          err_msg=f"rank {r} pool")
+    res = []
+    for r in range(R):
+        # the single-GPU layer on the same tokens and all experts
+        single = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+        o = single.forward(dx[r], i32_dev(idxs[r]), dw[r], W1, W2, moe.moe_config())
+        torch.cuda.synchronize()
+        res.append((outs[r], o.clone()))
+        single.close()
+    for b in own:
+        b.close()
+    return xs, idxs, ws, res
+
+
+EP_SHAPES = [
+    # name, T per rank, H, I, E, k, tile, R
+    ("R2", 200, 256, 256, 8, 2, 64, 2),
+    ("R4-tile128", 150, 384, 128, 16, 3, 128, 4),
+    ("R8-k8", 96, 256, 192, 32, 8, 64, 8),
+]
+
+
+@pytest.mark.parametrize("shape", EP_SHAPES, ids=[s[0] for s in EP_SHAPES])
+@pytest.mark.parametrize("drop", [0.0, 0.2])
+def test_ep_emulated_ranks_match_single_gpu_and_oracle(shape, drop):
+    from gpu_helpers import assert_layer_close, to_f64
+    name, T, H, I, E, k, tile, R = shape
+    cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=555 + T)
+    xs, idxs, ws, res = _run_ep(cfg, R, drop=drop)
+    W1h = [si.make_w1_expert(cfg, e) for e in range(E)]
+    W2h = [si.make_w2_expert(cfg, e) for e in range(E)]
+    for r, (ep_out, single_out) in enumerate(res):
+        assert torch.equal(ep_out.view(torch.int16), single_out.view(torch.int16)), f"rank {r}"
+        ref = oracle.get().moe_forward(xs[r], idxs[r], ws[r], W1h, W2h)
+        assert_layer_close(to_f64(ep_out), ref, f"{name} rank {r}")
+
+
+def test_ep_deepseek_shape_eight_ranks():
+    """Eight emulated ranks of the DeepSeek-V3 expert shape (H=7168, I=2048, 256 experts,
+    top-8) with 256 tokens each: outputs bit for bit the single-GPU layer's, sampled tokens
+    against the oracle."""
+    from gpu_helpers import assert_layer_close, sample_tokens, to_f64
+    base = si.CONFIGS["deepseek_v3"]
+    cfg = si.custom("ep-ds", T=256, H=base.H, I=base.I, E=base.E, k=base.k, tile=base.tile,
+                    seed=base.seed, routing=base.routing, bias_sigma=base.bias_sigma)
+    xs, idxs, ws, res = _run_ep(cfg, 8, check_pools=False)
+    for r, (ep_out, single_out) in enumerate(res):
+        assert torch.equal(ep_out.view(torch.int16), single_out.view(torch.int16)), f"rank {r}"
+    tok = sample_tokens(cfg.T, 8, seed=3)
+    W1h = [si.make_w1_expert(cfg, e) for e in range(cfg.E)]
+    W2h = [si.make_w2_expert(cfg, e) for e in range(cfg.E)]
+    ref = oracle.get().moe_forward(xs[0][tok], idxs[0][tok], ws[0][tok], W1h, W2h)
+    assert_layer_close(to_f64(res[0][0][torch.from_numpy(tok).to(res[0][0].device)]), ref,
+                       "deepseek-shaped EP rank 0")
+
+
+@pytest.mark.parametrize("bad", ["huge", "negative", "too_many_rows"])
+def test_ep_counts_that_disagree_with_the_plans_are_reported_not_followed(bad):
+    """A host-made failure: all_counts that no set of moe_plan calls can produce. The layout
+    clamps them and reports MOE_ERR_POOL_OVERFLOW; dispatch and combine place no row outside
+    a pool (guard rows after each pool stay untouched) and the context stays usable."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import DEV, bf16_dev, f32_dev, i32_dev
+    R = 2
+    cfg = si.custom("ep-bad", T=64, H=128, I=128, E=4, k=2, tile=64, seed=31)
+    rs = moe.moe_shape(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    rows = moe.moe_ep_pool_rows(rs, R)
+    guard = 64
+    own = [moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile, identity=True)
+           for _ in range(R)]
+    arenas = [torch.zeros(moe.moe_ep_arena_bytes(rs, R), dtype=torch.uint8, device=DEV)
+              for _ in range(R)]
+    ep = [moe.moe_ep_bind(rs, R, a.data_ptr()) for a in arenas]
+    pools = [torch.full((rows + guard, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+             for _ in range(R)]
+    ypools = [torch.zeros((rows + guard, cfg.H), dtype=torch.bfloat16, device=DEV)
+              for _ in range(R)]
+    outs = [torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    xs = [bf16_dev(si.make_x(cfg, r)) for r in range(R)]
+    routs = [si.make_routing(cfg, r) for r in range(R)]
+    for r in range(R):
+        moe.moe_plan(rs, i32_dev(routs[r][0]).data_ptr(), own[r].plan, 0, 0)
+    C = torch.stack([own[r].plan_view("counts")[: cfg.E] for r in range(R)]).contiguous()
+    if bad == "huge":
+        C[0, 1] = 1 << 30
+    elif bad == "negative":
+        C[1, 2] = -5
+    else:                      # within [0, T k] each, but moving rank 0's rows down
+        C[0, 0] = cfg.T * cfg.k
+    for r in range(R):
+        moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pools[r].data_ptr(), 0)
+    for r in range(R):
+        moe.moe_ep_dispatch(rs, R, r, xs[r].data_ptr(), own[r].plan, ep[r],
+                            [p.data_ptr() for p in pools], 0)
+    for r in range(R):
+        moe.moe_ep_combine(rs, R, r, [p.data_ptr() for p in ypools],
+                           f32_dev(routs[r][1]).data_ptr(), own[r].plan, ep[r],
+                           outs[r].data_ptr(), 0)
+    torch.cuda.synchronize()
+    codes = [moe.moe_get_status(ep[r].local)[0] for r in range(R)] + \
+            [moe.moe_get_status(own[r].plan)[0] for r in range(R)]
+    assert moe.MOE_ERR_POOL_OVERFLOW in codes, codes
+    assert set(codes) <= {0, moe.MOE_ERR_POOL_OVERFLOW}, codes
+    for r in range(R):
+        assert torch.isnan(pools[r][rows:].float()).all(), f"rank {r} guard rows written"
+    # the context still works: a clean single-GPU layer call
+    single = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    from gpu_helpers import weights_dev
+    W1, W2 = weights_dev(cfg)
+    single.forward(xs[0], i32_dev(routs[0][0]), f32_dev(routs[0][1]), W1, W2, moe.moe_config())
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(single.plan)[0] == 0
+    single.close()
+    for b in own:
+        b.close()
