@@ -57,6 +57,9 @@ def parse_args(argv=None):
                          "configuration, alternating on this GPU (reported under 'ab')")
     ap.add_argument("--backward", type=int, default=1,
                     help="1: also time moe_backward (after one forward), reported under 'backward'")
+    ap.add_argument("--ep", type=int, default=8,
+                    help="expert-parallel ranks emulated on this GPU for the 'ep' section "
+                         "(0: skip; needs E and T divisible by it)")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=16, help="oracle tokens per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -558,6 +561,117 @@ BUILT_LIBS = (os.path.join(ROOT, "combine_moe_plan_03_b200", "libmoe.so"),
               os.path.join(ROOT, "synth_inputs", "libsynth.so"))
 
 
+def time_ep(moe, cfg, dev, x, idx, w, W1, W2, packed, R, single_out, peaks, reps=10):
+    """The expert-parallel layer (moe_ep_*) with R ranks emulated on this GPU: rank r takes
+    tokens [r T/R, (r+1) T/R) of the workload and owns experts [r E/R, (r+1) E/R); every
+    rank's buffers live here, so the "peer" stores and loads are local HBM traffic. One
+    layer call = each rank's plan, the count exchange (a device copy standing in for the
+    all-gather of E integers), each rank's layout, dispatch, grouped FFN and combine, all on
+    one stream. Also reported: the bytes each rank would move over NVLink and the time they
+    need at the measured 770 GB/s per direction (other ranks' pairs only)."""
+    import torch
+    T_r, Er = cfg.T // R, cfg.E // R
+    H, I, E, k = cfg.H, cfg.I, cfg.E, cfg.k
+    rs = moe.moe_shape(T_r, H, I, E, k, cfg.tile)
+    ls = moe.moe_ep_local_shape(rs, R)
+    rows = moe.moe_ep_pool_rows(rs, R)
+    st = torch.cuda.current_stream().cuda_stream
+    bf = torch.bfloat16
+    own_arena = [torch.zeros(moe.moe_plan_arena_bytes(rs), dtype=torch.uint8, device=dev)
+                 for _ in range(R)]
+    own = [moe.moe_plan_bind(rs, a.data_ptr()) for a in own_arena]
+    ep_arena = [torch.zeros(moe.moe_ep_arena_bytes(rs, R), dtype=torch.uint8, device=dev)
+                for _ in range(R)]
+    ep = [moe.moe_ep_bind(rs, R, a.data_ptr()) for a in ep_arena]
+    pools = [torch.empty((rows, H), dtype=bf, device=dev) for _ in range(R)]
+    acts = [torch.empty((rows, I), dtype=bf, device=dev) for _ in range(R)]
+    ypools = [torch.empty((rows, H), dtype=bf, device=dev) for _ in range(R)]
+    out = torch.empty((cfg.T, H), dtype=bf, device=dev)
+    C = torch.zeros((R, E), dtype=torch.int32, device=dev)
+    counts = [own_arena[r][own[r].counts - own_arena[r].data_ptr():][: 4 * E].view(torch.int32)
+              for r in range(R)]
+    xr = [x[r * T_r:(r + 1) * T_r] for r in range(R)]
+    ir = [idx[r * T_r:(r + 1) * T_r] for r in range(R)]
+    wr = [w[r * T_r:(r + 1) * T_r] for r in range(R)]
+    # a rank's experts are a contiguous slice of the weights in either layout (the packed
+    # tiles are expert-major)
+    w1b = W1.numel() * W1.element_size() // E
+    w2b = W2.numel() * W2.element_size() // E
+    fcfg = moe.moe_config(packed_weights=packed)
+    pp, yp = [p.data_ptr() for p in pools], [p.data_ptr() for p in ypools]
+
+    def call(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record()
+        mark(0)
+        for r in range(R):
+            moe.moe_plan(rs, ir[r].data_ptr(), own[r], 0, st)
+        for r in range(R):
+            C[r].copy_(counts[r])
+        mark(1)
+        for r in range(R):
+            moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pp[r], st)
+        mark(2)
+        for r in range(R):
+            moe.moe_ep_dispatch(rs, R, r, xr[r].data_ptr(), own[r], ep[r], pp, st)
+        mark(3)
+        for r in range(R):
+            moe.moe_grouped_ffn(ls, pp[r], W1.data_ptr() + r * Er * w1b,
+                                W2.data_ptr() + r * Er * w2b, ep[r].local, acts[r].data_ptr(),
+                                yp[r], fcfg, st)
+        mark(4)
+        for r in range(R):
+            moe.moe_ep_combine(rs, R, r, yp, wr[r].data_ptr(), own[r], ep[r],
+                               out[r * T_r:(r + 1) * T_r].data_ptr(), st)
+        mark(5)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    codes = [moe.moe_get_status(p)[0] for p in own] + \
+        [moe.moe_get_status(e_.local)[0] for e_ in ep]
+    if any(codes):
+        raise RuntimeError(f"device status in the EP layer: {codes}")
+    matches = bool(torch.equal(out.view(torch.int16), single_out.view(torch.int16)))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(reps)]
+    for i in range(reps):
+        call(evs[i])
+    torch.cuda.synchronize()
+    names = ("plan_and_exchange", "layout", "dispatch", "grouped_ffn", "combine")
+    ph = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(reps)) / reps
+          for j, n in enumerate(names)}
+    total = sum(evs[i][0].elapsed_time(evs[i][5]) for i in range(reps)) / reps
+    idx_h = idx.cpu().numpy()
+    pairs = int((idx_h >= 0).sum())
+    remote = []
+    for r in range(R):
+        e_ = idx_h[r * T_r:(r + 1) * T_r]
+        e_ = e_[e_ >= 0]
+        remote.append(int((e_ // Er != r).sum()))
+    disp_b = cfg.T * H * 2 + pairs * H * 2
+    comb_b = pairs * H * 2 + pairs * 8 + cfg.T * H * 2
+    nv_b = max(remote) * H * 2
+    res = {"ranks": R, "tokens_per_rank": T_r, "experts_per_rank": Er,
+           "emulated": "all ranks on this GPU, their kernels one after another: peer "
+                       "stores and loads are local HBM traffic; on R GPUs the ranks run side "
+                       "by side and each rank's rows for other ranks cross NVLink",
+           "ms_per_layer_call": total, "tokens_per_s": cfg.T / (total / 1e3),
+           "phases_ms_per_call": {n: round(v, 5) for n, v in ph.items()},
+           "dispatch_gbs": disp_b / (ph["dispatch"] / 1e3) / 1e9,
+           "combine_gbs": comb_b / (ph["combine"] / 1e3) / 1e9,
+           "dispatch_frac_hbm": disp_b / (ph["dispatch"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+           "combine_frac_hbm": comb_b / (ph["combine"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+           "matches_single_gpu_layer": matches,
+           "nvlink": {"remote_pairs_per_rank_max": max(remote),
+                      "bytes_per_rank_each_way_max": nv_b,
+                      "dispatch_bound_ms_at_770_gbs": nv_b / 770e9 * 1e3,
+                      "note": "on R GPUs each rank's dispatch stores, and its combine loads, "
+                              "these bytes over NVLink (rows of pairs routed to other ranks)"},
+           "gpu_launches_per_call": R * (3 + 1 + 5 + 1 + 2 + 1)}
+    return res
+
+
 def ensure_library(local: int) -> None:
     """Build the libraries when one is missing (a checkout without built libraries): the first
     local rank builds all three, the others wait until all three exist. Every build writes
@@ -690,6 +804,18 @@ def run_moe(args):
     for i in idxs:
         cnt = np.bincount(i[i >= 0].reshape(-1), minlength=cfg.E)
         Ps.append(int(((cnt + cfg.tile - 1) // cfg.tile * cfg.tile).sum()))
+    # rows the grouped GEMMs compute: each expert's rows in ceil(c / 256) equal chunks (a
+    # multiple of 16), every chunk's live rows rounded up to 16 (the MMA's N granularity)
+    exec_rows = []
+    for i in idxs:
+        cnt = np.bincount(i[i >= 0].reshape(-1), minlength=cfg.E)
+        rows = 0
+        for c in cnt[cnt > 0].tolist():
+            n = -(-c // 256)
+            chunk = (-(-c // n) + 15) // 16 * 16
+            rows += sum((min(chunk, c - r) + 15) // 16 * 16 for r in range(0, c, chunk))
+        exec_rows.append(rows)
+    exec_rows_m = float(np.mean(exec_rows))
     pairs_m = float(np.mean(pairs))
     n_live_experts = float(np.mean([len(np.unique(i[i >= 0])) for i in idxs]))
     P_m = float(np.mean(Ps))
@@ -732,7 +858,7 @@ def run_moe(args):
         flops_y = pairs_m * 2.0 * H * I
         ffn_ms = ph["gemm_a"] + ph["gemm_y"]
         ffn_tflops = (flops_a + flops_y) / (ffn_ms / 1e3) / 1e12
-        exec_tflops = P_m * 6.0 * H * I / (ffn_ms / 1e3) / 1e12
+        exec_tflops = exec_rows_m * 6.0 * H * I / (ffn_ms / 1e3) / 1e12
         line["grouped_ffn"] = {"useful_tflops": ffn_tflops,
                                "frac_bf16_peak": ffn_tflops / peaks["bf16_tflops"],
                                "executed_tflops": exec_tflops,
@@ -833,6 +959,18 @@ def run_moe(args):
         line["backward"] = time_backward(moe, buf, cfg, dev, world, local, dx[0], didx[0], dw[0], W1,
                                          W2, W1u, W2u, packed, pairs[0], peaks, peak_src,
                                          args.steps)
+
+    # ---------------- expert parallelism with R ranks emulated on this GPU (moe_ep_*)
+    R = args.ep
+    if (R > 1 and world == 1 and not cfg.identity and mbs == 1 and cfg.E % R == 0
+            and cfg.T % R == 0):
+        buf.forward(dx[0], didx[0], dw[0], W1, W2, plain)
+        torch.cuda.synchronize()
+        single = buf.out.clone()
+        line["ep"] = time_ep(moe, cfg, dev, dx[0], didx[0], dw[0], W1, W2, packed, R, single,
+                             peaks)
+        del single
+        torch.cuda.empty_cache()
 
     # ---------------- e2e: pinned host inputs in, result out, copies inside the timed region
     hx = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in xs]

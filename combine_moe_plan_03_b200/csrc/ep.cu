@@ -65,15 +65,17 @@ __global__ void __launch_bounds__(kEpThreads)
   }
 }
 
-// Padding rows of this rank's pool: [offsets[e] + counts[e], offsets[e + 1]) per local expert.
+// Padding rows of this rank's pool: [offsets[e] + counts[e], offsets[e + 1]) per local expert,
+// every expert's rows spread over the whole grid (16-byte stores).
 __global__ void __launch_bounds__(kEpThreads)
     ep_pad_kernel(uint4 *__restrict__ pool, int32_t hv, const int32_t *__restrict__ counts,
                   const int32_t *__restrict__ offsets, int32_t Er) {
-  for (int e = blockIdx.x; e < Er; e += gridDim.x) {
+  const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t gsz = (int64_t)gridDim.x * blockDim.x;
+  for (int e = 0; e < Er; ++e) {
     const int64_t r0 = offsets[e] + counts[e], r1 = offsets[e + 1];
     const int64_t n = (r1 - r0) * hv;
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x)
-      pool[r0 * hv + i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t i = gtid; i < n; i += gsz) pool[r0 * hv + i] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -237,8 +239,7 @@ cudaError_t launch_ep_layout(const moe_shape &rank_shape, int32_t R, int32_t ran
   if (cudaMemsetAsync(ep.local.tile_flags, 0, sizeof(uint32_t) * (size_t)lg.n_tiles, st) !=
       cudaSuccess)
     return cudaErrorUnknown;
-  const int pgrid = Er < num_sms * 2 ? Er : num_sms * 2;
-  ep_pad_kernel<<<pgrid > 0 ? pgrid : 1, kEpThreads, 0, st>>>(
+  ep_pad_kernel<<<num_sms * 2, kEpThreads, 0, st>>>(
       static_cast<uint4 *>(pool), rank_shape.H / 8, ep.local.counts, ep.local.offsets, Er);
   return cudaGetLastError();
 }

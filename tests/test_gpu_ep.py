@@ -193,3 +193,28 @@ def test_ep_counts_that_disagree_with_the_plans_are_reported_not_followed(bad):
     single.close()
     for b in own:
         b.close()
+
+
+def test_bench_ep_section_matches_single_gpu_layer():
+    """bench.py's expert-parallel timing section on a small workload, with prepacked weights
+    sliced per rank: its output equals the single-GPU layer's bit for bit and its rates are
+    positive."""
+    import bench
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import DEV, bf16_dev, f32_dev, i32_dev, weights_dev
+    cfg = si.custom("ep-bench", T=512, H=512, I=256, E=16, k=4, tile=128, seed=91)
+    W1, W2 = weights_dev(cfg)
+    buf = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    W1p, W2p = buf.pack_weights(W1, W2)
+    x = bf16_dev(si.make_x(cfg))
+    idx, w = si.make_routing(cfg)
+    di, dw = i32_dev(idx), f32_dev(w)
+    single = buf.forward(x, di, dw, W1p, W2p, moe.moe_config(packed_weights=1))
+    torch.cuda.synchronize()
+    single = single.clone()
+    peaks, _ = bench.load_peaks()
+    res = bench.time_ep(moe, cfg, DEV, x, di, dw, W1p, W2p, 1, 4, single, peaks, reps=2)
+    assert res["matches_single_gpu_layer"]
+    assert res["ms_per_layer_call"] > 0 and res["dispatch_gbs"] > 0 and res["combine_gbs"] > 0
+    assert res["nvlink"]["remote_pairs_per_rank_max"] <= cfg.T // 4 * cfg.k
+    buf.close()
