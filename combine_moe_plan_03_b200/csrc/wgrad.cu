@@ -6,21 +6,25 @@
 // with A, B row-major [P_max, M] / [P_max, N] activations and D [E, M, N] bf16.
 //
 // Design (tcgen05, SM pairs as in ffn_gemm_pair.cu): a work unit is (expert, 256 rows of D,
-// 256 columns of D); one cta_group::2 MMA has M = 256 (128 rows of D per CTA) and N = 256
-// (each CTA holds 128 of B's columns), K = 16; the K loop runs over the expert's rows in
-// steps of 64 (its live rows rounded up to 64: rows past the live ones must be zero, which
-// zero_pad_rows_kernel ensures for the operands that are not zero there already). Both
-// operands are read MN-major straight from the activations (for A the rows of D are
-// contiguous in memory, for B its columns), two TMA boxes of 64 columns x 64 rows each per
-// operand and CTA: 32 KB per stage, 5 stages. One accumulator of 256 TMEM columns per unit
-// in two buffers, so the epilogue of one unit overlaps the MMAs of the next. In the epilogue
+// 512 columns of D); one cta_group::2 MMA has M = 256 (128 rows of D per CTA) and N = 256
+// (each CTA holds 128 of B's columns), K = 16, into one of two accumulators of 256 TMEM
+// columns; the K loop runs over the expert's rows in steps of 64 (its live rows rounded up
+// to 64: rows past the live ones must be zero, which zero_pad_rows_kernel ensures for the
+// operands that are not zero there already). Both operands are read MN-major straight from
+// the activations (for A the rows of D are contiguous in memory, for B its columns), TMA
+// boxes of 64 columns x 64 rows: per stage and CTA two of A and four of B (48 KB), 3 stages.
+// The epilogue hands the two accumulators back one at a time; the next unit's MMAs into the
+// first are issued while the second is still being read. (The narrow tiling, 256 columns
+// per unit with one accumulator in two buffers and 5 stages of 32 KB, is kept as the
+// MOE_WGRAD_WIDE=0 build: it draws a third more operand bytes per flop.) In the epilogue
 // each thread holds one row of D (its TMEM lane) and 32 consecutive columns per load; a
 // warp's 32 x 64 share of a unit goes through shared memory (128-byte swizzled) to one TMA
-// store, which writes whole 128-byte row segments; 16 epilogue warps keep the epilogue of a
-// unit shorter than its MMAs even for the experts with few rows (the gradients are 3·E·H·I bf16
-// values per call and their writes bound the kernel). An expert with no rows gets a zero
+// store, which writes whole 128-byte row segments (16 epilogue warps; the gradients are
+// 3·E·H·I bf16 values per call). An expert with no rows gets a zero
 // gradient. Waits are bounded as in the forward kernels; a wait that runs out reports
 // MOE_ERR_PIPE_TIMEOUT and raises both CTAs' abort flags.
+#include <mutex>
+
 #include "ffn_gemm.cuh"
 
 namespace moe {
@@ -30,9 +34,6 @@ namespace {
 constexpr int kBK = 64;
 constexpr int kBoxBytes = 64 * kBK * 2;       // 8 KB: 64 columns x 64 rows
 constexpr int kOpBytes = 2 * kBoxBytes;       // 16 KB: 128 columns of one operand
-constexpr int kStageBytes = 2 * kOpBytes;     // A and B
-constexpr int kStages = 5;
-constexpr int kRingBytes = kStages * kStageBytes;  // 160 KB
 constexpr int kTmemCols = 512;
 constexpr int kBufCols = 256;
 constexpr int kEpiWarps = 16;                  // 4 per TMEM lane quadrant, 64 columns each
@@ -42,9 +43,26 @@ constexpr int kSchedReaders = 1 + kEpiWarps + 1 + kEpiWarps;
 constexpr int kBarrierBytes = 256;
 constexpr int kStageOutBytes = 32 * 64 * 2;    // a warp's 32 rows x 64 columns of D
 constexpr int kOutBytes = kEpiWarps * kStageOutBytes;
-// shared memory: stage ring, then the epilogue's blocks (1024-byte aligned, as the 128-byte
-// swizzle of their TMA stores wants), then the barriers
-constexpr int kSmemBytes = kRingBytes + kOutBytes + kBarrierBytes + 1024;
+
+// Two tilings of D. Narrow: a unit is 256 x 256 of D, one accumulator of 256 TMEM columns in
+// two buffers (the epilogue of one unit overlaps the MMAs of the next), stages of A and one
+// B half (32 KB), 5 stages. Wide: a unit is 256 x 512 of D, two accumulators (all 512 TMEM
+// columns), stages of A and two B halves (48 KB), 3 stages: each A tile serves twice the
+// MMA work, so the SMs draw 25% fewer operand bytes per flop from L2; the accumulators are
+// handed back one at a time and the next unit's MMAs into the first start meanwhile.
+template <bool kWide>
+struct WgradGeom {
+  static constexpr int kAccs = kWide ? 2 : 1;               // accumulators per unit
+  static constexpr int kUnitCols = 256 * kAccs;             // columns of D per unit
+  static constexpr int kStageBytes = kOpBytes * (1 + kAccs);
+  static constexpr int kStages = kWide ? 3 : 5;
+  static constexpr int kRingBytes = kStages * kStageBytes;  // 160 KB / 144 KB
+  // shared memory: stage ring, then the epilogue's blocks (1024-byte aligned, as the
+  // 128-byte swizzle of their TMA stores wants), then the barriers
+  static constexpr int kSmemBytes = kRingBytes + kOutBytes + kBarrierBytes + 1024;
+};
+static_assert(WgradGeom<true>::kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(WgradGeom<false>::kSmemBytes <= 227 * 1024, "shared memory");
 constexpr uint64_t kAbortGraceNs = 1000000;
 constexpr uint32_t kParkNs = 20000;
 
@@ -54,7 +72,7 @@ struct WgradParams {
   int32_t *status;
   uint16_t *out;            // D [E, M, N]
   int32_t E, M, N;
-  int32_t mb_count, nb_count;  // blocks of 256 rows / columns of D
+  int32_t mb_count, nb_count;  // blocks of 256 rows / of the unit's columns of D
   int32_t *sched;           // {ticket, clusters done}
   uint64_t timeout_ns;
 };
@@ -70,17 +88,22 @@ __device__ __forceinline__ int32_t k_steps(const WgradParams &prm, int32_t e) {
   return (prm.counts[e] + kBK - 1) / kBK;
 }
 
+template <bool kWide>
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                       const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_d, const WgradParams prm) {
+  using G = WgradGeom<kWide>;
+  constexpr int kStages = G::kStages;
+  constexpr int kStageBytes = G::kStageBytes;
+  constexpr int kRingBytes = G::kRingBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRingBytes + kOutBytes);
   uint64_t *empty = full + kStages;
-  uint64_t *acc_full = empty + kStages;    // [2]
-  uint64_t *acc_empty = acc_full + 2;      // [2]
+  uint64_t *acc_full = empty + kStages;    // [2]: buffers (narrow) / one per unit (wide)
+  uint64_t *acc_empty = acc_full + 2;      // [2]: buffers (narrow) / accumulators (wide)
   uint64_t *drain = acc_empty + 2;
   uint64_t *sched_full = drain + 1;
   uint64_t *sched_empty = sched_full + kSchedSlots;
@@ -178,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t nb = rest % prm.nb_count;
         const int32_t row0 = prm.offsets[e];
         const int32_t acol = mb * 256 + (int32_t)rank * 128;
-        const int32_t bcol = nb * 256 + (int32_t)rank * 128;
+        const int32_t bcol = nb * G::kUnitCols + (int32_t)rank * 128;
         for (int32_t kb = 0; kb < kcount; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1u, 2 * prm.timeout_ns, abort)) {
             raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
@@ -197,6 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d_pair(sa + kBoxBytes, &tm_a, fb, acol + 64, r);
           tma_load_2d_pair(sb, &tm_b, fb, bcol, r);
           tma_load_2d_pair(sb + kBoxBytes, &tm_b, fb, bcol + 64, r);
+          if (kWide) {  // the second accumulator's B half: 256 columns further
+            tma_load_2d_pair(sb + kOpBytes, &tm_b, fb, bcol + 256, r);
+            tma_load_2d_pair(sb + kOpBytes + kBoxBytes, &tm_b, fb, bcol + 320, r);
+          }
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -236,13 +263,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           sphase ^= 1u;
         }
         if (u < 0) break;
-        const uint32_t buf = local & 1u, use = local >> 1;
-        if (!mbar_wait<true>(acc_empty + buf, (use + 1u) & 1u, 2 * prm.timeout_ns, abort)) {
+        // narrow: the unit's accumulator is buffer local % 2, in its (local / 2)-th use;
+        // wide: accumulators 0 and 1 (TMEM columns 0 and 256), each in its local-th use
+        const uint32_t buf = kWide ? 0u : (local & 1u);
+        const uint32_t empty_parity = kWide ? ((local + 1u) & 1u) : (((local >> 1) + 1u) & 1u);
+        if (!mbar_wait<true>(acc_empty + buf, empty_parity, 2 * prm.timeout_ns, abort)) {
           raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem_base + buf * kBufCols;
+        bool need1 = kWide;  // the second accumulator not yet handed back for this unit
         for (int32_t kb = 0; kb < kcount; ++kb) {
           if (!mbar_wait(full + stage, phase, 2 * prm.timeout_ns, abort)) {
             raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
@@ -260,6 +291,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = smem_desc_sw128(sb + kk * 2048, kBoxBytes, 1024);
             tc_mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
+          if (kWide) {
+            if (need1) {
+              // the first accumulator's MMAs of this k-step are queued; now the second
+              // accumulator must have been read by both CTAs' epilogues
+              if (!mbar_wait<true>(acc_empty + 1, empty_parity, 2 * prm.timeout_ns, abort)) {
+                raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              need1 = false;
+            }
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(sa + kk * 2048, kBoxBytes, 1024);
+              const uint64_t bd = smem_desc_sw128(sb + kOpBytes + kk * 2048, kBoxBytes, 1024);
+              tc_mma_bf16_pair(d + kBufCols, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+          }
           tc_commit_pair_mc(empty + stage, 0x3);
           if (++stage == kStages) {
             stage = 0;
@@ -267,6 +317,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
+        if (need1) {  // a unit without rows: still one use of the second accumulator
+          if (!mbar_wait<true>(acc_empty + 1, empty_parity, 2 * prm.timeout_ns, abort)) {
+            raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
+            break;
+          }
+          tc_fence_after();
+        }
         tc_commit_pair_mc(acc_full + buf, 0x3);
       }
       tc_commit_pair_mc(drain, 0x1);
@@ -318,11 +375,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t mb = rest / prm.nb_count;
       const int32_t nb = rest % prm.nb_count;
       const bool live = kc > 0;
-      const uint32_t buf = local & 1u, use = local >> 1;
+      const uint32_t buf = kWide ? 0u : (local & 1u);
+      const uint32_t full_parity = kWide ? (local & 1u) : ((local >> 1) & 1u);
       int ok = 1;
       if (lane == 0)
-        ok = mbar_wait_parked(acc_full + buf, use & 1u, 3 * prm.timeout_ns, abort, kParkNs) ? 1
-                                                                                          : 0;
+        ok = mbar_wait_parked(acc_full + buf, full_parity, 3 * prm.timeout_ns, abort, kParkNs)
+                 ? 1
+                 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
@@ -330,45 +389,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int32_t m0 = mb * 256 + (int32_t)rank * 128 + quad * 32;  // first row of D here
-      const int32_t ncol0 = nb * 256 + part * 64;                      // first column of D here
-      const bool store = m0 < prm.M && ncol0 < prm.N;                  // uniform across the warp
-      // the warp's 64 columns into registers as bf16 pairs, then the TMEM buffer goes back
-      // to the MMA thread before the (possibly waiting) staging and store
-      uint32_t pk[32];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t a[32];
-        __syncwarp();
-        if (live) {
-          tmem_ld_32x32b_x32(tq + buf * kBufCols + part * 64 + q * 32, a);
-          tmem_ld_wait();
+      for (int j = 0; j < G::kAccs; ++j) {
+        const uint32_t acc = kWide ? (uint32_t)j : buf;                 // TMEM buffer / barrier
+        const int32_t ncol0 = nb * G::kUnitCols + j * 256 + part * 64;  // first column of D here
+        const bool store = m0 < prm.M && ncol0 < prm.N;                 // uniform across the warp
+        // the warp's 64 columns into registers as bf16 pairs, then the accumulator goes back
+        // to the MMA thread before the (possibly waiting) staging and store
+        uint32_t pk[32];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t a[32];
+          __syncwarp();
+          if (live) {
+            tmem_ld_32x32b_x32(tq + acc * kBufCols + part * 64 + q * 32, a);
+            tmem_ld_wait();
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[16 * q + i] =
+                live ? pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])) : 0u;
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[16 * q + i] =
-              live ? pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])) : 0u;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (lead)
-          mbar_arrive(acc_empty + buf);
-        else
-          mbar_arrive_cluster(cluster_map(smem_u32(acc_empty + buf), 0));
-      }
-      if (store) {
-        // the previous unit's store has read the block
-        if (lane == 0) bulk_wait_group_read<0>();
-        __syncwarp();
-        uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 128);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          row[c ^ (lane & 7)] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tm_d, stg, ncol0, e * prm.M + m0);
-          bulk_commit_group();
+          if (lead)
+            mbar_arrive(acc_empty + acc);
+          else
+            mbar_arrive_cluster(cluster_map(smem_u32(acc_empty + acc), 0));
+        }
+        if (store) {
+          // the previous store has read the block
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+          uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            row[c ^ (lane & 7)] =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_d, stg, ncol0, e * prm.M + m0);
+            bulk_commit_group();
+          }
         }
       }
     }
@@ -416,18 +480,32 @@ cudaError_t launch_zero_pad_rows(const moe_shape &s, void *buf, int32_t width,
   return cudaGetLastError();
 }
 
-// D [E, M, N] = per expert A_e^T B_e over the expert's segment; A [P_max, M], B [P_max, N].
-int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, int32_t N,
-                 void *D, const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg,
-                 int num_sms, cudaStream_t st) {
-  const PlanGeom g = plan_geom(s);
-  CUtensorMap ta, tb, td;
-  const uint64_t rows = g.pmax > 0 ? (uint64_t)g.pmax : 1;
-  if (!make_tmap(&ta, A, (uint64_t)M, rows, kBK) || !make_tmap(&tb, B, (uint64_t)N, rows, kBK) ||
-      !make_tmap_box(&td, D, (uint64_t)N, (uint64_t)s.E * M, 64, 32, true))
-    return MOE_ERR_CUDA;
-  static bool attr_set[64] = {false};
-  static int fit_cache[64] = {0};
+// Cluster fit of one kernel variant per device, found once (under a lock: host threads may
+// launch at the same time).
+template <bool kWide>
+int wgrad_fit(int dev, cudaLaunchConfig_t lc) {
+  static std::mutex mu;
+  static int fit[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (fit[dev] == 0) {
+    if (cudaFuncSetAttribute(wgrad_pair_kernel<kWide>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             WgradGeom<kWide>::kSmemBytes) != cudaSuccess)
+      return 0;
+    lc.gridDim = dim3(2, 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, wgrad_pair_kernel<kWide>, &lc) != cudaSuccess || n < 1)
+      return 0;
+    fit[dev] = n;
+  }
+  return fit[dev];
+}
+
+template <bool kWide>
+int launch_wgrad_t(const moe_shape &s, const CUtensorMap &ta, const CUtensorMap &tb,
+                   const CUtensorMap &td, int32_t M, int32_t N, void *D,
+                   const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg, int num_sms,
+                   cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
@@ -438,23 +516,14 @@ int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, in
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
   lc.blockDim = dim3(kThreads, 1, 1);
-  lc.dynamicSmemBytes = kSmemBytes;
+  lc.dynamicSmemBytes = WgradGeom<kWide>::kSmemBytes;
   lc.attrs = at;
   lc.numAttrs = 1;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(wgrad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    lc.gridDim = dim3(2, 1, 1);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, wgrad_pair_kernel, &lc) != cudaSuccess || n < 1)
-      return MOE_ERR_CUDA;
-    fit_cache[dev] = n;
-    attr_set[dev] = true;
-  }
+  const int fit = wgrad_fit<kWide>(dev, lc);
+  if (fit < 1) return MOE_ERR_CUDA;
   int clusters = (cfg.ffn_ctas > 0 ? cfg.ffn_ctas : num_sms) / 2;
   if (clusters < 1) clusters = 1;
-  if (clusters > fit_cache[dev]) clusters = fit_cache[dev];
+  if (clusters > fit) clusters = fit;
   WgradParams prm{};
   prm.offsets = p.offsets;
   prm.counts = p.counts;
@@ -464,14 +533,33 @@ int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, in
   prm.M = M;
   prm.N = N;
   prm.mb_count = (M + 255) / 256;
-  prm.nb_count = (N + 255) / 256;
+  prm.nb_count = (N + WgradGeom<kWide>::kUnitCols - 1) / WgradGeom<kWide>::kUnitCols;
   prm.sched = sched;
   prm.timeout_ns = (uint64_t)(cfg.wait_timeout_us > 0 ? cfg.wait_timeout_us : 2000000) * 1000ull;
   lc.gridDim = dim3(2 * clusters, 1, 1);
   lc.stream = st;
-  if (cudaLaunchKernelEx(&lc, wgrad_pair_kernel, ta, tb, td, prm) != cudaSuccess)
+  if (cudaLaunchKernelEx(&lc, wgrad_pair_kernel<kWide>, ta, tb, td, prm) != cudaSuccess)
     return MOE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+#ifndef MOE_WGRAD_WIDE
+#define MOE_WGRAD_WIDE 1
+#endif
+
+// D [E, M, N] = per expert A_e^T B_e over the expert's segment; A [P_max, M], B [P_max, N].
+int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, int32_t N,
+                 void *D, const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg,
+                 int num_sms, cudaStream_t st) {
+  const PlanGeom g = plan_geom(s);
+  CUtensorMap ta, tb, td;
+  const uint64_t rows = g.pmax > 0 ? (uint64_t)g.pmax : 1;
+  if (!make_tmap(&ta, A, (uint64_t)M, rows, kBK) || !make_tmap(&tb, B, (uint64_t)N, rows, kBK) ||
+      !make_tmap_box(&td, D, (uint64_t)N, (uint64_t)s.E * M, 64, 32, true))
+    return MOE_ERR_CUDA;
+  if (MOE_WGRAD_WIDE)
+    return launch_wgrad_t<true>(s, ta, tb, td, M, N, D, p, sched, cfg, num_sms, st);
+  return launch_wgrad_t<false>(s, ta, tb, td, M, N, D, p, sched, cfg, num_sms, st);
 }
 
 }  // namespace moe
