@@ -49,6 +49,7 @@
 // MOE_ERR_PIPE_TIMEOUT / MOE_ERR_FLAG_TIMEOUT in the status word and raises a
 // CTA-wide abort flag; the roles then leave their loops, the producer waits for
 // the loads it has in flight, the MMA thread for its MMAs, and the TMEM is freed.
+#include <mutex>
 #include "ffn_gemm.cuh"
 
 namespace moe {
@@ -393,15 +394,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
+  // looked up once (a function-local static is initialised once, thread-safely)
+  static const EncodeTiledFn fn = [] {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
   return fn;
 }
 
@@ -429,15 +431,18 @@ template <int kMode>
 static cudaError_t launch_one(const CUtensorMap &tw, const CUtensorMap &tx, const FfnParams &prm,
                               int grid, cudaStream_t st) {
   static bool attr_set[64] = {false};
+  static std::mutex mu;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::unique_lock<std::mutex> lock(mu);
   if (!attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<kMode>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  lock.unlock();
   ffn_gemm_kernel<kMode><<<grid, kThreads, kSmemBytes, st>>>(tw, tx, prm);
   return cudaGetLastError();
 }

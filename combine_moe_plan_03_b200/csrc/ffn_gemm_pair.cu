@@ -40,6 +40,7 @@
 // leave through two cluster barriers (with a grace period between them after an
 // abort, for loads still in flight) so that neither exits while the other may still
 // write to its shared memory or barriers, and then free the TMEM.
+#include <mutex>
 #include "ffn_gemm.cuh"
 
 namespace moe {
@@ -724,14 +725,19 @@ template <int kMode, bool kAK, bool kEarly = false>
 cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnParams &prm,
                         int clusters, cudaStream_t st) {
   static bool attr_set[64] = {false};
+  static std::mutex mu;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK, kEarly>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK, kEarly>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
   }
   cudaLaunchConfig_t lc = {};
   cudaLaunchAttribute at[1];
@@ -753,8 +759,10 @@ cudaError_t launch_mode(const CUtensorMap &tw, const CUtensorMap &tx, const FfnP
 template <int kMode, bool kAK, bool kEarly = false>
 int max_clusters_mode() {
   static int cached[64] = {0};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
   if (cached[dev] == 0) {
     if (cudaFuncSetAttribute(ffn_gemm_pair_kernel<kMode, kAK, kEarly>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,

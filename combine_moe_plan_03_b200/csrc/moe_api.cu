@@ -1,6 +1,7 @@
 // C ABI of libmoe.so (declared in include/moe.h): argument checks, plan arena
 // layout, and the ordering of the layer's kernels on the caller's communicate
 // and compute streams (StreamEP README, How it works, "Caller-owned streams").
+#include <mutex>
 #include <string.h>
 
 #include "moe_common.cuh"
@@ -13,8 +14,10 @@ namespace {
 int sm_count_cached(int *out) {
   static int counts[64] = {0};
   static int ok[64] = {0};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
   if (!ok[dev]) {
     int major = 0, n = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
