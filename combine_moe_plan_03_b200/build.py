@@ -16,6 +16,8 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-shared",
     "--expt-relaxed-constexpr",
     "-Xptxas", "-v",
+    # export only the C ABI (moe_*)
+    "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map"),
 ]
 
 

@@ -481,9 +481,11 @@ cudaError_t launch_zero_pad_rows(const moe_shape &s, void *buf, int32_t width,
 }
 
 // Cluster fit of one kernel variant per device, found once (under a lock: host threads may
-// launch at the same time).
+// launch at the same time). Internal linkage: the static locals of a function template with
+// external linkage are one object per process, shared by every copy of this library that is
+// loaded, and another copy's cache would skip this copy's shared-memory attribute.
 template <bool kWide>
-int wgrad_fit(int dev, cudaLaunchConfig_t lc) {
+static int wgrad_fit(int dev, cudaLaunchConfig_t lc) {
   static std::mutex mu;
   static int fit[64] = {0};
   std::lock_guard<std::mutex> lock(mu);
@@ -502,7 +504,7 @@ int wgrad_fit(int dev, cudaLaunchConfig_t lc) {
 }
 
 template <bool kWide>
-int launch_wgrad_t(const moe_shape &s, const CUtensorMap &ta, const CUtensorMap &tb,
+static int launch_wgrad_t(const moe_shape &s, const CUtensorMap &ta, const CUtensorMap &tb,
                    const CUtensorMap &td, int32_t M, int32_t N, void *D,
                    const moe_plan_buffers &p, int32_t *sched, const moe_config &cfg, int num_sms,
                    cudaStream_t st) {
