@@ -597,10 +597,13 @@ def time_ep(moe, cfg, dev, x, idx, w, W1, W2, packed, R, single_out, peaks, reps
     # tiles are expert-major)
     w1b = W1.numel() * W1.element_size() // E
     w2b = W2.numel() * W2.element_size() // E
-    fcfg = moe.moe_config(packed_weights=packed)
     pp, yp = [p.data_ptr() for p in pools], [p.data_ptr() for p in ypools]
+    # every stored row is counted on its owner's tile flag; the 'streaming' pass lets each
+    # rank's GEMM A take tiles by their flags (here they are full: dispatches come first)
+    flags = [e_.local.tile_flags for e_ in ep]
+    fcfg = moe.moe_config(packed_weights=packed)
 
-    def call(evs=None):
+    def call(evs=None, fcfg=fcfg):
         def mark(i):
             if evs is not None:
                 evs[i].record()
@@ -614,7 +617,7 @@ def time_ep(moe, cfg, dev, x, idx, w, W1, W2, packed, R, single_out, peaks, reps
             moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pp[r], st)
         mark(2)
         for r in range(R):
-            moe.moe_ep_dispatch(rs, R, r, xr[r].data_ptr(), own[r], ep[r], pp, st)
+            moe.moe_ep_dispatch(rs, R, r, xr[r].data_ptr(), own[r], ep[r], pp, st, flags)
         mark(3)
         for r in range(R):
             moe.moe_grouped_ffn(ls, pp[r], W1.data_ptr() + r * Er * w1b,
@@ -642,6 +645,22 @@ def time_ep(moe, cfg, dev, x, idx, w, W1, W2, packed, R, single_out, peaks, reps
     ph = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(reps)) / reps
           for j, n in enumerate(names)}
     total = sum(evs[i][0].elapsed_time(evs[i][5]) for i in range(reps)) / reps
+    # the same calls with streaming grouped FFNs (GEMM A waits on the tile flags; on this
+    # one GPU they are full by then, and GEMM A leaves the dispatch SMs free)
+    scfg = moe.moe_config(packed_weights=packed, streaming=1)
+    out.zero_()
+    call(None, scfg)
+    torch.cuda.synchronize()
+    s_matches = bool(torch.equal(out.view(torch.int16), single_out.view(torch.int16)))
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(reps)]
+    for i in range(reps):
+        call(sev[i], scfg)
+    torch.cuda.synchronize()
+    s_total = sum(sev[i][0].elapsed_time(sev[i][5]) for i in range(reps)) / reps
+    codes = [moe.moe_get_status(p)[0] for p in own] + \
+        [moe.moe_get_status(e_.local)[0] for e_ in ep]
+    if any(codes):
+        raise RuntimeError(f"device status in the streaming EP layer: {codes}")
     idx_h = idx.cpu().numpy()
     pairs = int((idx_h >= 0).sum())
     remote = []
@@ -663,6 +682,8 @@ def time_ep(moe, cfg, dev, x, idx, w, W1, W2, packed, R, single_out, peaks, reps
            "dispatch_frac_hbm": disp_b / (ph["dispatch"] / 1e3) / 1e9 / peaks["hbm_gbs"],
            "combine_frac_hbm": comb_b / (ph["combine"] / 1e3) / 1e9 / peaks["hbm_gbs"],
            "matches_single_gpu_layer": matches,
+           "streaming": {"ms_per_layer_call": s_total, "matches_single_gpu_layer": s_matches,
+                         "note": "grouped FFNs with moe_config.streaming = 1 (tile flags)"},
            "nvlink": {"remote_pairs_per_rank_max": max(remote),
                       "bytes_per_rank_each_way_max": nv_b,
                       "dispatch_bound_ms_at_770_gbs": nv_b / 770e9 * 1e3,

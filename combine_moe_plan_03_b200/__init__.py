@@ -114,7 +114,7 @@ def _load():
         "moe_ep_bind": [P(moe_shape), i32, vp, P(moe_ep_plan)],
         "moe_ep_layout": [P(moe_shape), i32, i32, vp, P(moe_ep_plan), vp, vp],
         "moe_ep_dispatch": [P(moe_shape), i32, i32, vp, P(moe_plan_buffers), P(moe_ep_plan),
-                            P(vp), vp],
+                            P(vp), P(vp), vp],
         "moe_ep_combine": [P(moe_shape), i32, i32, P(vp), vp, P(moe_plan_buffers),
                            P(moe_ep_plan), vp, vp],
     }
@@ -227,10 +227,11 @@ def moe_ep_layout(shape, R: int, rank: int, all_counts_ptr: int, ep: moe_ep_plan
 
 
 def moe_ep_dispatch(shape, R: int, rank: int, x_ptr: int, own: moe_plan_buffers,
-                    ep: moe_ep_plan, pool_ptrs, stream: int = 0) -> None:
+                    ep: moe_ep_plan, pool_ptrs, stream: int = 0, flag_ptrs=None) -> None:
+    flags = _ptr_array(flag_ptrs) if flag_ptrs is not None else None
     _check("moe_ep_dispatch", _lib.moe_ep_dispatch(ctypes.byref(_shape(shape)), R, rank, x_ptr,
                                                    ctypes.byref(own), ctypes.byref(ep),
-                                                   _ptr_array(pool_ptrs), stream or None))
+                                                   _ptr_array(pool_ptrs), flags, stream or None))
 
 
 def moe_ep_combine(shape, R: int, rank: int, ypool_ptrs, topk_w_ptr: int,

@@ -12,10 +12,13 @@
 //                       and over this rank's E_r experts (the grouped FFN's plan)
 //   plan_scan_kernel    (plan.cu) twice: exclusive scans over the sources, padded offsets,
 //                       the FFN's tile and row-chunk tables
-//   ep_pad_kernel       zeroes this rank's padding rows
+//   ep_pad_kernel       zeroes this rank's padding rows, counting each on its tile's flag
 //   ep_dispatch_kernel  source side: x[t] staged once in shared memory, then stored (16-byte
 //                       vectors, every lane) into the pool rows of its k pairs, on whichever
-//                       rank owns each pair's expert (peer pointers)
+//                       rank owns each pair's expert (peer pointers); then each stored row is
+//                       counted on its owner's tile flag (release at system scope), so a
+//                       streaming grouped FFN on the owner takes a pool tile as soon as its
+//                       rows from every rank and its padding have landed (flag = tile rows)
 //   ep_combine_kernel   source side: out[t] = bf16(sum_j w[t, j] ypool_{owner}[row]) with the
 //                       k rows gathered from their owners' ypools (peer loads), the same fp32
 //                       FMA chain as combine.cu
@@ -33,6 +36,10 @@ constexpr int kEpThreads = 256;
 
 struct EpPeers {
   uint8_t *base[kMaxEpRanks];
+};
+
+struct EpFlags {
+  uint32_t *base[kMaxEpRanks];   // each rank's pool tile flags (ep->local.tile_flags); or none
 };
 
 __global__ void __launch_bounds__(kEpThreads)
@@ -66,16 +73,18 @@ __global__ void __launch_bounds__(kEpThreads)
 }
 
 // Padding rows of this rank's pool: [offsets[e] + counts[e], offsets[e + 1]) per local expert,
-// every expert's rows spread over the whole grid (16-byte stores).
+// one row per block at a time (16-byte stores); each zeroed row counts one on its tile's flag.
 __global__ void __launch_bounds__(kEpThreads)
     ep_pad_kernel(uint4 *__restrict__ pool, int32_t hv, const int32_t *__restrict__ counts,
-                  const int32_t *__restrict__ offsets, int32_t Er) {
-  const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t gsz = (int64_t)gridDim.x * blockDim.x;
+                  const int32_t *__restrict__ offsets, int32_t Er, uint32_t *__restrict__ flags,
+                  int32_t tile) {
   for (int e = 0; e < Er; ++e) {
     const int64_t r0 = offsets[e] + counts[e], r1 = offsets[e + 1];
-    const int64_t n = (r1 - r0) * hv;
-    for (int64_t i = gtid; i < n; i += gsz) pool[r0 * hv + i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t r = r0 + blockIdx.x; r < r1; r += gridDim.x) {  // uniform across the block
+      for (int i = threadIdx.x; i < hv; i += blockDim.x) pool[r * hv + i] = make_uint4(0u, 0u, 0u, 0u);
+      __syncthreads();
+      if (threadIdx.x == 0) red_release_sys_add(flags + r / tile, 1u);
+    }
   }
 }
 
@@ -114,7 +123,7 @@ __global__ void __launch_bounds__(kEpThreads)
                        const int32_t *__restrict__ g_src_base, int64_t max_rows,
                        const int32_t *__restrict__ own_counts,
                        const int32_t *__restrict__ g_counts, int32_t *__restrict__ status,
-                       const EpPeers pools) {
+                       const EpPeers pools, const EpFlags flags, bool signal) {
   extern __shared__ uint4 row[];  // [hv]: x[t]
   __shared__ int32_t s_row[kMaxTopK], s_dst[kMaxTopK];
   if (blockIdx.x == 0) {
@@ -144,6 +153,10 @@ __global__ void __launch_bounds__(kEpThreads)
       for (int i = threadIdx.x; i < hv; i += blockDim.x) dst[i] = row[i];
     }
     __syncthreads();
+    // every thread's stores of the token's rows precede the barrier; the release at system
+    // scope passes them on to the owner's acquire of the flag
+    if (signal && threadIdx.x < k && s_row[threadIdx.x] >= 0)
+      red_release_sys_add(flags.base[s_dst[threadIdx.x]] + s_row[threadIdx.x] / tile, 1u);
   }
 }
 
@@ -211,6 +224,12 @@ EpPeers peers_of(void *const *ptrs, int32_t R) {
   return p;
 }
 
+EpFlags flags_of(uint32_t *const *ptrs, int32_t R) {
+  EpFlags f{};
+  for (int i = 0; ptrs != nullptr && i < R && i < kMaxEpRanks; ++i) f.base[i] = ptrs[i];
+  return f;
+}
+
 }  // namespace
 
 cudaError_t launch_ep_layout(const moe_shape &rank_shape, int32_t R, int32_t rank,
@@ -236,17 +255,18 @@ cudaError_t launch_ep_layout(const moe_shape &rank_shape, int32_t R, int32_t ran
                             ep.local.offsets, ep.local.tile_expert, ep.local.mblk,
                             ep.local.meta, ep.local.status, st);
   if (e != cudaSuccess) return e;
-  if (cudaMemsetAsync(ep.local.tile_flags, 0, sizeof(uint32_t) * (size_t)lg.n_tiles, st) !=
-      cudaSuccess)
-    return cudaErrorUnknown;
+  // the tile flags are not reset here: other ranks' dispatches may already be counting on
+  // them; moe_ep_combine resets them after this rank's grouped FFN has used them
   ep_pad_kernel<<<num_sms * 2, kEpThreads, 0, st>>>(
-      static_cast<uint4 *>(pool), rank_shape.H / 8, ep.local.counts, ep.local.offsets, Er);
+      static_cast<uint4 *>(pool), rank_shape.H / 8, ep.local.counts, ep.local.offsets, Er,
+      reinterpret_cast<uint32_t *>(ep.local.tile_flags), rank_shape.tile);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ep_dispatch(const moe_shape &rank_shape, int32_t R, int32_t rank,
                                const void *x, const moe_plan_buffers &own, const moe_ep_plan &ep,
-                               void *const *pools, int num_sms, cudaStream_t st) {
+                               void *const *pools, uint32_t *const *tile_flags, int num_sms,
+                               cudaStream_t st) {
   if (rank_shape.T == 0) return cudaSuccess;
   const int hv = rank_shape.H / 8;
   const size_t smem = (size_t)hv * sizeof(uint4);  // one row of x (H <= 38,720 by check_shape)
@@ -260,7 +280,7 @@ cudaError_t launch_ep_dispatch(const moe_shape &rank_shape, int32_t R, int32_t r
       static_cast<const uint4 *>(x), rank_shape.T, rank_shape.k, hv, R, rank_shape.E / R,
       rank_shape.tile, rank, own.pool_row, own.tile_expert, own.offsets, ep.offsets,
       ep.src_base, plan_geom(ep_local_shape(rank_shape, R)).pmax, own.counts, ep.counts,
-      own.status, peers_of(pools, R));
+      own.status, peers_of(pools, R), flags_of(tile_flags, R), tile_flags != nullptr);
   return cudaGetLastError();
 }
 
@@ -268,7 +288,12 @@ cudaError_t launch_ep_combine(const moe_shape &rank_shape, int32_t R, int32_t ra
                               void *const *ypools, const float *topk_w,
                               const moe_plan_buffers &own, const moe_ep_plan &ep, void *out,
                               int num_sms, cudaStream_t st) {
-  if (rank_shape.T == 0) return cudaSuccess;
+  // this rank's pool tile flags, counted by every rank's dispatch and used by this rank's
+  // grouped FFN, back to zero for the next layer call (also when this rank has no tokens)
+  cudaError_t e = cudaMemsetAsync(
+      ep.local.tile_flags, 0,
+      sizeof(uint32_t) * (size_t)plan_geom(ep_local_shape(rank_shape, R)).n_tiles, st);
+  if (e != cudaSuccess || rank_shape.T == 0) return e;
   int64_t grid = (int64_t)num_sms * 8;
   if (grid > rank_shape.T) grid = rank_shape.T;
   ep_combine_kernel<<<(int)grid, kEpThreads, 0, st>>>(

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int32_t t = row0 / prm.tile; t <= t_end && !*abort; ++t) {
             const uint64_t t0 = globaltimer_ns();
             uint32_t it = 0;
-            while (ld_acquire_gpu(prm.flags + t) < (uint32_t)prm.tile) {
+            while (ld_acquire_sys(prm.flags + t) < (uint32_t)prm.tile) {
               if ((++it & 63u) == 0 && (*abort || globaltimer_ns() - t0 > prm.timeout_ns)) {
                 raise_abort(abort, prm.status, MOE_ERR_FLAG_TIMEOUT, t);
                 break;

@@ -597,14 +597,18 @@ int check_ep_call(const moe_shape *s, int32_t R, int32_t rank, const moe_plan_bu
 
 int moe_ep_dispatch(const moe_shape *s, int32_t R, int32_t rank, const void *x,
                     const moe_plan_buffers *own, const moe_ep_plan *ep, void *const *pools,
-                    void *stream) {
+                    uint32_t *const *tile_flags, void *stream) {
   int rc = check_ep_call(s, R, rank, own, ep, pools);
   if (rc != MOE_OK) return rc;
   if (x == nullptr && s->T > 0) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x)) return MOE_ERR_MISALIGNED;
+  if (tile_flags != nullptr)
+    for (int i = 0; i < R; ++i)
+      if (tile_flags[i] == nullptr || (reinterpret_cast<uintptr_t>(tile_flags[i]) & 3u) != 0)
+        return MOE_ERR_INVALID_ARG;
   int nsm;
   if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
-  if (launch_ep_dispatch(*s, R, rank, x, *own, *ep, pools, nsm,
+  if (launch_ep_dispatch(*s, R, rank, x, *own, *ep, pools, tile_flags, nsm,
                          static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;

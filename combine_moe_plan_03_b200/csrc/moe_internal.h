@@ -85,7 +85,8 @@ cudaError_t launch_ep_layout(const moe_shape &rank_shape, int32_t R, int32_t ran
                              int num_sms, cudaStream_t st);
 cudaError_t launch_ep_dispatch(const moe_shape &rank_shape, int32_t R, int32_t rank,
                                const void *x, const moe_plan_buffers &own, const moe_ep_plan &ep,
-                               void *const *pools, int num_sms, cudaStream_t st);
+                               void *const *pools, uint32_t *const *tile_flags, int num_sms,
+                               cudaStream_t st);
 cudaError_t launch_ep_combine(const moe_shape &rank_shape, int32_t R, int32_t rank,
                               void *const *ypools, const float *topk_w,
                               const moe_plan_buffers &own, const moe_ep_plan &ep, void *out,

@@ -379,8 +379,10 @@ int moe_hbm_probe(void *dst, const void *src, size_t bytes, int32_t mode, void *
  *      use of its pool
  *   3. moe_ep_layout(rank_shape, R, r, all_counts, ep, pool)   every rank's pool layout, this
  *      rank's pool plan (ep->local) and zero padding rows
- *   4. moe_ep_dispatch(..., pools)                 x rows into their owners' pools
- *   5. a barrier over the ranks (every rank's dispatch done)
+ *   4. moe_ep_dispatch(..., pools, tile_flags)     x rows into their owners' pools, each row
+ *      counted on its owner's tile flag
+ *   5. a barrier over the ranks (every rank's dispatch done); or none, with a streaming FFN
+ *      (moe_config.streaming = 1) that takes each pool tile once its flag is full
  *   6. moe_grouped_ffn(local_shape, pool, W1 / W2 of this rank's experts, &ep->local, ...)
  *      with local_shape from moe_ep_local_shape (T = R * rank T, E = E / R)
  *   7. a barrier (every rank's FFN done)
@@ -419,13 +421,21 @@ int moe_ep_layout(const moe_shape *rank_shape, int32_t R, int32_t rank,
                   const int32_t *all_counts, const moe_ep_plan *ep, void *pool, void *stream);
 
 /* Step 4: pool_{owner(e)}[row of pair f] = x[t] for every live pair f = t*k + j of this rank
- * (own: this rank's moe_plan). This rank's row of all_counts must equal own's counts, else
+ * (own: this rank's moe_plan). tile_flags: NULL, or a host array of R device pointers, each
+ * rank's ep->local.tile_flags (mapped for peer access); then every stored row adds one to
+ * its owner's tile flag (release at system scope) after the row's stores, and the owner's
+ * moe_ep_layout adds one per padding row, so a tile's flag reaches the tile height when all
+ * its rows have landed: a grouped FFN with moe_config.streaming = 1 on the owner takes each
+ * tile then (its waits acquire at system scope). The flags must be zero before the first
+ * call (a zeroed arena); moe_ep_combine zeroes the rank's own flags again after its FFN has
+ * used them, so no reset races with the next call's dispatches from other ranks (which
+ * follow the next count exchange). This rank's row of all_counts must equal own's counts, else
  * MOE_ERR_POOL_OVERFLOW (aux = expert) in own's status word. A row that all_counts would
  * place outside the owner's pool is skipped and reported the same way (aux = pair id);
  * moe_ep_combine checks rows the same way. */
 int moe_ep_dispatch(const moe_shape *rank_shape, int32_t R, int32_t rank, const void *x,
                     const moe_plan_buffers *own, const moe_ep_plan *ep, void *const *pools,
-                    void *stream);
+                    uint32_t *const *tile_flags, void *stream);
 
 /* Step 8: out[t] = bf16(sum_j topk_w[t,j] * ypool_{owner}[row of pair t*k + j]), fp32 FMA
  * chain over j ascending (moe_combine's arithmetic); dropped pairs add nothing. */

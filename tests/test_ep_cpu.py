@@ -51,6 +51,9 @@ def test_ep_calls_check_ranks_and_pointers_on_the_host():
     with pytest.raises(moe.MoEError) as ei:              # a missing peer pool
         moe.moe_ep_dispatch(rs, 2, 0, 1 << 26, own, ep, [1 << 27, 0])
     assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoEError) as ei:              # a misaligned tile-flag pointer
+        moe.moe_ep_dispatch(rs, 2, 0, 1 << 26, own, ep, [1 << 27, 1 << 28], 0, [1 << 20, 2])
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
     with pytest.raises(moe.MoEError) as ei:              # a misaligned peer ypool
         moe.moe_ep_combine(rs, 2, 1, [1 << 27, (1 << 28) + 8], 1 << 26, own, ep, 1 << 25)
     assert ei.value.code == moe.MOE_ERR_MISALIGNED

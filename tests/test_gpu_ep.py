@@ -16,7 +16,7 @@ import synth_inputs as si
 pytestmark = pytest.mark.gpu
 
 
-def _run_ep(cfg, R, drop=0.0, check_pools=True):
+def _run_ep(cfg, R, drop=0.0, check_pools=True, streaming=0, calls=1):
     import combine_moe_plan_03_b200 as moe
     from gpu_helpers import DEV, bf16_dev, bf16_host, f32_dev, i32_dev, weights_dev
     W1, W2 = weights_dev(cfg)
@@ -45,27 +45,38 @@ def _run_ep(cfg, R, drop=0.0, check_pools=True):
             for _ in range(R)]
     dx = [bf16_dev(x) for x in xs]
     dw = [f32_dev(w) for w in ws]
-    # 1. each rank's own plan over the E global experts
-    for r in range(R):
-        moe.moe_plan(rs, i32_dev(idxs[r]).data_ptr(), own[r].plan, 0, 0)
-    # 2. the all-gather of the counts (here: stacking the ranks' rows)
-    C = torch.stack([own[r].plan_view("counts")[: cfg.E] for r in range(R)]).contiguous()
     pool_ptrs = [p.data_ptr() for p in pools]
     ypool_ptrs = [p.data_ptr() for p in ypools]
-    # 3.-8. layout, dispatch into the owners' pools, each rank's FFN, combine from the owners
-    for r in range(R):
-        moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pools[r].data_ptr(), 0)
-    for r in range(R):
-        moe.moe_ep_dispatch(rs, R, r, dx[r].data_ptr(), own[r].plan, ep[r], pool_ptrs, 0)
-    for r in range(R):
-        w1 = W1[r * Er:(r + 1) * Er].contiguous()
-        w2 = W2[r * Er:(r + 1) * Er].contiguous()
-        moe.moe_grouped_ffn(ls, pools[r].data_ptr(), w1.data_ptr(), w2.data_ptr(), ep[r].local,
-                            acts[r].data_ptr(), ypools[r].data_ptr(), moe.moe_config(), 0)
-    for r in range(R):
-        moe.moe_ep_combine(rs, R, r, ypool_ptrs, dw[r].data_ptr(), own[r].plan, ep[r],
-                           outs[r].data_ptr(), 0)
+    # with streaming, every stored row is counted on its owner's tile flag and each rank's
+    # GEMM A takes a tile once its flag is full (here all dispatches precede the FFNs in
+    # stream order, so the flags are full when it looks)
+    flag_ptrs = [e_.local.tile_flags for e_ in ep] if streaming else None
+    w1s = [W1[r * Er:(r + 1) * Er].contiguous() for r in range(R)]
+    w2s = [W2[r * Er:(r + 1) * Er].contiguous() for r in range(R)]
+    for _ in range(calls):
+        # 1. each rank's own plan over the E global experts
+        for r in range(R):
+            moe.moe_plan(rs, i32_dev(idxs[r]).data_ptr(), own[r].plan, 0, 0)
+        # 2. the all-gather of the counts (here: stacking the ranks' rows)
+        C = torch.stack([own[r].plan_view("counts")[: cfg.E] for r in range(R)]).contiguous()
+        # 3.-8. layout, dispatch into the owners' pools, each rank's FFN, combine from the owners
+        for r in range(R):
+            moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pools[r].data_ptr(), 0)
+        for r in range(R):
+            moe.moe_ep_dispatch(rs, R, r, dx[r].data_ptr(), own[r].plan, ep[r], pool_ptrs, 0,
+                                flag_ptrs)
+        for r in range(R):
+            moe.moe_grouped_ffn(ls, pools[r].data_ptr(), w1s[r].data_ptr(), w2s[r].data_ptr(),
+                                ep[r].local, acts[r].data_ptr(), ypools[r].data_ptr(),
+                                moe.moe_config(streaming=streaming), 0)
+        for r in range(R):
+            moe.moe_ep_combine(rs, R, r, ypool_ptrs, dw[r].data_ptr(), own[r].plan, ep[r],
+                               outs[r].data_ptr(), 0)
     torch.cuda.synchronize()
+    for r in range(R):   # moe_ep_combine leaves the rank's tile flags at zero for the next call
+        n_tiles = rows // cfg.tile
+        off = ep[r].local.tile_flags - ep_arena[r].data_ptr()
+        assert not ep_arena[r][off:off + 4 * n_tiles].any(), f"rank {r} flags"
     for r in range(R):
         assert moe.moe_get_status(own[r].plan)[0] == 0
         assert moe.moe_get_status(ep[r].local)[0] == 0
@@ -100,13 +111,14 @@ EP_SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("streaming", [0, 1])
 @pytest.mark.parametrize("shape", EP_SHAPES, ids=[s[0] for s in EP_SHAPES])
 @pytest.mark.parametrize("drop", [0.0, 0.2])
-def test_ep_emulated_ranks_match_single_gpu_and_oracle(shape, drop):
+def test_ep_emulated_ranks_match_single_gpu_and_oracle(shape, drop, streaming):
     from gpu_helpers import assert_layer_close, to_f64
     name, T, H, I, E, k, tile, R = shape
     cfg = si.custom(name, T=T, H=H, I=I, E=E, k=k, tile=tile, seed=555 + T)
-    xs, idxs, ws, res = _run_ep(cfg, R, drop=drop)
+    xs, idxs, ws, res = _run_ep(cfg, R, drop=drop, streaming=streaming, calls=1 + streaming)
     W1h = [si.make_w1_expert(cfg, e) for e in range(E)]
     W2h = [si.make_w2_expert(cfg, e) for e in range(E)]
     for r, (ep_out, single_out) in enumerate(res):
@@ -171,7 +183,8 @@ def test_ep_counts_that_disagree_with_the_plans_are_reported_not_followed(bad):
         moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pools[r].data_ptr(), 0)
     for r in range(R):
         moe.moe_ep_dispatch(rs, R, r, xs[r].data_ptr(), own[r].plan, ep[r],
-                            [p.data_ptr() for p in pools], 0)
+                            [p.data_ptr() for p in pools], 0,
+                            [e_.local.tile_flags for e_ in ep])
     for r in range(R):
         moe.moe_ep_combine(rs, R, r, [p.data_ptr() for p in ypools],
                            f32_dev(routs[r][1]).data_ptr(), own[r].plan, ep[r],
@@ -218,3 +231,50 @@ def test_bench_ep_section_matches_single_gpu_layer():
     assert res["ms_per_layer_call"] > 0 and res["dispatch_gbs"] > 0 and res["combine_gbs"] > 0
     assert res["nvlink"]["remote_pairs_per_rank_max"] <= cfg.T // 4 * cfg.k
     buf.close()
+
+
+def test_ep_streaming_ffn_times_out_without_the_dispatch_flags():
+    """A host-made failure: dispatch without tile flags, then a streaming grouped FFN on the
+    owner: its pool tiles never fill (only the padding rows were counted), GEMM A's bounded
+    wait reports MOE_ERR_FLAG_TIMEOUT, and after moe_clear_status a non-streaming FFN on the
+    same context is correct."""
+    import combine_moe_plan_03_b200 as moe
+    from gpu_helpers import DEV, bf16_dev, i32_dev, weights_dev
+    R = 2
+    cfg = si.custom("ep-to", T=128, H=256, I=128, E=4, k=2, tile=64, seed=5)
+    W1, W2 = weights_dev(cfg)
+    rs = moe.moe_shape(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    ls = moe.moe_ep_local_shape(rs, R)
+    rows = moe.moe_ep_pool_rows(rs, R)
+    own = [moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile, identity=True)
+           for _ in range(R)]
+    arenas = [torch.zeros(moe.moe_ep_arena_bytes(rs, R), dtype=torch.uint8, device=DEV)
+              for _ in range(R)]
+    ep = [moe.moe_ep_bind(rs, R, a.data_ptr()) for a in arenas]
+    pools = [torch.empty((rows, cfg.H), dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    act = torch.empty((rows, cfg.I), dtype=torch.bfloat16, device=DEV)
+    ypool = torch.empty((rows, cfg.H), dtype=torch.bfloat16, device=DEV)
+    xs = [bf16_dev(si.make_x(cfg, r)) for r in range(R)]
+    for r in range(R):
+        moe.moe_plan(rs, i32_dev(si.make_routing(cfg, r)[0]).data_ptr(), own[r].plan, 0, 0)
+    C = torch.stack([own[r].plan_view("counts")[: cfg.E] for r in range(R)]).contiguous()
+    for r in range(R):
+        moe.moe_ep_layout(rs, R, r, C.data_ptr(), ep[r], pools[r].data_ptr(), 0)
+    for r in range(R):
+        moe.moe_ep_dispatch(rs, R, r, xs[r].data_ptr(), own[r].plan, ep[r],
+                            [p.data_ptr() for p in pools], 0)        # no flags
+    Er = cfg.E // R
+    w1, w2 = W1[:Er].contiguous(), W2[:Er].contiguous()
+    moe.moe_grouped_ffn(ls, pools[0].data_ptr(), w1.data_ptr(), w2.data_ptr(), ep[0].local,
+                        act.data_ptr(), ypool.data_ptr(),
+                        moe.moe_config(streaming=1, wait_timeout_us=2000), 0)
+    torch.cuda.synchronize()
+    code, aux = moe.moe_get_status(ep[0].local)
+    assert code == moe.MOE_ERR_FLAG_TIMEOUT, (moe.moe_strerror(code), aux)
+    moe.moe_clear_status(ep[0].local, 0)
+    moe.moe_grouped_ffn(ls, pools[0].data_ptr(), w1.data_ptr(), w2.data_ptr(), ep[0].local,
+                        act.data_ptr(), ypool.data_ptr(), moe.moe_config(), 0)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(ep[0].local)[0] == 0
+    for b in own:
+        b.close()
