@@ -537,7 +537,36 @@ def time_backward(moe, buf, cfg, dev, world, local, x, idx, w, W1, W2, W1u, W2u,
                                        "of d(g, u) read + of d(pool) written"}
     cb_bytes = T * H * 2 + 2 * pairs * H * 2 + T * cfg.k * 8
     db_bytes = pairs * H * 2 + T * H * 2
+    # the backward's mirrored overlaps against the serial order, alternating on this GPU:
+    # early dispatch backward (folded into backward A) and the streaming combine backward
+    # (tile order on the communicate stream, backward Y taking tiles on the compute stream)
+    overlap = None
+    if world == 1:
+        def bwd_ms(c_, n=3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(buf.compute)
+            for _ in range(n):
+                buf.backward(dy, w, W1u, W2u, c_, dx=gx, dw=gw, dW1=gW1, dW2=gW2)
+            e1.record(buf.compute)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / n
+        variants = {"serial": moe.moe_config(), "early_dispatch_bwd": moe.moe_config(early_combine=1),
+                    "streaming_combine_bwd": moe.moe_config(streaming=1),
+                    "both": moe.moe_config(streaming=1, early_combine=1)}
+        for c_ in variants.values():
+            bwd_ms(c_, 1)
+        acc = {k: [] for k in variants}
+        for _ in range(3):
+            for k_, c_ in variants.items():
+                acc[k_].append(bwd_ms(c_))
+        code, aux = moe.moe_get_status(buf.plan)
+        if code != 0:
+            raise RuntimeError(f"device status after the backward A/B: {moe.moe_strerror(code)}")
+        overlap = {"ms_per_call": {k: float(np.median(v)) for k, v in acc.items()},
+                   "note": "median of 3 alternating rounds of 3 calls each, with weight gradients"}
     return {"ms_per_call": total, "tokens_per_s": world * T / (total / 1e3),
+            "overlap_ab": overlap,
             "train_step": {"forward_saving_gate_up_ms": fwd_ms,
                            "forward_gemm_a_ms": fwd_gemm_a, "backward_ms": total,
                            "ms": fwd_ms + total,

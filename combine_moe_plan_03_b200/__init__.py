@@ -96,6 +96,8 @@ def _load():
                         P(moe_config), vp, vp, vp, vp],
         "moe_backward": [P(moe_shape), vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp, vp, vp,
                          vp, vp, vp, vp, vp, P(moe_config), vp],
+        "moe_backward_streams": [P(moe_shape), vp, vp, vp, vp, P(moe_plan_buffers), vp, vp, vp,
+                                 vp, vp, vp, vp, vp, vp, vp, P(moe_config), vp, vp, vp, vp],
         "moe_events_create": [P(vp), i32],
         "moe_timing_events_create": [P(vp), i32],
         "moe_event_elapsed_ms": [vp, vp, P(ctypes.c_float)],
@@ -134,7 +136,7 @@ _lib = _load()
 # Names exported by include/moe.h, in declaration order.
 EXPORTS = ["moe_route", "moe_route_plan", "moe_packed_weight_bytes", "moe_pack_weights", "moe_pool_rows_max", "moe_plan_arena_bytes", "moe_plan_bind", "moe_plan",
            "moe_dispatch", "moe_grouped_ffn", "moe_grouped_ffn_combine", "moe_combine",
-           "moe_forward", "moe_backward",
+           "moe_forward", "moe_backward", "moe_backward_streams",
            "moe_events_create",
            "moe_events_destroy", "moe_timing_events_create", "moe_event_elapsed_ms",
            "moe_get_status", "moe_clear_status", "moe_strerror", "moe_plan_noalloc",
@@ -346,6 +348,20 @@ def moe_backward(shape, dy_ptr: int, topk_w_ptr: int, w1_ptr: int, w2_ptr: int,
         w2_ptr or None, ctypes.byref(plan), pool_ptr or None, act_ptr or None, ypool_ptr or None,
         gu_ptr or None, dgu_ptr or None, dpool_ptr or None, dx_ptr or None, dw_ptr or None,
         dw1_ptr or None, dw2_ptr or None, ctypes.byref(cfg), stream or None))
+
+
+def moe_backward_streams(shape, dy_ptr: int, topk_w_ptr: int, w1_ptr: int, w2_ptr: int,
+                         plan: moe_plan_buffers, pool_ptr: int, act_ptr: int, ypool_ptr: int,
+                         gu_ptr: int, dgu_ptr: int, dpool_ptr: int, dx_ptr: int, dw_ptr: int,
+                         dw1_ptr: int, dw2_ptr: int, cfg: moe_config | None, comm_stream: int,
+                         compute_stream: int, ev_a: int, ev_b: int) -> None:
+    cfg = cfg or moe_config()
+    _check("moe_backward_streams", _lib.moe_backward_streams(
+        ctypes.byref(_shape(shape)), dy_ptr or None, topk_w_ptr or None, w1_ptr or None,
+        w2_ptr or None, ctypes.byref(plan), pool_ptr or None, act_ptr or None, ypool_ptr or None,
+        gu_ptr or None, dgu_ptr or None, dpool_ptr or None, dx_ptr or None, dw_ptr or None,
+        dw1_ptr or None, dw2_ptr or None, ctypes.byref(cfg), comm_stream or None,
+        compute_stream or None, ev_a or None, ev_b or None))
 
 
 def moe_events_create(n: int) -> list[int]:

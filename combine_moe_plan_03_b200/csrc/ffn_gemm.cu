@@ -595,7 +595,7 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
                         const moe_plan_buffers &p, const void *pool, void *act,
                         void *dypool_dpool, void *gu, void *dgu, void *dW1, void *dW2,
                         const moe_config &cfg, int num_sms, cudaStream_t st,
-                        cudaEvent_t const *tev) {
+                        cudaEvent_t const *tev, void *early_dx, cudaEvent_t combine_done) {
   const PlanGeom g = plan_geom(s);
   if (g.pmax == 0) {
     // no rows at all (T = 0): the weight gradients are zero, the phases empty
@@ -668,7 +668,19 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   y.aux = static_cast<const uint16_t *>(gu);
   y.aux_ld = 2 * s.I;
   y.aux_off = s.I;
-  if (launch_ffn_pair(2, true, tw2_k, tx_dy, y, clusters, st) != cudaSuccess) return MOE_ERR_CUDA;
+  // streaming: the combine backward fills dypool tile by tile on other SMs and raises the
+  // tiles' flags; backward Y takes a chunk once the flags of its tiles are full
+  y.streaming = cfg.streaming;
+  int clusters_y = clusters;
+  if (cfg.streaming) {
+    clusters_y = (num_sms - kStreamDispatchSMs) / 2;
+    if (clusters_y > clusters) clusters_y = clusters;
+    if (clusters_y < 1) clusters_y = 1;
+  }
+  if (launch_ffn_pair(2, true, tw2_k, tx_dy, y, clusters_y, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (combine_done != nullptr && cudaStreamWaitEvent(st, combine_done, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[3], st) != cudaSuccess) return MOE_ERR_CUDA;
 
   // dW2 = act^T . dypool per expert (before backward A overwrites dypool)
@@ -693,7 +705,20 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   a.n_out1 = s.H;
   a.k_rows = s.H;
   a.sched = p.meta + 4;
-  if (launch_ffn_pair(1, true, tw1_k, tx_dgu, a, clusters, st) != cudaSuccess)
+  const bool early = early_dx != nullptr;
+  if (early) {
+    // dx[t] = bf16(sum_j dpool[pool_row[t, j]]) for each token as soon as its rows are
+    // stored (unit weights: no topk_w), in the CTAs that finished their GEMM work
+    a.row_src = p.row_src;
+    a.pool_row = p.pool_row;
+    a.topk_w = nullptr;
+    a.tok_pending = p.tok_pending;
+    a.ready = p.ready;
+    a.comb_out = static_cast<uint16_t *>(early_dx);
+    a.T = s.T;
+    a.k = s.k;
+  }
+  if (launch_ffn_pair(1, true, tw1_k, tx_dgu, a, clusters, st, early) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;
 

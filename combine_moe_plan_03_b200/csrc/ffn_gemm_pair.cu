@@ -148,7 +148,7 @@ __device__ void early_combine_drain(const FfnParams &prm, int lane, uint64_t tim
     float my_w = 0.0f;
     if (lane < prm.k) {
       my_row = prm.pool_row[t * prm.k + lane];
-      my_w = prm.topk_w[t * prm.k + lane];
+      my_w = prm.topk_w != nullptr ? prm.topk_w[t * prm.k + lane] : 1.0f;  // none: unit weights
     }
     // every lane runs every iteration (the shuffles below need the whole warp); a lane's
     // vectors past the row's end are masked
@@ -194,7 +194,7 @@ template <int kMode, bool kAK, bool kEarly>
 __global__ void __launch_bounds__(threads_for(kEarly), 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                          const __grid_constant__ CUtensorMap tm_x, const FfnParams prm) {
-  static_assert(!kEarly || (kMode == 1 && !kAK), "early combine is GEMM Y's");
+  static_assert(!kEarly || kMode == 1, "early combine folds into GEMM Y or backward A");
   constexpr int kSchedReaders = sched_readers(kEarly);
   extern __shared__ uint8_t smem_raw[];
   // The same offsets in both CTAs (the MMA reads both CTAs' operands at one address).
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
         const int32_t half_rows = ((rows + 15) & ~15) >> 1;   // N / 2
         const int nbox = (half_rows + kRowBox - 1) / kRowBox;  // same in both CTAs
         const int32_t xrow0 = row0 + (int32_t)rank * half_rows;
-        if ((kMode == 0 || kMode == 3) && prm.streaming) {
+        if ((kMode == 0 || kMode == 2 || kMode == 3) && prm.streaming) {
           const int32_t t_end = (row0 + rows - 1) / prm.tile;
           for (int32_t t = row0 / prm.tile; t <= t_end && !*abort; ++t) {
             const uint64_t t0 = globaltimer_ns();
@@ -793,11 +793,14 @@ cudaError_t launch_ffn_pair(int mode, bool a_kmajor, const CUtensorMap &tw,
                             const CUtensorMap &tx, const FfnParams &prm, int clusters,
                             cudaStream_t st, bool early) {
   if (early) {
-    if (mode != 1 || a_kmajor) return cudaErrorInvalidValue;
+    // GEMM Y (weights MN-major) or backward A (K-major) with the combine folded in
+    if (mode != 1) return cudaErrorInvalidValue;
     // the extra signal warp: as many clusters as fit with it (at most those asked for)
-    const int fit = max_clusters_mode<1, false, true>();
+    const int fit = a_kmajor ? max_clusters_mode<1, true, true>() : max_clusters_mode<1, false, true>();
     if (fit < 1) return cudaErrorInvalidConfiguration;
-    return launch_mode<1, false, true>(tw, tx, prm, clusters < fit ? clusters : fit, st);
+    const int c = clusters < fit ? clusters : fit;
+    return a_kmajor ? launch_mode<1, true, true>(tw, tx, prm, c, st)
+                    : launch_mode<1, false, true>(tw, tx, prm, c, st);
   }
   if (!a_kmajor)
     return mode == 0   ? launch_mode<0, false>(tw, tx, prm, clusters, st)

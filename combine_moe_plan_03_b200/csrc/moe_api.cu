@@ -326,10 +326,18 @@ int moe_combine(const moe_shape *s, const void *ypool, const float *topk_w,
   return MOE_OK;
 }
 
-int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
-                 const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
-                 const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
-                 void *dW1, void *dW2, const moe_config *cfg, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward on one stream (comm == compute, no events) or, with cfg->streaming, with the
+// combine backward on comm in pool-tile order while backward Y on compute takes the tiles
+// as their flags fill (the mirror of the streaming forward).
+int backward_entry(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
+                   const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
+                   const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
+                   void *dW1, void *dW2, const moe_config *cfg, cudaStream_t comm,
+                   cudaStream_t st, cudaEvent_t ev_a, cudaEvent_t ev_b) {
   int rc = check_shape(s, true);
   if (rc != MOE_OK) return rc;
   if ((rc = check_plan(p)) != MOE_OK) return rc;
@@ -344,22 +352,68 @@ int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const 
   moe_config c{};
   if (cfg != nullptr) c = *cfg;
   if ((rc = check_config(c)) != MOE_OK) return rc;
-  if (c.packed_weights || c.streaming || c.ffn_kernel == MOE_FFN_ONE_SM)
+  if (c.packed_weights || c.ffn_kernel == MOE_FFN_ONE_SM) return MOE_ERR_INVALID_ARG;
+  const bool streaming = c.streaming && s->T > 0;
+  if (c.streaming && (comm == st || ev_a == nullptr || ev_b == nullptr))
     return MOE_ERR_INVALID_ARG;
   int nsm;
   if ((rc = sm_count_cached(&nsm)) != MOE_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaEvent_t const *tev = reinterpret_cast<cudaEvent_t const *>(c.timing_events);
   if (tev != nullptr && cudaEventRecord(tev[0], st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_combine_backward(*s, dy, ypool, topk_w, *p, dpool, dw, nsm, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (tev != nullptr && cudaEventRecord(tev[1], st) != cudaSuccess) return MOE_ERR_CUDA;
+  // early_combine: the dispatch backward folds into backward A (the mirror of early combine)
+  const bool early = c.early_combine && s->T > 0;
+  if (early && (!p->tok_pending || !p->ready)) return MOE_ERR_INVALID_ARG;
+  if (early && launch_arm_tokens(*s, *p, nsm, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (streaming) {
+    // flags and dw cleared in stream order before either stream starts on them
+    const PlanGeom g = plan_geom(*s);
+    if (cudaMemsetAsync(p->tile_flags, 0, sizeof(uint32_t) * (size_t)g.n_tiles, st) !=
+            cudaSuccess ||
+        cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)s->T * s->k, st) != cudaSuccess ||
+        cudaEventRecord(ev_a, st) != cudaSuccess || cudaStreamWaitEvent(comm, ev_a, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (launch_combine_backward_tiles(*s, dy, ypool, topk_w, *p, dpool, dw, kStreamDispatchSMs * 4,
+                                      comm) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (tev != nullptr && cudaEventRecord(tev[1], comm) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaEventRecord(ev_b, comm) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    if (launch_combine_backward(*s, dy, ypool, topk_w, *p, dpool, dw, nsm, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (tev != nullptr && cudaEventRecord(tev[1], st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   if ((rc = launch_ffn_backward(*s, W1, W2, *p, pool, act, dpool, gu, dgu, dW1, dW2, c, nsm, st,
-                                tev)) != MOE_OK)
+                                tev, early ? dx : nullptr, streaming ? ev_b : nullptr)) != MOE_OK)
     return rc;
-  if (launch_combine(*s, dpool, nullptr, *p, dx, nsm, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!early && launch_combine(*s, dpool, nullptr, *p, dx, nsm, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[7], st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
+                 const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
+                 const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
+                 void *dW1, void *dW2, const moe_config *cfg, void *stream) {
+  if (cfg != nullptr && cfg->streaming) return MOE_ERR_INVALID_ARG;  // needs two streams
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return backward_entry(s, dy, topk_w, W1, W2, p, pool, act, ypool, gu, dgu, dpool, dx, dw, dW1,
+                        dW2, cfg, st, st, nullptr, nullptr);
+}
+
+int moe_backward_streams(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
+                         const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
+                         const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
+                         void *dW1, void *dW2, const moe_config *cfg, void *comm_stream,
+                         void *compute_stream, void *ev_a, void *ev_b) {
+  return backward_entry(s, dy, topk_w, W1, W2, p, pool, act, ypool, gu, dgu, dpool, dx, dw, dW1,
+                        dW2, cfg, static_cast<cudaStream_t>(comm_stream),
+                        static_cast<cudaStream_t>(compute_stream),
+                        static_cast<cudaEvent_t>(ev_a), static_cast<cudaEvent_t>(ev_b));
 }
 
 int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, const float *topk_w,

@@ -103,15 +103,26 @@ cudaError_t launch_dispatch(const moe_shape &s, const void *x, const moe_plan_bu
                             void *pool, int flags, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const moe_shape &s, const void *ypool, const float *topk_w,
                            const moe_plan_buffers &p, void *out, int num_sms, cudaStream_t st);
+cudaError_t launch_arm_tokens(const moe_shape &s, const moe_plan_buffers &p, int num_sms,
+                              cudaStream_t st);
+cudaError_t launch_combine_backward_tiles(const moe_shape &s, const void *dy, const void *ypool,
+                                          const float *topk_w, const moe_plan_buffers &p,
+                                          void *dypool, float *dw, int blocks, cudaStream_t st);
 cudaError_t launch_combine_backward(const moe_shape &s, const void *dy, const void *ypool,
                                     const float *topk_w, const moe_plan_buffers &p,
                                     void *dypool, float *dw, int num_sms, cudaStream_t st);
 // Returns MOE_OK or a MOE_ERR_* code. With dW1 / dW2 (and act) also the weight gradients.
+// early_dx: with cfg.early_combine, backward A also writes the dispatch backward into it
+// (the token counters armed by launch_arm_tokens first); nullptr: backward A alone.
+// combine_done: with cfg.streaming, the event after the tile-ordered combine backward on the
+// other stream; st waits for it once backward Y is queued (dW2 and the caller need all of
+// dypool and dw).
 int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
                         const moe_plan_buffers &p, const void *pool, void *act,
                         void *dypool_dpool, void *gu, void *dgu, void *dW1, void *dW2,
                         const moe_config &cfg, int num_sms, cudaStream_t st,
-                        cudaEvent_t const *tev);
+                        cudaEvent_t const *tev, void *early_dx = nullptr,
+                        cudaEvent_t combine_done = nullptr);
 // wgrad.cu: D [E, M, N] = per expert A_e^T B_e over its pool segment (rows past the live
 // ones must be zero in A and B); and the kernel that zeroes those rows of a buffer.
 int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, int32_t N,

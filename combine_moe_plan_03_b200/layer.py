@@ -10,9 +10,10 @@ import ctypes
 
 import torch
 
-from . import (moe_backward, moe_config, moe_events_create, moe_events_destroy, moe_forward,
-               moe_pack_weights, moe_packed_weight_bytes, moe_plan_arena_bytes, moe_plan_bind,
-               moe_pool_rows_max, moe_shape)
+from . import (moe_backward, moe_backward_streams, moe_config, moe_events_create,
+               moe_events_destroy, moe_forward, moe_pack_weights, moe_packed_weight_bytes,
+               moe_plan_arena_bytes, moe_plan_bind, moe_pool_rows_max, moe_shape)
+
 
 def ctypes_copy(dst: ctypes.Structure, src: ctypes.Structure) -> None:
     ctypes.memmove(ctypes.addressof(dst), ctypes.addressof(src), ctypes.sizeof(dst))
@@ -163,9 +164,16 @@ class MoELayerBuffers:
             dw = torch.empty((max(s.T, 1), s.k), dtype=torch.float32, device=self.device)[: s.T]
         for t, shp in ((dW1, (s.E, s.H, 2 * s.I)), (dW2, (s.E, s.I, s.H))):
             assert t is None or (t.dtype == bf and tuple(t.shape) == shp and t.is_contiguous())
-        moe_backward(s, dy.data_ptr(), topk_w.data_ptr(), W1.data_ptr(), W2.data_ptr(), self.plan,
-                     self.pool.data_ptr(), self.act.data_ptr(), self.ypool.data_ptr(),
-                     self.gu.data_ptr(), self.dgu.data_ptr(), self.dpool.data_ptr(),
-                     dx.data_ptr(), dw.data_ptr(), dW1.data_ptr() if dW1 is not None else 0,
-                     dW2.data_ptr() if dW2 is not None else 0, cfg, self.compute.cuda_stream)
+        args = (s, dy.data_ptr(), topk_w.data_ptr(), W1.data_ptr(), W2.data_ptr(), self.plan,
+                self.pool.data_ptr(), self.act.data_ptr(), self.ypool.data_ptr(),
+                self.gu.data_ptr(), self.dgu.data_ptr(), self.dpool.data_ptr(),
+                dx.data_ptr(), dw.data_ptr(), dW1.data_ptr() if dW1 is not None else 0,
+                dW2.data_ptr() if dW2 is not None else 0, cfg)
+        if cfg.streaming:
+            # the combine backward in tile order on the communicate stream, backward Y
+            # taking tiles on the compute stream (moe_backward_streams)
+            moe_backward_streams(*args, self.comm.cuda_stream, self.compute.cuda_stream,
+                                 self.events[0], self.events[1])
+        else:
+            moe_backward(*args, self.compute.cuda_stream)
         return dx, dw

@@ -293,15 +293,37 @@ int moe_forward(const moe_shape *s, const void *x, const int32_t *topk_idx, cons
  * Work buffers (device, caller-owned, 16-byte aligned): gu and dgu [P_max, 2I] bf16,
  * dpool [P_max, H] bf16. Outputs: dx [T, H] bf16, dw [T, k] fp32, dW1, dW2 bf16. The grouped
  * GEMMs run on SM pairs (cfg->ffn_kernel must be 0 or MOE_FFN_SM_PAIR; cfg->packed_weights
- * and cfg->streaming must be 0). cfg->timing_events, if set, holds 8 events recorded on
- * `stream`: [0] before, [1] after the combine backward, [2] after the recompute, [3] after
- * backward Y, [4] after dW2, [5] after backward A, [6] after dW1, [7] after the dispatch
- * backward.
+ * and cfg->streaming must be 0: streaming needs moe_backward_streams). cfg->early_combine = 1
+ * mirrors early combine: the dispatch
+ * backward is folded into backward A, whose CTAs sum each token's k dpool rows as soon as
+ * they are stored (p's tok_pending and ready are re-armed first; dx is bit-identical);
+ * cfg->wait_timeout_us bounds that wait too (MOE_ERR_COMBINE_TIMEOUT). cfg->timing_events,
+ * if set, holds 8 events recorded on `stream`: [0] before, [1] after the combine backward,
+ * [2] after the recompute, [3] after backward Y, [4] after dW2, [5] after backward A, [6]
+ * after dW1, [7] after the dispatch backward (with early_combine: after dW1 as well).
  */
 int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
                  const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
                  const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
                  void *dW1, void *dW2, const moe_config *cfg, void *stream);
+
+/*
+ * moe_backward on the caller's two streams (the layer's communicate and compute streams, as
+ * in moe_forward), which also accepts cfg->streaming = 1: the mirror of the streaming
+ * forward. The combine backward then runs in pool-tile order on comm_stream (on a few SMs:
+ * 64 blocks), raising each pool tile's flag once its dypool rows and dw are written (dw is
+ * zeroed first, so dropped pairs keep 0), while backward Y on compute_stream takes each row
+ * chunk as soon as the flags of its tiles are full (bounded wait: MOE_ERR_FLAG_TIMEOUT);
+ * everything else runs on compute_stream, which waits for the combine backward before the
+ * weight gradients. Results are bit-identical to moe_backward's. ev_a / ev_b: two events
+ * (moe_events_create) for the ordering; comm_stream must differ from compute_stream when
+ * streaming. With cfg->streaming = 0 it is moe_backward on compute_stream.
+ */
+int moe_backward_streams(const moe_shape *s, const void *dy, const float *topk_w, const void *W1,
+                         const void *W2, const moe_plan_buffers *p, const void *pool, void *act,
+                         const void *ypool, void *gu, void *dgu, void *dpool, void *dx, float *dw,
+                         void *dW1, void *dW2, const moe_config *cfg, void *comm_stream,
+                         void *compute_stream, void *ev_a, void *ev_b);
 
 /* Create / destroy n cudaEvent_t (timing disabled) for moe_forward's ordering. */
 int moe_events_create(void **events, int32_t n);

@@ -126,3 +126,20 @@ def test_ep_count_exchange_over_two_gloo_ranks_and_layout_against_the_oracle():
                 assert (d, row) == (-1, -1)
                 continue
             assert row == g - ref["offsets"][d * Er]
+
+
+def test_backward_streaming_needs_two_streams_and_events():
+    """Host checks only (no launch): moe_backward refuses cfg.streaming (it has one stream);
+    moe_backward_streams refuses it with one stream for both roles or without events."""
+    import combine_moe_plan_03_b200 as moe
+    s = moe.moe_shape(64, 128, 128, 4, 2, 64)
+    plan = moe.moe_plan_bind(s, 1 << 24)
+    a = [1 << 28] * 12
+    cfg = moe.moe_config(streaming=1)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_backward(s, *a[:4], plan, *a[4:], 0, 0, cfg, 0)
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+    for comm, comp, ea, eb in ((1 << 12, 1 << 12, 1 << 13, 1 << 14), (1 << 12, 1 << 15, 0, 1 << 14)):
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_backward_streams(s, *a[:4], plan, *a[4:], 0, 0, cfg, comm, comp, ea, eb)
+        assert ei.value.code == moe.MOE_ERR_INVALID_ARG
