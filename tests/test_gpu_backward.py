@@ -32,6 +32,7 @@ def _run(cfg, W1, W2, x, idx, w, dy, weight_grads=False):
                          device=W1.device),
               torch.full((cfg.E, cfg.I, cfg.H), float("nan"), dtype=torch.bfloat16,
                          device=W1.device))
+    torch.cuda.synchronize()   # the fills (default stream) before the backward (compute stream)
     dx, dwg = buf.backward(bf16_dev(dy), dw_dev, W1, W2, dW1=gW[0] if gW else None,
                            dW2=gW[1] if gW else None)
     torch.cuda.synchronize()
@@ -182,6 +183,7 @@ def test_backward_no_live_pairs_and_no_tokens():
     buf.forward(e, ei, ew, W1, W2)
     gW1 = torch.full((4, 128, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
     gW2 = torch.full((4, 128, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()   # the fills (default stream) before the backward (compute stream)
     dx, dw = buf.backward(e, ew, W1, W2, dW1=gW1, dW2=gW2)
     torch.cuda.synchronize()
     assert moe.moe_get_status(buf.plan)[0] == 0 and dx.numel() == 0 and dw.numel() == 0

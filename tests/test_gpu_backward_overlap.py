@@ -36,6 +36,9 @@ def _backward(cfg, W1, W2, x, idx, w, dy, early, weight_grads=True):
               torch.full((cfg.E, cfg.I, cfg.H), float("nan"), dtype=torch.bfloat16,
                          device=W1.device))
     dx = torch.full((cfg.T, cfg.H), float("nan"), dtype=torch.bfloat16, device=W1.device)
+    # the poisoned outputs are filled on the default stream; the backward runs on the
+    # layer's compute stream: the fills must be done before it writes
+    torch.cuda.synchronize()
     dx, dwg = buf.backward(bf16_dev(dy), dw_dev, W1, W2, moe.moe_config(early_combine=early),
                            dx=dx, dW1=gW[0] if gW else None, dW2=gW[1] if gW else None)
     torch.cuda.synchronize()
@@ -125,6 +128,7 @@ def _backward_cfg(cfg, W1, W2, x, idx, w, dy, mcfg):
                      device=W1.device),
           torch.full((cfg.E, cfg.I, cfg.H), float("nan"), dtype=torch.bfloat16, device=W1.device))
     dw_out = torch.full((cfg.T, cfg.k), float("nan"), dtype=torch.float32, device=W1.device)
+    torch.cuda.synchronize()   # fills (default stream) before the backward (compute stream)
     dx, dwg = buf.backward(bf16_dev(dy), dw_dev, W1, W2, mcfg, dw=dw_out, dW1=gW[0], dW2=gW[1])
     torch.cuda.synchronize()
     code, aux = moe.moe_get_status(buf.plan)
