@@ -81,8 +81,10 @@ class MoELayerBuffers:
         b1, b2 = moe_packed_weight_bytes(s)
         W1p = torch.empty(b1 // 2, dtype=torch.bfloat16, device=self.device)
         W2p = torch.empty(b2 // 2, dtype=torch.bfloat16, device=self.device)
+        cur = self._enter()
         moe_pack_weights(s, W1.data_ptr(), W2.data_ptr(), W1p.data_ptr(), W2p.data_ptr(),
                          self.compute.cuda_stream)
+        self._leave(cur)
         self.compute.synchronize()
         return W1p, W2p
 
@@ -130,11 +132,27 @@ class MoELayerBuffers:
                 assert tuple(W2.shape) == (s.E, s.I, s.H)
             w1, w2 = W1.data_ptr(), W2.data_ptr()
             act, ypool = self.act.data_ptr(), self.ypool.data_ptr()
+        cur = self._enter()
         moe_forward(s, x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), w1, w2, self.plan,
                     self.pool.data_ptr(), act, ypool, out.data_ptr(), cfg,
                     self.comm.cuda_stream, self.compute.cuda_stream, self.events[0],
                     self.events[1])
+        self._leave(cur)
         return out
+
+    def _enter(self) -> torch.cuda.Stream:
+        # the layer's streams start after the caller's work so far on its current stream
+        # (inputs made there are complete) ...
+        cur = torch.cuda.current_stream(self.device)
+        self.comm.wait_stream(cur)
+        self.compute.wait_stream(cur)
+        return cur
+
+    def _leave(self, cur: torch.cuda.Stream) -> None:
+        # ... and the caller's stream continues after the layer: the outputs are ready in its
+        # stream order, and memory of its tensors that it frees (temporaries passed in) is
+        # reused only by work that runs after the layer's kernels
+        cur.wait_stream(self.compute)
 
     def backward(self, dy: torch.Tensor, topk_w: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor,
                  cfg: moe_config | None = None, dx: torch.Tensor | None = None,
@@ -169,6 +187,7 @@ class MoELayerBuffers:
                 self.gu.data_ptr(), self.dgu.data_ptr(), self.dpool.data_ptr(),
                 dx.data_ptr(), dw.data_ptr(), dW1.data_ptr() if dW1 is not None else 0,
                 dW2.data_ptr() if dW2 is not None else 0, cfg)
+        cur = self._enter()
         if cfg.streaming:
             # the combine backward in tile order on the communicate stream, backward Y
             # taking tiles on the compute stream (moe_backward_streams)
@@ -176,4 +195,5 @@ class MoELayerBuffers:
                                  self.events[0], self.events[1])
         else:
             moe_backward(*args, self.compute.cuda_stream)
+        self._leave(cur)
         return dx, dw
