@@ -668,11 +668,18 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
   y.aux = static_cast<const uint16_t *>(gu);
   y.aux_ld = 2 * s.I;
   y.aux_off = s.I;
-  // streaming: the combine backward fills dypool tile by tile in blocks that sit beside
-  // backward Y's CTAs and raises the tiles' flags; backward Y takes a chunk once the flags
-  // of its tiles are full
+  // streaming: the combine backward fills dypool tile by tile on the SMs backward Y leaves
+  // free and raises the tiles' flags; backward Y takes a chunk once the flags of its tiles
+  // are full. (Whether other blocks can sit beside the GEMM's CTAs is not relied on: with
+  // the GEMM on every SM the combine backward it waits for could not start.)
   y.streaming = cfg.streaming;
-  if (launch_ffn_pair(2, true, tw2_k, tx_dy, y, clusters, st) != cudaSuccess)
+  int clusters_y = clusters;
+  if (cfg.streaming) {
+    clusters_y = (num_sms - kStreamDispatchSMs) / 2;
+    if (clusters_y > clusters) clusters_y = clusters;
+    if (clusters_y < 1) clusters_y = 1;
+  }
+  if (launch_ffn_pair(2, true, tw2_k, tx_dy, y, clusters_y, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (combine_done != nullptr && cudaStreamWaitEvent(st, combine_done, 0) != cudaSuccess)
     return MOE_ERR_CUDA;

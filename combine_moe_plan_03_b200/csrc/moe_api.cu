@@ -372,10 +372,10 @@ int backward_entry(const moe_shape *s, const void *dy, const float *topk_w, cons
         cudaMemsetAsync(dw, 0, sizeof(float) * (size_t)s->T * s->k, st) != cudaSuccess ||
         cudaEventRecord(ev_a, st) != cudaSuccess || cudaStreamWaitEvent(comm, ev_a, 0) != cudaSuccess)
       return MOE_ERR_CUDA;
-    // 4 blocks of 128 threads per SM: they fit beside backward Y's one CTA per SM (its 320
-    // threads and 214 KB of shared memory leave room), so tiles fill across the whole GPU
-    if (launch_combine_backward_tiles(*s, dy, ypool, topk_w, *p, dpool, dw, nsm * 4, comm) !=
-        cudaSuccess)
+    // 8 blocks of 128 threads for each of the SMs that backward Y leaves free: the combine
+    // backward never depends on finding room beside backward Y's CTAs (which wait for it)
+    if (launch_combine_backward_tiles(*s, dy, ypool, topk_w, *p, dpool, dw,
+                                      kStreamDispatchSMs * 8, comm) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (tev != nullptr && cudaEventRecord(tev[1], comm) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaEventRecord(ev_b, comm) != cudaSuccess) return MOE_ERR_CUDA;

@@ -310,9 +310,9 @@ int moe_backward(const moe_shape *s, const void *dy, const float *topk_w, const 
 /*
  * moe_backward on the caller's two streams (the layer's communicate and compute streams, as
  * in moe_forward), which also accepts cfg->streaming = 1: the mirror of the streaming
- * forward. The combine backward then runs in pool-tile order on comm_stream (4 small
- * blocks per SM, beside backward Y's CTAs), raising each pool tile's flag once its dypool
- * rows and dw are written (dw is
+ * forward. The combine backward then runs in pool-tile order on comm_stream (on the 16 SMs
+ * backward Y leaves free), raising each pool tile's flag once its dypool rows and dw are
+ * written (dw is
  * zeroed first, so dropped pairs keep 0), while backward Y on compute_stream takes each row
  * chunk as soon as the flags of its tiles are full (bounded wait: MOE_ERR_FLAG_TIMEOUT);
  * everything else runs on compute_stream, which waits for the combine backward before the
