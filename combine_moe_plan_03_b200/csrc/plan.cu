@@ -152,7 +152,11 @@ __global__ void __launch_bounds__(256)
     const int32_t chunk = gemm_chunk_rows(c);
     if (c > 0) my_blk += (c + chunk - 1) / chunk;
   }
-  atomicAdd(&s_rows, (unsigned long long)rows64);
+  // the block's total in 64 bits: a warp sum, then one shared atomic per warp
+  unsigned long long wsum = (unsigned long long)rows64;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  if ((threadIdx.x & 31) == 0) atomicAdd(&s_rows, wsum);
   __syncthreads();
   // Counts beyond the dropless bound (only counts passed in by a caller, as in expert
   // parallelism, can do this): leave an empty plan, whose tables fit any arena, and report.
