@@ -13,8 +13,8 @@
 //   plan_scan_kernel    (plan.cu) twice: exclusive scans over the sources, padded offsets,
 //                       the FFN's tile and row-chunk tables
 //   ep_pad_kernel       zeroes this rank's padding rows, counting each on its tile's flag
-//   ep_dispatch_kernel  source side, a warp per token: each 16-byte vector of x[t] loaded once
-//                       and stored into the pool rows of its k pairs, on whichever
+//   ep_dispatch_kernel  source side: x[t] staged once in shared memory, then stored (16-byte
+//                       vectors, every lane) into the pool rows of its k pairs, on whichever
 //                       rank owns each pair's expert (peer pointers); then each stored row is
 //                       counted on its owner's tile flag (release at system scope), so a
 //                       streaming grouped FFN on the owner takes a pool tile as soon as its
@@ -113,9 +113,6 @@ __device__ __forceinline__ int32_t ep_dest_row(int32_t f, int32_t src, int32_t R
   return (int32_t)row;
 }
 
-// One warp per token (grid-stride over tokens): lane j < k finds pair j's row and owner; then
-// every lane loads its 16-byte vectors of x[t] once and stores each to all the token's live
-// rows. Whole tokens per warp keep every token of a rank in flight at once (a rank has few).
 __global__ void __launch_bounds__(kEpThreads)
     ep_dispatch_kernel(const uint4 *__restrict__ x, int32_t T, int32_t k, int32_t hv,
                        int32_t R, int32_t Er, int32_t tile, int32_t src,
@@ -127,7 +124,8 @@ __global__ void __launch_bounds__(kEpThreads)
                        const int32_t *__restrict__ own_counts,
                        const int32_t *__restrict__ g_counts, int32_t *__restrict__ status,
                        const EpPeers pools, const EpFlags flags, bool signal) {
-  __shared__ uint4 *s_dst[kEpThreads / 32][kMaxTopK];
+  extern __shared__ uint4 row[];  // [hv]: x[t]
+  __shared__ int32_t s_row[kMaxTopK], s_dst[kMaxTopK];
   if (blockIdx.x == 0) {
     // this rank's row of all_counts, recovered from the scanned sources, must be its own
     // plan's counts; a mismatch means the caller's all_counts are not the ranks' plans
@@ -138,30 +136,27 @@ __global__ void __launch_bounds__(kEpThreads)
         report(status, MOE_ERR_POOL_OVERFLOW, e);
     }
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
-    int32_t my_row = -1, my_dst = 0;
-    if (lane < k)
-      my_row = ep_dest_row((int32_t)(t * k + lane), src, R, Er, tile, own_pool_row,
-                           own_tile_expert, own_offsets, g_offsets, g_src_base, max_rows, status,
-                           &my_dst);
-    if (lane < k)
-      s_dst[warp][lane] =
-          my_row < 0 ? nullptr : reinterpret_cast<uint4 *>(pools.base[my_dst]) + (size_t)my_row * hv;
-    __syncwarp();
-    for (int v = lane; v < hv; v += 32) {
-      const uint4 val = x[t * hv + v];
-      for (int j = 0; j < k; ++j) {
-        uint4 *d = s_dst[warp][j];
-        if (d != nullptr) d[v] = val;
-      }
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    for (int i = threadIdx.x; i < hv; i += blockDim.x) row[i] = x[t * hv + i];
+    if (threadIdx.x < k) {
+      int32_t d = 0;
+      s_row[threadIdx.x] = ep_dest_row((int32_t)(t * k + threadIdx.x), src, R, Er, tile,
+                                       own_pool_row, own_tile_expert, own_offsets, g_offsets,
+                                       g_src_base, max_rows, status, &d);
+      s_dst[threadIdx.x] = d;
     }
-    // every lane's stores of the token's rows precede the warp barrier; the release at
-    // system scope passes them on to the owner's acquire of the flag
-    __syncwarp();
-    if (signal && lane < k && my_row >= 0)
-      red_release_sys_add(flags.base[my_dst] + my_row / tile, 1u);
+    __syncthreads();
+    for (int j = 0; j < k; ++j) {
+      const int32_t r = s_row[j];
+      if (r < 0) continue;  // uniform across the block
+      uint4 *dst = reinterpret_cast<uint4 *>(pools.base[s_dst[j]]) + (size_t)r * hv;
+      for (int i = threadIdx.x; i < hv; i += blockDim.x) dst[i] = row[i];
+    }
+    __syncthreads();
+    // every thread's stores of the token's rows precede the barrier; the release at system
+    // scope passes them on to the owner's acquire of the flag
+    if (signal && threadIdx.x < k && s_row[threadIdx.x] >= 0)
+      red_release_sys_add(flags.base[s_dst[threadIdx.x]] + s_row[threadIdx.x] / tile, 1u);
   }
 }
 
@@ -173,9 +168,6 @@ __device__ __forceinline__ uint4 ld_nc_v4_ep(const uint4 *p) {
   return v;
 }
 
-// One warp per token: lane j < k finds pair j's row in its owner's ypool and its weight;
-// each lane then combines its 16-byte vectors of the row, all k loads of a group of 8 pairs
-// issued before their FMAs (the fp32 chain over j ascending of combine.cu).
 __global__ void __launch_bounds__(kEpThreads)
     ep_combine_kernel(const float *__restrict__ topk_w, uint4 *__restrict__ out, int32_t T,
                       int32_t k, int32_t hv, int32_t R, int32_t Er, int32_t tile, int32_t src,
@@ -185,37 +177,32 @@ __global__ void __launch_bounds__(kEpThreads)
                       const int32_t *__restrict__ g_offsets,
                       const int32_t *__restrict__ g_src_base, int64_t max_rows,
                       int32_t *__restrict__ status, const EpPeers ypools) {
-  __shared__ const uint4 *s_src[kEpThreads / 32][kMaxTopK];
-  __shared__ float s_w[kEpThreads / 32][kMaxTopK];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
-    if (lane < k) {
+  __shared__ const uint4 *s_src[kMaxTopK];
+  __shared__ float s_w[kMaxTopK];
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) {
       int32_t d = 0;
-      const int32_t r = ep_dest_row((int32_t)(t * k + lane), src, R, Er, tile, own_pool_row,
-                                    own_tile_expert, own_offsets, g_offsets, g_src_base,
-                                    max_rows, status, &d);
-      s_src[warp][lane] =
+      const int32_t r = ep_dest_row((int32_t)(t * k + threadIdx.x), src, R, Er, tile,
+                                    own_pool_row, own_tile_expert, own_offsets, g_offsets,
+                                    g_src_base, max_rows, status, &d);
+      s_src[threadIdx.x] =
           r < 0 ? nullptr : reinterpret_cast<const uint4 *>(ypools.base[d]) + (size_t)r * hv;
-      s_w[warp][lane] = topk_w[t * k + lane];
+      s_w[threadIdx.x] = topk_w[t * k + threadIdx.x];
     }
-    __syncwarp();
-    for (int v = lane; v < hv; v += 32) {
+    __syncthreads();
+    for (int v = threadIdx.x; v < hv; v += blockDim.x) {
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
       for (int j0 = 0; j0 < k; j0 += 8) {
         uint4 y[8];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const uint4 *p = j0 + jj < k ? s_src[warp][j0 + jj] : nullptr;
-          if (p != nullptr) y[jj] = ld_nc_v4_ep(p + v);
-        }
+        for (int jj = 0; jj < 8; ++jj)
+          if (j0 + jj < k && s_src[j0 + jj] != nullptr) y[jj] = ld_nc_v4_ep(s_src[j0 + jj] + v);
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const uint4 *p = j0 + jj < k ? s_src[warp][j0 + jj] : nullptr;
-          if (p != nullptr) {
-            const float w = s_w[warp][j0 + jj];
+        for (int jj = 0; jj < 8; ++jj)
+          if (j0 + jj < k && s_src[j0 + jj] != nullptr) {
+            const float w = s_w[j0 + jj];
             const uint32_t u[4] = {y[jj].x, y[jj].y, y[jj].z, y[jj].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -223,12 +210,11 @@ __global__ void __launch_bounds__(kEpThreads)
               acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
             }
           }
-        }
       }
       out[t * hv + v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                    pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
     }
-    __syncwarp();  // the next token's pointers overwrite this one's
+    __syncthreads();
   }
 }
 
@@ -283,10 +269,14 @@ cudaError_t launch_ep_dispatch(const moe_shape &rank_shape, int32_t R, int32_t r
                                cudaStream_t st) {
   if (rank_shape.T == 0) return cudaSuccess;
   const int hv = rank_shape.H / 8;
-  // a warp per token: every token of the rank in flight at once, up to 8 blocks per SM
-  int64_t grid = ((int64_t)rank_shape.T + kEpThreads / 32 - 1) / (kEpThreads / 32);
-  if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
-  ep_dispatch_kernel<<<(int)grid, kEpThreads, 0, st>>>(
+  const size_t smem = (size_t)hv * sizeof(uint4);  // one row of x (H <= 38,720 by check_shape)
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(ep_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return cudaErrorUnknown;
+  int64_t grid = (int64_t)num_sms * 4;
+  if (grid > rank_shape.T) grid = rank_shape.T;
+  ep_dispatch_kernel<<<(int)grid, kEpThreads, smem, st>>>(
       static_cast<const uint4 *>(x), rank_shape.T, rank_shape.k, hv, R, rank_shape.E / R,
       rank_shape.tile, rank, own.pool_row, own.tile_expert, own.offsets, ep.offsets,
       ep.src_base, plan_geom(ep_local_shape(rank_shape, R)).pmax, own.counts, ep.counts,
@@ -304,8 +294,8 @@ cudaError_t launch_ep_combine(const moe_shape &rank_shape, int32_t R, int32_t ra
       ep.local.tile_flags, 0,
       sizeof(uint32_t) * (size_t)plan_geom(ep_local_shape(rank_shape, R)).n_tiles, st);
   if (e != cudaSuccess || rank_shape.T == 0) return e;
-  int64_t grid = ((int64_t)rank_shape.T + kEpThreads / 32 - 1) / (kEpThreads / 32);
-  if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
+  int64_t grid = (int64_t)num_sms * 8;
+  if (grid > rank_shape.T) grid = rank_shape.T;
   ep_combine_kernel<<<(int)grid, kEpThreads, 0, st>>>(
       topk_w, static_cast<uint4 *>(out), rank_shape.T, rank_shape.k, rank_shape.H / 8, R,
       rank_shape.E / R, rank_shape.tile, rank, own.pool_row, own.tile_expert, own.offsets,
