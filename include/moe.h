@@ -430,7 +430,11 @@ typedef struct moe_ep_plan {
 } moe_ep_plan;
 
 /* Local shape {R * T, H, I, E / R, k, tile} of a rank's pool; pool rows (dropless bound for
- * all ranks' pairs on E / R experts); bytes of the EP plan arena; binding the arena. */
+ * all ranks' pairs on E / R experts); bytes of the EP plan arena; binding the arena (host
+ * only: 256-byte aligned slices of the caller's device arena, which must be zeroed once
+ * before the first layer call: its status word and pool tile flags start at zero).
+ * Errors: MOE_ERR_INVALID_ARG (R outside [1, MOE_EP_MAX_RANKS], E not a multiple of R, a
+ * shape that check fails, NULL pointers), MOE_ERR_UNSUPPORTED_SHAPE. */
 int moe_ep_local_shape(const moe_shape *rank_shape, int32_t R, moe_shape *out);
 int moe_ep_pool_rows(const moe_shape *rank_shape, int32_t R, int64_t *rows_out);
 int moe_ep_arena_bytes(const moe_shape *rank_shape, int32_t R, size_t *bytes_out);
