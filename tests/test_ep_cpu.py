@@ -143,3 +143,33 @@ def test_backward_streaming_needs_two_streams_and_events():
         with pytest.raises(moe.MoEError) as ei:
             moe.moe_backward_streams(s, *a[:4], plan, *a[4:], 0, 0, cfg, comm, comp, ea, eb)
         assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+
+
+def _exchange_rank(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from combine_moe_plan_03_b200.ep import exchange
+    got = exchange((rank, [bytes([rank] * 64), bytes([rank + 1] * 64)], 256 * (rank + 1)))
+    q.put((rank, got))
+    dist.destroy_process_group()
+
+
+def test_ep_layer_handle_exchange_over_two_gloo_ranks():
+    """EPLayer's one host-side exchange (each rank's IPC handles and flag offset, gathered in
+    rank order), over two gloo ranks on the CPU."""
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_exchange_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank in range(2):
+        assert [g[0] for g in res[rank]] == [0, 1]
+        assert res[rank][1][1][0] == bytes([1] * 64) and res[rank][0][2] == 256

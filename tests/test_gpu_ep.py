@@ -278,3 +278,28 @@ def test_ep_streaming_ffn_times_out_without_the_dispatch_flags():
     assert moe.moe_get_status(ep[0].local)[0] == 0
     for b in own:
         b.close()
+
+
+@pytest.mark.parametrize("streaming", [0, 1])
+def test_ep_layer_one_rank_matches_single_gpu(streaming):
+    """EPLayer (the process-group runner of the EP calls) with one rank: its peer pointers are
+    its own buffers; two calls in a row equal the single-GPU layer bit for bit."""
+    import combine_moe_plan_03_b200 as moe
+    from combine_moe_plan_03_b200.ep import EPLayer
+    from gpu_helpers import bf16_dev, f32_dev, i32_dev, weights_dev
+    cfg = si.custom("ep-layer", T=300, H=384, I=256, E=6, k=2, tile=64, seed=71)
+    W1, W2 = weights_dev(cfg)
+    layer = EPLayer(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    single = moe.MoELayerBuffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.tile)
+    for mb in range(2):
+        x, di, dw = bf16_dev(si.make_x(cfg, mb)), None, None
+        idx, w = si.make_routing(cfg, mb)
+        di, dw = i32_dev(idx), f32_dev(w)
+        torch.cuda.synchronize()
+        out = layer.forward(x, di, dw, W1, W2, moe.moe_config(streaming=streaming))
+        ref = single.forward(x, di, dw, W1, W2)
+        torch.cuda.synchronize()
+        assert layer.status()[0] == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), mb
+    layer.close()
+    single.close()
