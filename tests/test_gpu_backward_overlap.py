@@ -20,6 +20,8 @@ SHAPES = [
     ("wide-H", 150, 1088, 128, 5, 3, 64, 0.1),        # three column blocks, the last ragged
     ("k8", 96, 512, 256, 16, 8, 64, 0.2),
     ("half-dropped", 90, 128, 128, 4, 2, 64, 0.5),
+    ("E1-k1", 100, 128, 192, 1, 1, 128, 0.0),         # one expert, one pair per token
+    ("k16", 64, 128, 128, 32, 16, 64, 0.1),           # two groups of 8 pairs per token
 ]
 
 
