@@ -879,9 +879,9 @@ def run_moe(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",
-            "config": dict(config_block(cfg, world),
-                           weights="prepacked tiles (moe_pack_weights, once before timing)"
-                           if packed else "as given: W1 [E,H,2I], W2 [E,I,H]"),
+            "config": config_block(cfg, world),
+            "weights": ("prepacked tiles (moe_pack_weights, once before timing)"
+                        if packed else "as given: W1 [E,H,2I], W2 [E,I,H]"),
             "streaming": streaming, "ffn_kernel": ffn_kernel, "early_combine": early,
             "phases_ms_per_call": {k: round(v, 5) for k, v in ph.items()},
             "phases_mcycles_per_call": ({k: round(v * clocks["sm_mhz"] / 1000.0, 4)
