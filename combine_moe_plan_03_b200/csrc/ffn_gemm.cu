@@ -543,6 +543,11 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
         cudaStreamWaitEvent(st, helper_done, 0) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
+  // early combine counts GEMM Y's row chunks in the tile flags (GEMM A, the only reader of
+  // the flags, is done; there are no more chunks than tiles): zero them first
+  if (early && cudaMemsetAsync(p.tile_flags, 0, sizeof(uint32_t) * (size_t)g.n_tiles, st) !=
+                   cudaSuccess)
+    return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[4], st) != cudaSuccess) return MOE_ERR_CUDA;
 
   FfnParams y = a;
@@ -574,6 +579,7 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
     y.row_src = p.row_src;
     y.pool_row = p.pool_row;
     y.topk_w = topk_w;
+    y.chunk_cnt = reinterpret_cast<int32_t *>(p.tile_flags);
     y.tok_pending = p.tok_pending;
     y.ready = p.ready;
     y.comb_out = static_cast<uint16_t *>(out);
@@ -714,12 +720,18 @@ int launch_ffn_backward(const moe_shape &s, const void *W1, const void *W2,
     a.row_src = p.row_src;
     a.pool_row = p.pool_row;
     a.topk_w = nullptr;
+    a.chunk_cnt = reinterpret_cast<int32_t *>(p.tile_flags);
     a.tok_pending = p.tok_pending;
     a.ready = p.ready;
     a.comb_out = static_cast<uint16_t *>(early_dx);
     a.T = s.T;
     a.k = s.k;
   }
+  // its row-chunk counters live in the tile flags (backward Y, their only other reader, is
+  // done): zero them first
+  if (early && cudaMemsetAsync(p.tile_flags, 0, sizeof(uint32_t) * (size_t)g.n_tiles, st) !=
+                   cudaSuccess)
+    return MOE_ERR_CUDA;
   if (launch_ffn_pair(1, true, tw1_k, tx_dgu, a, clusters, st, early) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (tev != nullptr && cudaEventRecord(tev[5], st) != cudaSuccess) return MOE_ERR_CUDA;

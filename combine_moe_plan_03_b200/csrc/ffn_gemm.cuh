@@ -40,13 +40,15 @@ struct FfnParams {
   // mode 3 (GEMM A saving gate / up): out = [g | u], act = bf16(silu(g) u) to out2
   uint16_t *out2;
   int64_t out2_ld;
-  // early combine (GEMM Y of the SM-pair kernel): per stored unit row, tok_pending[t] of the
-  // row's token t = row_src[p] / k drops by one; at zero t + 1 goes to the ready queue
+  // early combine (GEMM Y of the SM-pair kernel): once all units of a row chunk are stored
+  // (chunk_cnt reaches both CTAs x the column blocks), tok_pending[t] of each live row's
+  // token t = row_src[p] / k drops by one; at zero t + 1 goes to the ready queue
   // ready[0 .. T) (tail at ready[T + 1]); after their GEMM work the CTAs pop tokens (head
   // at ready[T]) and write comb_out[t] = bf16(sum_j topk_w[t, j] ypool[pool_row[t, j]]).
   const int32_t *row_src;
   const int32_t *pool_row;
   const float *topk_w;
+  int32_t *chunk_cnt;      // per row chunk: units stored by both CTAs (zero at launch)
   int32_t *tok_pending;
   int32_t *ready;
   uint16_t *comb_out;

@@ -492,12 +492,20 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
         if (lane == 0) raise_abort_pair(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, u);
         break;
       }
-      // every row of the unit once per CTA: the token's count drops by one (release: the
-      // epilogue's stores before it; acquire: the other CTAs' stores, for the combine)
+      // this CTA's share of the unit is stored: count it on the row chunk (release: the
+      // epilogue's stores before it; acquire: the other units' stores). The last of the
+      // chunk's 2 x n_blocks counts drops each live row's token count by one, so a token's
+      // count falls once per live pair instead of once per pair, column block and CTA.
       int32_t mb, nb;
       unit_coords(prm.mblk, u, prm.n_blocks, mb, nb);
       const int32_t row0 = prm.mblk[kMblkInts * mb + 0];
       const int32_t rows = prm.mblk[kMblkInts * mb + 2];
+      int last = 0;
+      if (lane == 0)
+        last = atom_add_acq_rel_gpu(prm.chunk_cnt + mb, 1) == 2 * prm.n_blocks - 1 ? 1 : 0;
+      last = __shfl_sync(0xffffffffu, last, 0);
+      __syncwarp();  // lane 0's acquire orders the other lanes' releases below
+      if (!last) continue;
       for (int r = lane; r < rows; r += 32) {
         const int32_t f = prm.row_src[row0 + r];
         if (f < 0) continue;

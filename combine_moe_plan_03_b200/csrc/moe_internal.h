@@ -140,11 +140,11 @@ int launch_ffn(const moe_shape &s, const void *pool, const void *W1, const void 
                void *out, const moe_config &cfg, int num_sms, cudaStream_t st,
                cudaStream_t helper_stream = nullptr, cudaEvent_t helper_done = nullptr);
 
-// Early combine: GEMM Y units of the SM-pair kernel cover 512 output columns, and both CTAs
-// of a pair count a unit's rows once each, so a token with n live pairs waits for
-// n * early_combine_arrivals(H) row counts.
-__host__ __device__ inline int32_t early_combine_arrivals(int32_t H) {
-  return 2 * ((H + 511) / 512);
+// Early combine: a row chunk counts once per token row when all its units (every column
+// block, both CTAs of a pair) are stored, so a token with n live pairs waits for
+// n * early_combine_arrivals(H) = n counts.
+__host__ __device__ inline int32_t early_combine_arrivals(int32_t) {
+  return 1;
 }
 
 }  // namespace moe
