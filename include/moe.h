@@ -100,7 +100,8 @@ typedef struct moe_plan_buffers {
   int32_t *workspace;   /* plan scratch: per-(expert, 256-pair chunk) counts + 1 counter */
   int32_t *status;      /* [4]          code, aux, 0, 0 (first device error wins) */
   /* early combine (moe_config.early_combine); may be NULL otherwise. moe_plan zeroes both. */
-  int32_t *tok_pending; /* [T]          expert-row stores still missing per token */
+  int32_t *tok_pending; /* [T]          live pairs per token whose GEMM Y row chunk is not
+                                        complete yet */
   int32_t *ready;       /* [T + 4]      queue of finished tokens (t + 1; 0 = not yet), then
                                         its head and tail counters */
 } moe_plan_buffers;
@@ -237,8 +238,10 @@ int moe_grouped_ffn(const moe_shape *s, const void *pool, const void *W1, const 
  * moe_combine computes it (fp32 FMA chain, j ascending), each token combined by the GEMM Y
  * kernel's CTAs as soon as its k rows are stored. Needs cfg->early_combine = 1, the SM-pair
  * kernel, p->tok_pending / p->ready, and moe_dispatch run with MOE_DISPATCH_ARM_COMBINE
- * after this call's moe_plan. A token whose rows never arrive (the counters were not armed)
- * gives MOE_ERR_COMBINE_TIMEOUT in the status word after cfg->wait_timeout_us.
+ * after this call's moe_plan. GEMM Y counts its finished units per row chunk in
+ * p->tile_flags (zeroed after GEMM A, their streaming reader, is done). A token whose rows
+ * never arrive (the counters were not armed) gives MOE_ERR_COMBINE_TIMEOUT in the status
+ * word after cfg->wait_timeout_us.
  */
 int moe_grouped_ffn_combine(const moe_shape *s, const void *pool, const void *W1, const void *W2,
                             const moe_plan_buffers *p, void *act, void *ypool,
