@@ -12,7 +12,8 @@
 //                       and over this rank's E_r experts (the grouped FFN's plan)
 //   plan_scan_kernel    (plan.cu) twice: exclusive scans over the sources, padded offsets,
 //                       the FFN's tile and row-chunk tables
-//   ep_pad_kernel       zeroes this rank's padding rows, counting each on its tile's flag
+//   ep_pad_kernel       zeroes this rank's padding rows (a block per row), counting each on
+//                       its tile's flag
 //   ep_dispatch_kernel  source side: x[t] staged once in shared memory, then stored (16-byte
 //                       vectors, every lane) into the pool rows of its k pairs, on whichever
 //                       rank owns each pair's expert (peer pointers); then each stored row is
@@ -72,20 +73,19 @@ __global__ void __launch_bounds__(kEpThreads)
   }
 }
 
-// Padding rows of this rank's pool: [offsets[e] + counts[e], offsets[e + 1]) per local expert,
-// one row per block at a time (16-byte stores); each zeroed row counts one on its tile's flag.
+// Padding rows of this rank's pool: [offsets[e] + counts[e], offsets[e + 1]) per local expert.
+// Block (j, e) zeroes padding row j of expert e if it has one (16-byte stores; an expert has
+// fewer than tile padding rows) and counts it on its tile's flag: every row in parallel.
 __global__ void __launch_bounds__(kEpThreads)
     ep_pad_kernel(uint4 *__restrict__ pool, int32_t hv, const int32_t *__restrict__ counts,
-                  const int32_t *__restrict__ offsets, int32_t Er, uint32_t *__restrict__ flags,
+                  const int32_t *__restrict__ offsets, uint32_t *__restrict__ flags,
                   int32_t tile) {
-  for (int e = 0; e < Er; ++e) {
-    const int64_t r0 = offsets[e] + counts[e], r1 = offsets[e + 1];
-    for (int64_t r = r0 + blockIdx.x; r < r1; r += gridDim.x) {  // uniform across the block
-      for (int i = threadIdx.x; i < hv; i += blockDim.x) pool[r * hv + i] = make_uint4(0u, 0u, 0u, 0u);
-      __syncthreads();
-      if (threadIdx.x == 0) red_release_sys_add(flags + r / tile, 1u);
-    }
-  }
+  const int e = blockIdx.y;
+  const int64_t r = (int64_t)offsets[e] + counts[e] + blockIdx.x;
+  if (r >= offsets[e + 1]) return;  // uniform across the block
+  for (int i = threadIdx.x; i < hv; i += blockDim.x) pool[r * hv + i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if (threadIdx.x == 0) red_release_sys_add(flags + r / tile, 1u);
 }
 
 // Row of pair f in its owner's pool, and the owner. own_*: the source's own plan over the
@@ -257,8 +257,8 @@ cudaError_t launch_ep_layout(const moe_shape &rank_shape, int32_t R, int32_t ran
   if (e != cudaSuccess) return e;
   // the tile flags are not reset here: other ranks' dispatches may already be counting on
   // them; moe_ep_combine resets them after this rank's grouped FFN has used them
-  ep_pad_kernel<<<num_sms * 2, kEpThreads, 0, st>>>(
-      static_cast<uint4 *>(pool), rank_shape.H / 8, ep.local.counts, ep.local.offsets, Er,
+  ep_pad_kernel<<<dim3(rank_shape.tile - 1, Er), kEpThreads, 0, st>>>(
+      static_cast<uint4 *>(pool), rank_shape.H / 8, ep.local.counts, ep.local.offsets,
       reinterpret_cast<uint32_t *>(ep.local.tile_flags), rank_shape.tile);
   return cudaGetLastError();
 }
