@@ -274,7 +274,9 @@ cudaError_t launch_ep_dispatch(const moe_shape &rank_shape, int32_t R, int32_t r
       cudaFuncSetAttribute(ep_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return cudaErrorUnknown;
-  int64_t grid = (int64_t)num_sms * 4;
+  // a block per token, every token of the rank in flight at once where they fit (8 blocks
+  // of 256 threads per SM)
+  int64_t grid = (int64_t)num_sms * 8;
   if (grid > rank_shape.T) grid = rank_shape.T;
   ep_dispatch_kernel<<<(int)grid, kEpThreads, smem, st>>>(
       static_cast<const uint4 *>(x), rank_shape.T, rank_shape.k, hv, R, rank_shape.E / R,
