@@ -221,6 +221,33 @@ def test_weight_gradients_small_shapes_every_expert(shape):
     buf.close()
 
 
+def test_weight_gradients_every_row_residue():
+    """Experts whose row counts fall in every residue class of the weight-gradient K loop
+    (steps of 64 rows, MMAs of 16): 1, 15, 16, 17, 31, ..., 129 rows, one expert each, and
+    one expert without rows; dW1 and dW2 of each against the oracle."""
+    from gpu_helpers import to_f64, weights_dev
+    counts = [1, 15, 16, 17, 31, 32, 33, 47, 48, 49, 63, 64, 65, 80, 127, 128, 129, 0]
+    E, T = len(counts), sum(counts)
+    cfg = si.custom("row-residues", T=T, H=256, I=128, E=E, k=1, tile=64, seed=4242)
+    W1, W2 = weights_dev(cfg)
+    x = si.make_x(cfg)
+    _, w = si.make_routing(cfg)
+    order = np.random.default_rng(4242).permutation(T)
+    idx = np.repeat(np.arange(E, dtype=np.int32), counts)[order].reshape(T, 1)
+    dy = si.make_dy(cfg)
+    buf, dx, dw, (gW1, gW2) = _run(cfg, W1, W2, x, idx, w, dy, weight_grads=True)
+    for e in range(E):
+        g1, g2 = to_f64(gW1[e]), to_f64(gW2[e])
+        if counts[e] == 0:
+            assert not np.any(g1) and not np.any(g2), f"expert {e} without rows"
+            continue
+        r1, r2 = oracle.get().expert_weight_grads(x, idx, w, si.make_w1_expert(cfg, e),
+                                                  si.make_w2_expert(cfg, e), e, dy)
+        _close(g1, r1, f"dW1[{e}] ({counts[e]} rows)")
+        _close(g2, r2, f"dW2[{e}] ({counts[e]} rows)")
+    buf.close()
+
+
 def _oracle_weight_grads_threaded(x, idx, w, W1e, W2e, e, dy, threads=8):
     """The oracle's weight gradients of expert e, with the expert's tokens split into
     `threads` contiguous slices computed at once (the oracle releases the GIL) and the
