@@ -613,9 +613,9 @@ __global__ void __launch_bounds__(threads_for(kEarly), 1)
       __syncwarp();
       if (lane == 0) {
         if (lead)
-          mbar_arrive(acc_empty);
+          mbar_arrive_relaxed(acc_empty);
         else
-          mbar_arrive_cluster(acc_empty_lead);
+          mbar_arrive_cluster_relaxed(acc_empty_lead);
       }
 #pragma unroll
       for (int g = 0; g < kGroupsPerWarp; ++g) {

@@ -414,9 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) {
           if (lead)
-            mbar_arrive(acc_empty + acc);
+            mbar_arrive_relaxed(acc_empty + acc);
           else
-            mbar_arrive_cluster(cluster_map(smem_u32(acc_empty + acc), 0));
+            mbar_arrive_cluster_relaxed(cluster_map(smem_u32(acc_empty + acc), 0));
         }
         if (store) {
           // the previous store has read the block
