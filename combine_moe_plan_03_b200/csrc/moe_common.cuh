@@ -279,11 +279,12 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
-// Arrives with relaxed semantics, for handing a TMEM accumulator back to the MMA thread: the
-// epilogue's tcgen05.ld results are in registers once tcgen05.wait::ld returns, and nothing in
-// memory has to be made visible to the waiter, so no release is needed. (A release at cluster
-// scope from the second CTA of a pair waits for that thread's earlier memory operations, such
-// as the previous tile's stores, and stalled the hand-back.)
+// Arrives with relaxed semantics, for handing a resource back when nothing in memory has to be
+// made visible to the waiter: a TMEM accumulator (the epilogue's tcgen05.ld results are in
+// registers once tcgen05.wait::ld returns), or a schedule slot whose values the caller has
+// already read into registers (the arrive must depend on them, so it is not issued before the
+// reads return). A release at cluster scope from the second CTA of a pair waits for that
+// thread's earlier memory operations, such as the previous tile's stores, and stalled both.
 __device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar) {
   asm volatile(
       "{\n\t.reg .b64 st;\n\t"

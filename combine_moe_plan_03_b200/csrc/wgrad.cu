@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // overlaps the loads of the current unit (the units are short: a few k-steps)
       int32_t next_ticket = lead ? atomicAdd(prm.sched + 0, 1) : 0;
       for (;;) {
-        int32_t u;
+        int32_t u, kpeer = 0;
         if (lead) {
           if (!mbar_wait<true>(sched_empty + sslot, sphase ^ 1u, 2 * prm.timeout_ns, abort)) {
             raise_abort_w(abort, peer_abort, prm.status, MOE_ERR_PIPE_TIMEOUT, -1);
@@ -187,9 +187,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           u = sched[sslot];
-          mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
+          kpeer = sched_k[sslot];
+          if (u >= -1 && kpeer >= 0)   // issued once both reads have returned
+            mbar_arrive_cluster_relaxed(cluster_map(smem_u32(sched_empty + sslot), 0));
         }
-        const int32_t kcount = sched_k[sslot];
+        const int32_t kcount = lead ? sched_k[sslot] : kpeer;
         if (++sslot == kSchedSlots) {
           sslot = 0;
           sphase ^= 1u;
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int32_t u = sched[sslot];
         const int32_t kcount = sched_k[sslot];
-        mbar_arrive(sched_empty + sslot);
+        if (u >= -1 && kcount >= 0) mbar_arrive_relaxed(sched_empty + sslot);
         if (++sslot == kSchedSlots) {
           sslot = 0;
           sphase ^= 1u;
@@ -352,15 +354,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (got) {
           u = sched[sslot];
           kc = sched_k[sslot];
-          if (lead)
-            mbar_arrive(sched_empty + sslot);
-          else
-            mbar_arrive_cluster(cluster_map(smem_u32(sched_empty + sslot), 0));
         }
       }
       got = __shfl_sync(0xffffffffu, got, 0);
       u = __shfl_sync(0xffffffffu, u, 0);
       kc = __shfl_sync(0xffffffffu, kc, 0);
+      if (lane == 0 && got) {   // after the shuffles: the slot's values are in registers
+        if (lead)
+          mbar_arrive_relaxed(sched_empty + sslot);
+        else
+          mbar_arrive_cluster_relaxed(cluster_map(smem_u32(sched_empty + sslot), 0));
+      }
       if (++sslot == kSchedSlots) {
         sslot = 0;
         sphase ^= 1u;
