@@ -408,7 +408,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 bool make_tmap_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-                   uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+                   uint32_t box_inner, uint32_t box_outer, uint32_t swizzle_bytes) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -417,14 +417,16 @@ bool make_tmap_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t ou
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                   : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                         : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
                uint32_t box_outer) {
-  return make_tmap_box(m, base, inner, outer, 64, box_outer, true);
+  return make_tmap_box(m, base, inner, outer, 64, box_outer, 128);
 }
 
 template <int kMode>

@@ -126,9 +126,9 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
 // 128-byte swizzle (the canonical layout tcgen05 descriptors read). ffn_gemm.cu.
 bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
                uint32_t box_outer);
-// The same with any box and no swizzle or the 128-byte one (for TMA stores, no swizzle).
+// The same with any box and a swizzle of 0, 64 or 128 bytes (the span of one swizzled row).
 bool make_tmap_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-                   uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+                   uint32_t box_inner, uint32_t box_outer, uint32_t swizzle_bytes);
 
 // Pair-kernel launch (ffn_gemm_pair.cu): grid = 2 * clusters CTAs, clusters of two.
 // mode 0: SwiGLU epilogue (GEMM A); 1: plain bf16 (GEMM Y, backward A, gate / up

@@ -12,15 +12,15 @@
 // to 64: rows past the live ones must be zero, which zero_pad_rows_kernel ensures for the
 // operands that are not zero there already). Both operands are read MN-major straight from
 // the activations (for A the rows of D are contiguous in memory, for B its columns), TMA
-// boxes of 64 columns x 64 rows: per stage and CTA two of A and four of B (48 KB), 3 stages.
+// boxes of 64 columns x 64 rows: per stage and CTA two of A and four of B (48 KB), 4 stages.
 // The epilogue hands the two accumulators back one at a time; the next unit's MMAs into the
 // first are issued while the second is still being read. (The narrow tiling, 256 columns
 // per unit with one accumulator in two buffers and 5 stages of 32 KB, is kept as the
 // MOE_WGRAD_WIDE=0 build: it draws a third more operand bytes per flop.) In the epilogue
 // each thread holds one row of D (its TMEM lane) and 32 consecutive columns per load; a
-// warp's 32 x 64 share of a unit goes through shared memory (128-byte swizzled) to one TMA
-// store, which writes whole 128-byte row segments (16 epilogue warps; the gradients are
-// 3·E·H·I bf16 values per call). An expert with no rows gets a zero
+// warp's 32 x 64 share of a unit goes through shared memory as two 32 x 32 blocks (64-byte
+// swizzled, 2 KB: small enough to leave room for the 4th stage) to two TMA stores (16
+// epilogue warps; the gradients are 3·E·H·I bf16 values per call). An expert with no rows gets a zero
 // gradient. Waits are bounded as in the forward kernels; a wait that runs out reports
 // MOE_ERR_PIPE_TIMEOUT and raises both CTAs' abort flags.
 #include <mutex>
@@ -41,13 +41,13 @@ constexpr int kThreads = 64 + kEpiWarps * 32;
 constexpr int kSchedSlots = 4;
 constexpr int kSchedReaders = 1 + kEpiWarps + 1 + kEpiWarps;
 constexpr int kBarrierBytes = 256;
-constexpr int kStageOutBytes = 32 * 64 * 2;    // a warp's 32 rows x 64 columns of D
+constexpr int kStageOutBytes = 32 * 32 * 2;    // a warp's 32 rows x 32 columns of D
 constexpr int kOutBytes = kEpiWarps * kStageOutBytes;
 
 // Two tilings of D. Narrow: a unit is 256 x 256 of D, one accumulator of 256 TMEM columns in
 // two buffers (the epilogue of one unit overlaps the MMAs of the next), stages of A and one
 // B half (32 KB), 5 stages. Wide: a unit is 256 x 512 of D, two accumulators (all 512 TMEM
-// columns), stages of A and two B halves (48 KB), 3 stages: each A tile serves twice the
+// columns), stages of A and two B halves (48 KB), 4 stages: each A tile serves twice the
 // MMA work, so the SMs draw 25% fewer operand bytes per flop from L2; the accumulators are
 // handed back one at a time and the next unit's MMAs into the first start meanwhile.
 template <bool kWide>
@@ -55,10 +55,10 @@ struct WgradGeom {
   static constexpr int kAccs = kWide ? 2 : 1;               // accumulators per unit
   static constexpr int kUnitCols = 256 * kAccs;             // columns of D per unit
   static constexpr int kStageBytes = kOpBytes * (1 + kAccs);
-  static constexpr int kStages = kWide ? 3 : 5;
-  static constexpr int kRingBytes = kStages * kStageBytes;  // 160 KB / 144 KB
-  // shared memory: stage ring, then the epilogue's blocks (1024-byte aligned, as the
-  // 128-byte swizzle of their TMA stores wants), then the barriers
+  static constexpr int kStages = kWide ? 4 : 5;
+  static constexpr int kRingBytes = kStages * kStageBytes;  // 192 KB / 160 KB
+  // shared memory: stage ring, then the epilogue's blocks (1024-byte aligned, more than the
+  // 64-byte swizzle of their TMA stores wants), then the barriers
   static constexpr int kSmemBytes = kRingBytes + kOutBytes + kBarrierBytes + 1024;
 };
 static_assert(WgradGeom<true>::kSmemBytes <= 227 * 1024, "shared memory");
@@ -335,9 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------------- epilogue
     // warp w reads TMEM lanes 32 (w % 4) ... (32 rows of D) and columns 64 h ... 64 h + 63,
     // h = (w - 2) / 4, of the unit's 256 columns, 32 at a time: each thread puts its row's
-    // 64 columns into the warp's 32 x 64 block in shared memory, in the 128-byte swizzled
-    // order (16-byte chunk c of row r at c ^ (r % 8), so a warp's stores hit every bank
-    // once), and one thread writes the block to D with a TMA store.
+    // 64 columns, 32 at a time, into the warp's 32 x 32 block in shared memory, in the
+    // 64-byte swizzled order (16-byte chunk c of row r at c ^ ((r / 2) % 4), so each group
+    // of 8 lanes hits every bank once), and one thread writes the block to D with a TMA
+    // store.
     const int quad = warp & 3;
     const int part = (warp - 2) >> 2;
     const uint32_t tq = tmem_base + ((uint32_t)(quad * 32) << 16);
@@ -423,19 +424,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_cluster_relaxed(cluster_map(smem_u32(acc_empty + acc), 0));
         }
         if (store) {
-          // the previous store has read the block
-          if (lane == 0) bulk_wait_group_read<0>();
-          __syncwarp();
-          uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 128);
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            row[c ^ (lane & 7)] =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tm_d, stg, ncol0, e * prm.M + m0);
-            bulk_commit_group();
+          for (int h = 0; h < 2; ++h) {   // the warp's 64 columns as two 32 x 32 blocks
+            if (lane == 0) bulk_wait_group_read<0>();   // the previous store has read the block
+            __syncwarp();
+            uint4 *row = reinterpret_cast<uint4 *>(stg + lane * 64);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              row[c ^ ((lane >> 1) & 3)] =
+                  make_uint4(pk[16 * h + 4 * c], pk[16 * h + 4 * c + 1], pk[16 * h + 4 * c + 2],
+                             pk[16 * h + 4 * c + 3]);
+            fence_proxy_async_shared();   // the block, written by threads, is read by the TMA
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_d, stg, ncol0 + 32 * h, e * prm.M + m0);
+              bulk_commit_group();
+            }
           }
         }
       }
@@ -561,7 +565,7 @@ int launch_wgrad(const moe_shape &s, const void *A, int32_t M, const void *B, in
   CUtensorMap ta, tb, td;
   const uint64_t rows = g.pmax > 0 ? (uint64_t)g.pmax : 1;
   if (!make_tmap(&ta, A, (uint64_t)M, rows, kBK) || !make_tmap(&tb, B, (uint64_t)N, rows, kBK) ||
-      !make_tmap_box(&td, D, (uint64_t)N, (uint64_t)s.E * M, 64, 32, true))
+      !make_tmap_box(&td, D, (uint64_t)N, (uint64_t)s.E * M, 32, 32, 64))
     return MOE_ERR_CUDA;
   if (MOE_WGRAD_WIDE)
     return launch_wgrad_t<true>(s, ta, tb, td, M, N, D, p, sched, cfg, num_sms, st);
